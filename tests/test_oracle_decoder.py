@@ -1,0 +1,171 @@
+"""Pins for oracle.decoder: window independence, speculative-commit invariant, bookkeeping edge cases."""
+
+import numpy as np
+import pytest
+
+from oracle.decoder import ERR_ACCEPTED, ERR_NO_VERIFY, ERR_PENDING, ReplayOracle
+from synth import (GDN_B256, MAMBA2_TINY, accepted_lengths, gdn_draft_inputs, gdn_initial_state,
+                   gdn_step_inputs, mamba2_draft_inputs, mamba2_params, mamba2_step_inputs)
+
+M_WL = MAMBA2_TINY.replace(batch=3, nheads=4, headdim=8, dstate=32, init="normal")
+G_WL = GDN_B256.replace(batch=3, nheads=2, dk=16, dv=8)
+
+
+def _rel(a, b):
+    return np.linalg.norm(a - b) / np.linalg.norm(b)
+
+
+def _mamba(L, **kw):
+    rng = np.random.default_rng(0)
+    S0 = rng.standard_normal((M_WL.batch, M_WL.nheads, M_WL.headdim, M_WL.dstate)) * 0.05
+    return ReplayOracle("mamba2", S0, L, nheads=M_WL.nheads, ngroups=M_WL.ngroups, params=mamba2_params(M_WL), **kw)
+
+
+def _gdn(L, **kw):
+    return ReplayOracle("gdn", gdn_initial_state(G_WL), L, nheads=G_WL.nheads, **kw)
+
+
+@pytest.mark.parametrize("L", [1, 4, 8, 16, 32])
+@pytest.mark.parametrize("kind", ["mamba2", "gdn"])
+def test_window_independence_and_fold_schedule(kind, L):
+    o = _mamba(L) if kind == "mamba2" else _gdn(L)
+    gen = (lambda t: mamba2_step_inputs(M_WL, t)) if kind == "mamba2" else (lambda t: gdn_step_inputs(G_WL, t))
+    for t in range(40):
+        y, y_true = o.step(gen(t))
+        assert _rel(y, y_true) < 2e-6                       # fp32 checkpoint at folds, f64 elsewhere
+        np.testing.assert_array_equal(o.count, (t + 1) % L)
+        np.testing.assert_array_equal(o.epoch, (t + 1) // L)
+    assert o.err is None
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn"])
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_commit_prefix_equals_decoding_prefix(kind, T):
+    """verify(T) + commit(a) then decoding on == decoding only the first a drafts, for every a in 0..T."""
+    L = 8
+    for a in range(T + 1):
+        spec = _mamba(L) if kind == "mamba2" else _gdn(L)
+        plain = _mamba(L) if kind == "mamba2" else _gdn(L)
+        step = (lambda t: mamba2_step_inputs(M_WL, t)) if kind == "mamba2" else (lambda t: gdn_step_inputs(G_WL, t))
+        drafts = mamba2_draft_inputs(M_WL, 0, T) if kind == "mamba2" else gdn_draft_inputs(G_WL, 0, T)
+        for t in range(5):                                  # leave count = 5 so that verify may pre-fold
+            spec.step(step(t))
+            plain.step(step(t))
+        yv, yv_true = spec.verify(T, drafts)
+        spec.commit(np.full(M_WL.batch, a))
+        for j in range(a):
+            one = {k: v[:, j] for k, v in drafts.items()}
+            yp, yp_true = plain.step(one)
+            np.testing.assert_allclose(yv_true[:, j], yp_true, rtol=1e-12, atol=1e-12)
+            assert _rel(yv[:, j], yp) < 2e-6
+        for t in range(5, 25):
+            ys, ys_true = spec.step(step(t))
+            yp, yp_true = plain.step(step(t))
+            np.testing.assert_allclose(ys_true, yp_true, rtol=1e-11, atol=1e-12)
+            assert _rel(ys, yp) < 2e-6
+        np.testing.assert_allclose(spec.S_true, plain.S_true, rtol=1e-11, atol=1e-13)
+        assert spec.err is None
+
+
+def test_verify_prefold_and_commit_to_full_window():
+    L, T = 8, 4
+    o = _mamba(L)
+    for t in range(6):
+        o.step(mamba2_step_inputs(M_WL, t))
+    np.testing.assert_array_equal(o.count, 6)
+    o.verify(T, mamba2_draft_inputs(M_WL, 0, T))            # 6 + 4 > 8: fold the 6 committed records first
+    np.testing.assert_array_equal(o.count, 0)
+    np.testing.assert_array_equal(o.epoch, 1)
+    np.testing.assert_array_equal(o.pending, T)
+    o.commit(np.full(M_WL.batch, T))
+    np.testing.assert_array_equal(o.count, 4)
+    o.verify(T, mamba2_draft_inputs(M_WL, 1, T))            # 4 + 4 == 8: no fold
+    o.commit(np.full(M_WL.batch, T))
+    np.testing.assert_array_equal(o.count, 8)                # a full window after commit, not yet folded
+    np.testing.assert_array_equal(o.epoch, 1)
+    y, y_true = o.step(mamba2_step_inputs(M_WL, 6))          # pre-fold, then append
+    np.testing.assert_array_equal(o.count, 1)
+    np.testing.assert_array_equal(o.epoch, 2)
+    assert _rel(y, y_true) < 2e-6
+
+
+def test_bookkeeping_errors_leave_state_untouched():
+    o = _mamba(8)
+    o.step(mamba2_step_inputs(M_WL, 0))
+    o.commit(np.zeros(M_WL.batch, np.int32))                 # commit without verify
+    assert o.err == (0, ERR_NO_VERIFY)
+    o2 = _gdn(8)
+    o2.verify(4, gdn_draft_inputs(G_WL, 0, 4))
+    y, _ = o2.step(gdn_step_inputs(G_WL, 0))                 # step while verify pending
+    assert o2.err == (0, ERR_PENDING) and np.all(np.isnan(y))
+    np.testing.assert_array_equal(o2.count, 0)
+    o2.flush()
+    np.testing.assert_array_equal(o2.count, 0)
+    o2.commit(np.array([1, 7, 2]))                           # sequence 1 asks for more than T
+    np.testing.assert_array_equal(o2.count, [1, 0, 2])
+    np.testing.assert_array_equal(o2.pending, [0, 4, 0])
+    assert o2.err == (0, ERR_PENDING)                        # lowest failing sequence is kept
+    o3 = _gdn(8)
+    o3.verify(2, gdn_draft_inputs(G_WL, 0, 2))
+    o3.commit(np.array([0, 3, 1]))
+    assert o3.err == (1, ERR_ACCEPTED)
+
+
+def test_flush_masks_and_random_speculation():
+    """A long random verify/commit/step/flush schedule keeps the truth-side invariant."""
+    L, T = 16, 4
+    o = _mamba(L)
+    step_t, rnd = 0, 0
+    rng = np.random.default_rng(3)
+    for it in range(30):
+        op = rng.integers(0, 3)
+        if op == 0:
+            o.step(mamba2_step_inputs(M_WL, step_t)); step_t += 1
+        elif op == 1:
+            y, y_true = o.verify(T, mamba2_draft_inputs(M_WL, rnd, T))
+            assert _rel(y, y_true) < 2e-6
+            o.commit(accepted_lengths(M_WL, rnd, T)); rnd += 1
+        else:
+            mask = rng.integers(0, 2, M_WL.batch).astype(bool)
+            before = o.count.copy()
+            o.flush(mask)
+            np.testing.assert_array_equal(o.count, np.where(mask, 0, before))
+        assert np.all(o.count <= L) and o.err is None
+
+
+@pytest.mark.parametrize("kind", ["mamba2", "gdn"])
+def test_read_copy_never_reenters_recurrence(kind):
+    """Separate precision: the checkpoint and fold-step outputs are those of the fp32 run, bit for bit."""
+    L = 4
+    ref = _mamba(L) if kind == "mamba2" else _gdn(L)
+    sep = _mamba(L, read="nvfp4") if kind == "mamba2" else _gdn(L, read="nvfp4")
+    shared = _mamba(L, read="shared_nvfp4") if kind == "mamba2" else _gdn(L, read="shared_nvfp4")
+    gen = (lambda t: mamba2_step_inputs(M_WL, t)) if kind == "mamba2" else (lambda t: gdn_step_inputs(G_WL, t))
+    err_sep = []
+    for t in range(24):
+        inp = gen(t)
+        y_ref, y_true = ref.step(inp)
+        y_sep, _ = sep.step(inp)
+        shared.step(inp)
+        np.testing.assert_array_equal(sep.hp, ref.hp)
+        if (t + 1) % L == 0:
+            np.testing.assert_array_equal(y_sep, y_ref)     # fold step: full-precision state
+        else:
+            err_sep.append(_rel(y_sep, y_true))
+        np.testing.assert_array_equal(shared.hp, shared.rd)
+    assert 0 < max(err_sep) < 0.2
+
+
+def test_fp16_checkpoint_is_on_the_fp16_grid():
+    o = _gdn(4, hp="f16sr", seed=123)
+    for t in range(8):
+        o.step(gdn_step_inputs(G_WL, t))
+    np.testing.assert_array_equal(o.hp.astype(np.float16).astype(np.float64), o.hp)
+    # same seed, same words: deterministic; different seed: different roundings
+    o2 = _gdn(4, hp="f16sr", seed=123)
+    o3 = _gdn(4, hp="f16sr", seed=124)
+    for t in range(8):
+        o2.step(gdn_step_inputs(G_WL, t))
+        o3.step(gdn_step_inputs(G_WL, t))
+    np.testing.assert_array_equal(o.hp, o2.hp)
+    assert np.any(o.hp != o3.hp)

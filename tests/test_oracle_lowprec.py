@@ -1,0 +1,189 @@
+"""Pins for oracle.lowprec and oracle.philox: library conversions, exhaustive grids, thresholds, published vectors."""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lowprec as lp
+from oracle.philox import philox4x32_10, sr_words
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------- Philox
+
+def test_philox_known_answer_vectors():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")) if l.strip() and l[0] != "#"]
+    assert len(rows) == 3
+    for row in rows:
+        v = [int(w, 16) for w in row]
+        out = philox4x32_10(*v[:4], v[4], v[5])
+        assert [int(w) for w in out] == v[6:]
+
+
+def test_sr_words_layout():
+    w = sr_words(0x1234567890ABCDEF, 5, 3, 10)
+    ref = philox4x32_10([5, 5, 5], [3, 3, 3], [0, 1, 2], 0, 0x90ABCDEF, 0x12345678)
+    flat = np.stack(ref, axis=-1).reshape(-1)[:10]
+    np.testing.assert_array_equal(w, flat)
+
+
+# ----------------------------------------------------------------------------- FP16 stochastic rounding
+
+def _all_finite_fp16():
+    v = np.arange(0, 0x10000, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    return v[np.isfinite(v)]
+
+
+def test_sr_grid_points_unchanged():
+    v = _all_finite_fp16().astype(np.float32)
+    for r in (0, 1, 0x80000000, 0xFFFFFFFF):
+        out = lp.fp16_stochastic_round(v, np.full(v.shape, r, np.uint32))
+        np.testing.assert_array_equal(out.view(np.uint16), v.astype(np.float16).view(np.uint16))
+
+
+def _neighbours(x):
+    """fp16 values just below and above |x| (toward and away from zero), from numpy's float16."""
+    a = np.abs(x).astype(np.float32)
+    rn = a.astype(np.float16)
+    lo = np.where(rn.astype(np.float32) <= a, rn, np.nextafter(rn, np.float16(0)))
+    hi = np.where(rn.astype(np.float32) >= a, rn, np.nextafter(rn, np.float16(np.inf)))
+    return lo, hi
+
+
+def test_sr_extreme_words_truncate_or_round_away():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.uniform(-9, 4, 20000)]).astype(np.float32)
+    x = x[np.abs(x) < 65504]
+    lo, hi = _neighbours(x)
+    down = lp.fp16_stochastic_round(x, np.full(x.shape, 0xFFFFFFFF, np.uint32))
+    up = lp.fp16_stochastic_round(x, np.zeros(x.shape, np.uint32))
+    np.testing.assert_array_equal(np.abs(down), lo)                # largest word: always toward zero
+    np.testing.assert_array_equal(np.abs(up), hi)                  # zero word: away from zero unless exact
+    assert np.all(np.signbit(down) == np.signbit(x))
+
+
+def test_sr_threshold_is_exact_fraction():
+    # x = (q + k/8) ulp rounds up exactly for r < k * 2^29, in the normal and the subnormal range
+    for base, ulp in ((1.0, 2.0 ** -10), (2.0 ** -20, 2.0 ** -24), (300.0, 0.25)):
+        for k in range(1, 8):
+            x = np.float32(base + k / 8 * ulp)
+            thr = k << 29
+            r = np.array([thr - 1, thr, 0, 0xFFFFFFFF], np.uint32)
+            out = lp.fp16_stochastic_round(np.full(4, x), r).astype(np.float64)
+            assert out[0] == base + ulp and out[2] == base + ulp
+            assert out[1] == base and out[3] == base
+
+
+def test_sr_unbiased_over_all_words():
+    # averaging over r = 0, 2^16, 2*2^16, ... reproduces x to within ulp * 2^-16
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal(64) * 10.0 ** rng.uniform(-6, 3, 64)).astype(np.float32)
+    r = (np.arange(65536, dtype=np.uint64) << np.uint64(16)).astype(np.uint32)
+    for xi in x:
+        out = lp.fp16_stochastic_round(np.full(r.shape, xi), r).astype(np.float64)
+        _, hi = _neighbours(np.array([xi]))
+        lo, _ = _neighbours(np.array([xi]))
+        ulp = float(hi[0]) - float(lo[0]) or 2.0 ** -24
+        assert abs(out.mean() - float(xi)) <= ulp * 2.0 ** -16 * 1.0001
+
+
+def test_sr_saturation_and_sign():
+    x = np.array([70000.0, -1e9, 65519.0, -65519.0, 0.0, -0.0], np.float32)
+    out = lp.fp16_stochastic_round(x, np.zeros(6, np.uint32)).astype(np.float64)
+    np.testing.assert_array_equal(out[:4], [65504.0, -65504.0, 65504.0, -65504.0])
+    assert out[4] == 0 and not np.signbit(out[4]) and np.signbit(out[5])
+    rng = np.random.default_rng(4)
+    xs = rng.standard_normal(1000).astype(np.float32)
+    r = rng.integers(0, 2 ** 32, 1000, dtype=np.uint64).astype(np.uint32)
+    np.testing.assert_array_equal(lp.fp16_stochastic_round(-xs, r), -lp.fp16_stochastic_round(xs, r))
+
+
+# ----------------------------------------------------------------------------- E4M3 / E2M1
+
+def test_e4m3_matches_torch_below_saturation():
+    rng = np.random.default_rng(5)
+    codes = np.arange(0, 0x7F, dtype=np.int64)                      # every finite non-negative code
+    grid = lp.e4m3_value(codes)
+    mids = (grid[:-1] + grid[1:]) / 2                                # ties
+    vals = np.concatenate([grid, mids, rng.uniform(0, 448, 20000), rng.uniform(0, 2 ** -6, 5000)])
+    vals = vals.astype(np.float32)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn)
+    ours = lp.e4m3_round(vals)
+    np.testing.assert_array_equal(ours, ref.float().numpy().astype(np.float64))
+    np.testing.assert_array_equal(lp.e4m3_code(ours), ref.view(torch.uint8).numpy())
+    np.testing.assert_array_equal(lp.e4m3_value(lp.e4m3_code(grid)), grid)
+
+
+def test_e4m3_saturates():
+    np.testing.assert_array_equal(lp.e4m3_round(np.array([448.0, 460.0, 470.0, 1e6])), [448.0] * 4)
+
+
+def _e2m1_bruteforce(y):
+    """Nearest of {0, .5, 1, 1.5, 2, 3, 4, 6}; on a tie the even index wins; beyond 6 -> 6."""
+    a = abs(float(y))
+    if a >= 6.0:
+        return 7
+    best = None
+    for i, g in enumerate(lp.E2M1_VALUES):
+        d = abs(a - g)
+        if best is None or d < best[0] or (d == best[0] and i % 2 == 0):
+            best = (d, i)
+    return best[1]
+
+
+def test_e2m1_against_bruteforce():
+    g = lp.E2M1_VALUES
+    pts = np.concatenate([g, (g[:-1] + g[1:]) / 2, np.linspace(0, 8, 4001), [6.5, 7.0, 100.0]])
+    pts = np.concatenate([pts, -pts, np.nextafter(pts, 10), np.nextafter(pts, -10)])
+    ours = lp.e2m1_magnitude_code(pts)
+    ref = np.array([_e2m1_bruteforce(p) for p in pts])
+    np.testing.assert_array_equal(ours, ref)
+
+
+# ----------------------------------------------------------------------------- NVFP4 read copy
+
+def test_nvfp4_grid_tile_roundtrips_exactly():
+    rng = np.random.default_rng(6)
+    R, C = 8, 64
+    g = np.float32(2.0 ** -10)
+    s_grid = lp.e4m3_value(np.arange(8, 0x7F))                     # normal e4m3 scales, up to 448
+    s_b = rng.choice(s_grid, (R, C // 16))
+    s_b[0, 0] = 448.0                                                # tile amax = 6 * 448 * g
+    vals = rng.choice(lp.E2M1_VALUES, (R, C // 16, 16)) * rng.choice([-1, 1], (R, C // 16, 16))
+    vals[..., 0] = 6.0                                               # every block reaches its amax
+    tile = (vals * (s_b * g)[..., None]).reshape(R, C).astype(np.float32)
+    q = lp.nvfp4_quantize(tile)
+    assert q["g"] == g
+    np.testing.assert_array_equal(lp.e4m3_value(q["scales"]), s_b)
+    np.testing.assert_array_equal(lp.nvfp4_dequantize(q["codes"], q["scales"], q["g"]), tile)
+
+
+def test_nvfp4_zero_tile_and_packing():
+    q = lp.nvfp4_quantize(np.zeros((2, 4, 32), np.float32))
+    assert np.all(q["codes"] == 0) and np.all(q["g"] == 1.0) and np.all(q["scales"] == 0)
+    rng = np.random.default_rng(7)
+    t = rng.standard_normal((3, 4, 32)).astype(np.float32)
+    q = lp.nvfp4_quantize(t)
+    np.testing.assert_array_equal(q["packed"] & 0xF, q["codes"][..., 0::2])
+    np.testing.assert_array_equal(q["packed"] >> 4, q["codes"][..., 1::2])
+    assert q["codes"].max() <= 15
+
+
+def test_nvfp4_error_bound_and_scale_choice():
+    rng = np.random.default_rng(8)
+    t = (rng.standard_normal((16, 64, 128)) * 10.0 ** rng.uniform(-3, 2, (16, 1, 1))).astype(np.float32)
+    q = lp.nvfp4_quantize(t)
+    d = lp.nvfp4_dequantize(q["codes"], q["scales"], q["g"])
+    blocks = np.abs(t).reshape(16, 64, 8, 16)
+    amax_b = blocks.max(-1, keepdims=True)
+    err = np.abs(d - t).reshape(blocks.shape)
+    # per element: half an E2M1 step at the top of the range (1 of 6) plus the E4M3 scale rounding (1/16)
+    assert np.all(err <= amax_b * (1 / 6 + 1 / 16) * 1.01 + 1e-30)
+    # the tile scale maps the tile maximum to 6 * 448
+    np.testing.assert_allclose(q["g"], np.abs(t).reshape(16, -1).max(-1) / 2688.0, rtol=1e-7)
+    # each block maximum lands within a scale step of code 6 (i.e. value 6 after rounding)
+    top = lp.E2M1_VALUES[(q["codes"] & 7).reshape(blocks.shape).max(-1)]
+    assert np.all(top[amax_b[..., 0] > 1e-4 * np.abs(t).max()] >= 4.0)
