@@ -1,0 +1,356 @@
+"""Benchmark: ReplaySSM Mamba-2 decode on B200, batch 256, L = 16 (the 120B-class layer).
+
+One step = one decode token for every sequence of the layer (batch 256, 128
+heads, P 64, N 128, 8 groups, bf16 inputs, fp32 checkpoint of 1 GiB), i.e. one
+launch of the replay kernel; every 16th step folds the window into a new
+checkpoint.  The timed region is whole steps on the device with the inputs
+already resident (a pool of distinct seeded token inputs, cycled); the
+checkpoint stream (1 GiB per step) is larger than L2, so no flush is needed.
+
+Printed (one JSON line, rank 0): tokens/s of replay decode, the conventional
+step-by-step kernel on the same layer (reads and writes the state every token)
+for comparison, the roofline of the replay kernel against the measured HBM
+bandwidth, an end-to-end number through the public API with host buffers, and
+the CPU oracle timed on a bounded sample.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {rssm,reference}]
+Multi-GPU (weak scaling, independent replicas, no collective on the data path):
+  python -m torch.distributed.run --nproc-per-node N --master-addr 127.0.0.1 bench.py --gpus N
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import MAMBA2_120B, mamba2_initial_state, mamba2_params, mamba2_step_inputs  # noqa: E402
+
+WL = MAMBA2_120B
+METRIC = "SSM decode tokens/s & achieved HBM GB/s at B=256, L=16 vs step-by-step kernel"
+POOL = 32  # distinct token inputs cycled through the timed region
+
+
+def traffic_model(wl, count_before: int) -> dict:
+    """Algorithmic HBM bytes of one replay step whose sequences hold ``count_before`` records.
+
+    checkpoint read + checkpoint write (fold steps only) + buffered records read +
+    token inputs read + record appended + fp32 output written.
+    """
+    Bt, H, P, N, G, L = wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window
+    esz = 2 if wl.in_dtype == "bf16" else 4
+    state = Bt * H * P * N * 4
+    rec = Bt * (H * P * esz + G * N * esz + H * 4)          # one record in the ring (x, B, dt as fp32)
+    tok = Bt * (H * P * esz + 2 * G * N * esz + H * esz)     # x, B, C, dt of the token
+    fold = count_before + 1 == L
+    return {"state_read": state, "state_write": state if fold else 0, "ring_read": count_before * rec,
+            "inputs": tok, "append": rec, "y": Bt * H * P * 4}
+
+
+def conventional_bytes(wl) -> int:
+    Bt, H, P, N, G = wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    esz = 2 if wl.in_dtype == "bf16" else 4
+    return 2 * Bt * H * P * N * 4 + Bt * (H * P * esz + 2 * G * N * esz + H * esz) + Bt * H * P * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle (baseline leg)
+
+class OracleArm:
+    """The float64 oracle, as it stands, decoding ``nseq`` sequences (all heads) of the workload on one host thread."""
+
+    def __init__(self, nseq: int):
+        from oracle.decoder import ReplayOracle
+        self.seqs = list(range(nseq))
+        S0 = mamba2_initial_state(WL, seqs=self.seqs)
+        self.inputs = [{k: v[self.seqs] for k, v in mamba2_step_inputs(WL, t).items()} for t in range(4)]
+        self.orc = ReplayOracle("mamba2", S0, WL.window, nheads=WL.nheads, ngroups=WL.ngroups,
+                                params=mamba2_params(WL))
+        self.i = 0
+
+    def step(self):
+        self.orc.step(self.inputs[self.i % len(self.inputs)])
+        self.i += 1
+
+
+def _limits():
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(1)
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    """Oracle tokens/s on a bounded sample: 4 sequences x all heads, whole decode steps for ~budget_s."""
+    with _limits():
+        arm = OracleArm(4)
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget_s:
+            arm.step()
+        dt = time.perf_counter() - t0
+    return {"value": len(arm.seqs) * arm.i / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(arm.seqs)} of {WL.batch} sequences x all {WL.nheads} heads, {arm.i} decode steps "
+                      f"(float64 step-by-step + replay bookkeeping), {dt:.1f} s on 1 host thread"}
+
+
+def reference_arm(args) -> dict:
+    """--impl reference: the oracle timed per step on a bounded sample sized so the run takes ~2 minutes."""
+    with _limits():
+        probe = OracleArm(1)
+        t0 = time.perf_counter()
+        for _ in range(3):
+            probe.step()
+        per_seq_step = (time.perf_counter() - t0) / 3
+        nseq = int(max(1, min(WL.batch, 120.0 / ((args.steps + args.warmup) * per_seq_step))))
+        arm = OracleArm(nseq)
+        for _ in range(args.warmup):
+            arm.step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            arm.step()
+        dt = time.perf_counter() - t0
+    v = nseq * args.steps / dt
+    cb = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+          "sample": f"{nseq} of {WL.batch} sequences x all {WL.nheads} heads per step, {args.steps} steps, "
+                    f"{dt:.1f} s on 1 host thread"}
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "mamba2 replay decode, batch 256, 128 heads, P 64, N 128, 8 groups, L 16 "
+                                   "(oracle: sampled sequences per step)"},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, rank, world):
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM, conv_mamba2_step, make_config
+    torch.cuda.set_device(rank % torch.cuda.device_count())
+    dev = torch.device("cuda")
+    bf = torch.bfloat16
+    p = mamba2_params(WL)
+    A = torch.from_numpy(p["A"]).to(dev)
+    D = torch.from_numpy(p["D"]).to(dev)
+    layer = ReplaySSM("mamba2", WL.batch, WL.nheads, WL.headdim, WL.dstate, WL.ngroups, WL.window, 0, bf,
+                      A=A, D=D)
+    S0 = torch.from_numpy(mamba2_initial_state(WL)).to(dev)
+    layer.load_checkpoint(S0)
+    host_pool = [mamba2_step_inputs(WL.replace(seed=WL.seed + 1000 * rank), t) for t in range(POOL)]
+    pool = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in inp.items()} for inp in host_pool]
+    y = torch.empty(WL.batch, WL.nheads, WL.headdim, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        t = pool[i % POOL]
+        layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], y)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # the timed region starts at a window boundary so that the fold count is exact
+    count0 = args.warmup % WL.window
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev[0].record(stream)
+        for i in range(K):
+            step(args.warmup + i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    total_ms = ev[0].elapsed_time(ev[K])
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    model = [traffic_model(WL, (count0 + i) % WL.window) for i in range(K)]
+    bytes_avg = sum(sum(m.values()) for m in model) / K
+    step_ms = total_ms / K
+    mean_launch_ms = sum(per) / K
+    hbm_peak, peak_kind = load_peaks()
+    achieved = bytes_avg / (mean_launch_ms * 1e-3) / 1e9
+    fold_ms = [d for d, m in zip(per, model) if m["state_write"]]
+    plain_ms = [d for d, m in zip(per, model) if not m["state_write"]]
+    err = layer.get_error()
+
+    # conventional step-by-step kernel on the same layer (comparison)
+    cfg = make_config("mamba2", WL.batch, WL.nheads, WL.headdim, WL.dstate, WL.ngroups, WL.window, 0, bf, A=A, D=D)
+    S = S0.clone()
+    Kc = max(16, K // 4)
+    for i in range(8):
+        t = pool[i % POOL]
+        conv_mamba2_step(cfg, S, t["x"], t["B"], t["C"], t["dt"], y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(Kc):
+        t = pool[i % POOL]
+        conv_mamba2_step(cfg, S, t["x"], t["B"], t["C"], t["dt"], y)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    conv_ms = e0.elapsed_time(e1) / Kc
+    del S
+
+    # end to end through the public API: pinned host inputs in, output back to pinned host memory
+    pinned = [{k: torch.from_numpy(v).to(bf).pin_memory() for k, v in inp.items()} for inp in host_pool[:8]]
+    y_host = torch.empty(WL.batch, WL.nheads, WL.headdim, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned[0].values())
+    d2h = y_host.numel() * 4
+    Ke = max(16, K // 4)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(Ke):
+        src = pinned[i % len(pinned)]
+        t = {k: v.to(dev, non_blocking=True) for k, v in src.items()}
+        layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], y)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([e2e_ms, conv_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms, conv_ms = float(tt[0].item()), float(tt[1].item())
+
+    tokens = WL.batch * world
+    res = {
+        "metric": METRIC, "value": tokens * K / (total_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; bf16 token inputs, fp32 checkpoint)",
+        "config": {"workload": "mamba2 replay decode, batch 256 per GPU, 128 heads, P 64, N 128, 8 groups, L 16, "
+                               "bf16 inputs, fp32 checkpoint 1 GiB", "batch_per_gpu": WL.batch,
+                   "global_batch": WL.batch * world, "nheads": WL.nheads, "headdim": WL.headdim,
+                   "dstate": WL.dstate, "ngroups": WL.ngroups, "window": WL.window,
+                   "parallelism": f"replicas x{world} (batch shards, no collective)",
+                   "l2": "checkpoint stream (1 GiB/step) exceeds L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": None,
+                     "kernel": "m2_replay_kernel", "bytes_per_launch": bytes_avg,
+                     "mean_launch_ms": mean_launch_ms,
+                     "fold_launch_ms": statistics.mean(fold_ms) if fold_ms else None,
+                     "plain_launch_ms": statistics.median(plain_ms) if plain_ms else None},
+        "comparison": {"conventional_tokens_per_s": tokens / (conv_ms * 1e-3), "conventional_ms_per_step": conv_ms,
+                       "conventional_bytes_per_step": conventional_bytes(WL),
+                       "conventional_GBps": conventional_bytes(WL) / (conv_ms * 1e-3) / 1e9,
+                       "replay_speedup": conv_ms / step_ms},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": K,
+        "clocks": clk.summary(),
+        "device_error": err,
+    }
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=64)
+    ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        # the reference arm is the CPU oracle, on rank 0 only; other ranks exit without work
+        if rank == 0:
+            print(json.dumps(reference_arm(args)))
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_gpu(args, rank, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

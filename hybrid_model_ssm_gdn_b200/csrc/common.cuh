@@ -1,0 +1,216 @@
+// common.cuh -- device helpers shared by the ReplaySSM kernels (sm_100a).
+//
+// * mbarrier + cp.async.bulk (TMA bulk copy, global -> shared) primitives used by
+//   the persistent streaming kernels: one producer warp issues bulk copies of a
+//   head's checkpoint tile and its buffered inputs into a shared-memory stage,
+//   consumer warps wait on the stage's "full" barrier and release it through an
+//   "empty" barrier.  Every wait is bounded: after ~1 s of polling it records
+//   RSSM_DEV_TIMEOUT in the context's error word and the kernel winds down.
+// * warp-level transpose reduction: each lane holds V partial sums; after
+//   log2(32) exchange levels every value has been summed over the 32 lanes and
+//   each lane keeps max(V/32, 1) of them (lane l keeps indices l*V/32 + i).
+// * arena layout shared by the host API and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rssm.h"
+
+namespace rssm {
+
+constexpr int kCols = 128;           // contiguous state axis (N or d_k)
+constexpr int kMaxWindow = 32;
+constexpr int kMaxDraft = 8;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;  // + one producer warp
+constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at B200 clocks
+
+// error word: min over (seq * 16 + code); 0x7fffffff = clean
+constexpr int kErrClean = 0x7fffffff;
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ inline int dt_stride(int L) { return (int)align_up((size_t)(2 * L), 4); }  // fp32 slots per ring row
+
+// Byte offsets of the regions of a context's arena.
+struct ArenaLayout {
+  size_t meta;     // int4 [2][Bt]: count, epoch, pending, 0  (ping-pong by call parity)
+  size_t err;      // int [1]
+  size_t hp;       // checkpoint: fp32 or fp16 [Bt][H][R][128]
+  size_t rq;       // NVFP4 codes u8 [Bt][H][R][64]
+  size_t rs;       // NVFP4 block scales u8 [Bt][H][R][8]
+  size_t rg;       // NVFP4 tile scale fp32 [Bt][H]
+  size_t ring_a;   // Mamba-2 x [Bt][H][2L][P] / GDN k [Bt][H][2L][128]   (input dtype)
+  size_t ring_b;   // Mamba-2 B [Bt][G][2L][128] / GDN v [Bt][H][2L][d_v] (input dtype)
+  size_t ring_c;   // Mamba-2 dt / GDN alpha: fp32 [Bt][H][dt_stride(L)]
+  size_t ring_d;   // GDN beta: fp32 [Bt][H][dt_stride(L)]
+  size_t total;
+};
+
+inline ArenaLayout make_layout(const rssm_config &c) {
+  ArenaLayout a{};
+  const size_t Bt = c.batch, H = c.nheads, R = c.headdim, L = c.window;
+  const size_t esz = c.in_dtype == RSSM_BF16 ? 2 : 4;
+  const size_t units = Bt * H;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  a.meta = take(2 * Bt * 16);
+  a.err = take(16);
+  const bool shared_fp4 = c.read == RSSM_READ_SHARED_NVFP4;
+  a.hp = take(shared_fp4 ? 0 : units * R * kCols * (c.hp == RSSM_HP_F16_SR ? 2 : 4));
+  const bool fp4 = c.read != RSSM_READ_SAME;
+  a.rq = take(fp4 ? units * R * kCols / 2 : 0);
+  a.rs = take(fp4 ? units * R * kCols / 16 : 0);
+  a.rg = take(fp4 ? units * 4 : 0);
+  if (c.kind == RSSM_MAMBA2) {
+    a.ring_a = take(units * 2 * L * R * esz);
+    a.ring_b = take(Bt * c.ngroups * 2 * L * kCols * esz);
+    a.ring_c = take(units * dt_stride(c.window) * 4);
+    a.ring_d = take(0);
+  } else {
+    a.ring_a = take(units * 2 * L * kCols * esz);
+    a.ring_b = take(units * 2 * L * R * esz);
+    a.ring_c = take(units * dt_stride(c.window) * 4);
+    a.ring_d = take(units * dt_stride(c.window) * 4);
+  }
+  a.total = off;
+  return a;
+}
+
+// ------------------------------------------------------------------------------------------
+// loads / conversions
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// 4 consecutive elements starting at p (16-byte aligned for float, 8-byte for bf16)
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+  uint2 u = *reinterpret_cast<const uint2 *>(p);
+  float4 r;
+  r.x = __uint_as_float(u.x << 16);
+  r.y = __uint_as_float(u.x & 0xffff0000u);
+  r.z = __uint_as_float(u.y << 16);
+  r.w = __uint_as_float(u.y & 0xffff0000u);
+  return r;
+}
+
+__device__ __forceinline__ void record_error(int *err, int seq, int code) { atomicMin(err, seq * 16 + code); }
+
+// ------------------------------------------------------------------------------------------
+// mbarrier / bulk copy
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+
+// Bounded wait that also gives up as soon as another warp of the block has flagged an abort.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// global -> shared bulk copy completing on an mbarrier; dst, src 16-byte aligned, bytes % 16 == 0
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// consumer-only named barrier (the producer warp does not take part)
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
+
+// ------------------------------------------------------------------------------------------
+// warp reductions
+
+template <int V>
+__device__ __forceinline__ void warp_transpose_reduce(float (&v)[V], int lane) {
+  int cur = V;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (cur > 1) {
+      const int half = cur / 2;
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < V / 2; ++i) {
+        if (i < half) {
+          float send = upper ? v[i] : v[i + half];
+          float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      cur = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+}  // namespace rssm

@@ -36,7 +36,8 @@ Readings taken where the pages are silent (per sequence; L = window):
   state that forbids it (step, verify or flush with a verify pending; commit
   without one; accepted length out of range) leaves that sequence untouched,
   writes none of its outputs, and records an error: the error word keeps the
-  lowest sequence index that ever failed, with its code.
+  lowest sequence index that ever failed, with its code (the lowest code if
+  that sequence failed in several ways).
 * Outputs of a call that folds come from the freshly folded state at full
   precision; the stored checkpoint is read for folding, the read copy for
   outputs of calls that do not fold.
@@ -163,7 +164,7 @@ class ReplayOracle:
 
     def _error(self, b, code):
         s = int(self.seq_ids[b])
-        if self.err is None or s < self.err[0]:
+        if self.err is None or (s, code) < self.err:
             self.err = (s, code)
 
     # ------------------------------------------------------------------ calls
