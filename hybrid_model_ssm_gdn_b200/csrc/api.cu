@@ -78,12 +78,11 @@ rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, c
   M2Args a{};
   a.Bt = c.batch; a.H = c.nheads; a.P = c.headdim; a.G = c.ngroups; a.L = c.window;
   a.T = T; a.tmax = op == OP_VERIFY ? T : 1; a.op = op;
-  a.units = c.batch * c.nheads;
+  a.units = m2_units(c.batch, c.nheads, c.ngroups);
   a.grid = a.units < x->num_sms ? a.units : x->num_sms;
-  const int esz = esize(c), no = pow2_outputs(a.tmax);
-  const int sb = m2_stage_bytes(a.P, a.L, a.tmax, esz, no);
-  a.nstage = pick_stages(x, sb, m2_table_bytes(a.P, a.L, a.tmax, no));
-  if (16 * a.nstage + m2_table_bytes(a.P, a.L, a.tmax, no) + a.nstage * sb > x->smem_optin) return RSSM_ERR_SHAPE;
+  const int esz = esize(c);
+  a.nstage = x->nstage_override > 0 ? x->nstage_override : m2_max_stages(a.P, a.L, a.tmax, esz, x->smem_optin - 1024);
+  if (a.nstage < 2 || a.nstage > 8 || m2_smem_bytes(a.P, a.L, a.tmax, esz, a.nstage) > x->smem_optin) return RSSM_ERR_SHAPE;
   a.meta_in = meta_cur(x); a.meta_out = meta_next(x); a.err = err_word(x);
   a.hp = reinterpret_cast<float *>(x->arena + x->lay.hp);
   a.ring_x = x->arena + x->lay.ring_a; a.ring_B = x->arena + x->lay.ring_b;

@@ -26,8 +26,9 @@ struct M2Args {
   const float *A, *D;
   float *y;                       // [Bt][T][H][P]
 };
-int m2_stage_bytes(int P, int L, int tmax, int esz, int no);
-int m2_table_bytes(int P, int L, int tmax, int no);
+int m2_smem_bytes(int P, int L, int tmax, int esz, int nstage);
+int m2_max_stages(int P, int L, int tmax, int esz, int smem_budget);
+int m2_units(int Bt, int H, int G);  // work units: (sequence, group chunk of <= 16 heads)
 cudaError_t launch_m2_replay(M2Args a, int esz, cudaStream_t stream);
 
 // Gated DeltaNet replay kernel (step / verify / flush) with the precision modes.

@@ -4,25 +4,31 @@
 // Per (sequence b, head h) the state is a fp32 checkpoint S0 in R^{P x 128} plus the
 // inputs (x, B, dt) of the tokens since it, kept in a ring in HBM ("SSM decoding stops
 // writing state every step", Synopsis and Interpretation, second paragraph).  For a
-// call, the records of one unit are laid out as r = 0..n_rec-1 (buffered records in
+// call, the records of a sequence are laid out as r = 0..n_rec-1 (buffered records in
 // token order, then the call's new tokens); the first m of them are folded into the
-// state and every output j replays records m..e_j-1 against the (possibly folded)
-// state.  Unrolling the Mamba-2 recurrence S_t = exp(dt_t A) S_{t-1} + dt_t x_t B_t^T,
-// y_t = S_t C_t + D x_t gives, with s(a, b) = sum_{a<=l<b} dt_l,
+// state and output j replays records m..e_j-1 against the (possibly folded) state.
+// Unrolling S_t = exp(dt_t A) S_{t-1} + dt_t x_t B_t^T, y_t = S_t C_t + D x_t gives,
+// with s(a, b) = sum_{a<=l<b} dt_l,
 //
 //   fold:   S' = exp(A s(0,m)) S0 + sum_{r<m} dt_r exp(A s(r+1,m)) x_r B_r^T
 //   output: y_j = exp(A s(m,e_j)) S' C_j
 //               + sum_{m<=r<e_j} dt_r exp(A s(r+1,e_j)) (B_r . C_j) x_r + D x_{e_j - 1}
 //
-// (the products of exp(dt A) are taken in log space).  Only a fold writes the state;
-// a plain step reads the checkpoint once and writes its output and its input record.
+// (products of exp(dt A) taken in log space).  Only a fold writes the state; a plain
+// step reads the checkpoint once and writes its output and its input record.
 //
-// Data movement: a producer warp reads the bookkeeping word of the unit's sequence,
-// decides the call's schedule (pre-fold / eager fold / error) and issues TMA bulk
-// copies (cp.async.bulk, evict-first for the checkpoint stream) of the checkpoint tile,
-// the buffered records and the new tokens into a shared-memory stage.  Eight consumer
-// warps compute: warp w owns rows 8w..8w+7 of the tile, lane l owns columns 4l..4l+3,
-// the row dot products with C are finished by a warp transpose reduction.
+// Work unit: (sequence, group of <= 16 heads sharing B and C).  Warp roles in a block:
+//  * producer warp: issues TMA bulk copies (cp.async.bulk; evict-first for the
+//    checkpoint stream) into a double-buffered group buffer (B, C and dt rows of the
+//    unit) and into a ring of tile stages (one head's checkpoint tile + its x records);
+//  * prep warp: one unit ahead of the consumers, computes from the group buffer the
+//    dot products B_r . C_j and every head's decay weights into double-buffered tables,
+//    appends the group's B records and writes the sequence's bookkeeping word;
+//  * eight consumer warps: warp w owns rows 8w..8w+7 of every tile, lane l columns
+//    4l..4l+3; a warp waits on the stage's full barrier, computes its rows (fold, dot
+//    products, transpose reduction, buffered part of y) and releases the stage on its
+//    own.  No block-wide barrier sits on the streaming path, so one block per SM keeps
+//    the checkpoint stream in flight while the next unit is being prepared.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,87 +36,117 @@ namespace rssm {
 
 namespace {
 
-// header ints / floats at the start of each stage
+constexpr int kHG = 16;          // heads per unit (a group is split into chunks of <= 16)
+constexpr int kGHdr = 1024;      // group header bytes
+
+// group header: ints then floats
 enum {
-  H_FLAGS = 0,   // bit0 compute, bit1 state is written (m > 0), bit2 this unit writes the meta word
-  H_NREC,        // records in the stage
-  H_M,           // records folded into the state
-  H_NRING,       // records taken from the ring (slots base_e + 0..n_ring-1)
-  H_NNEW,        // new tokens of this call (appended)
-  H_TOUT,        // outputs
-  H_SLOT0,       // absolute ring slot of the first appended token
-  H_MC, H_ME, H_MP,  // meta to write: count, epoch, pending
-  H_B, H_H,
-  H_BASE,        // absolute ring slot of buffered record 0 (window base before the call)
-  H_F = 16       // floats from here: dt of new tokens [8], A, D
-};
-constexpr int kHdrBytes = 256;
-
-struct M2Stage {
-  int tile, xr, br, cr, dtr, bytes;
+  G_ACTIVE = 0, G_NREC, G_M, G_NRING, G_NNEW, G_TOUT, G_SLOT0, G_MC, G_ME, G_MP, G_B, G_G, G_H0, G_NH,
+  G_BASE, G_WMETA, G_WB,
+  G_A = 32,                  // floats: A[16]
+  G_D = G_A + kHG,           // D[16]
+  G_DT = G_D + kHG           // dt of new tokens [8][16]
 };
 
-__host__ __device__ inline M2Stage m2_stage_layout(int P, int L, int tmax, int esz, int no) {
-  M2Stage s;
-  const int rmax = L + (tmax > 1 ? tmax : 1);
-  s.tile = kHdrBytes;
-  s.xr = s.tile + P * kCols * 4;
-  s.br = (int)align_up(s.xr + rmax * P * esz, 16);
-  s.cr = (int)align_up(s.br + rmax * kCols * esz, 16);
-  s.dtr = (int)align_up(s.cr + no * kCols * esz, 16);
-  s.bytes = (int)align_up(s.dtr + dt_stride(L) * 4, 128);
-  return s;
+struct M2Layout {
+  int rmax, no;
+  int tile_bytes;            // P*128*4
+  int xr;                    // offset of the x records in a tile stage
+  int stage_bytes;
+  int gb_B, gb_C, gb_dt, gb_bytes;  // group buffer
+  int tab_bytes;
+};
+
+__host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
+  M2Layout l;
+  l.no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
+  l.rmax = L + (tmax > 1 ? tmax : 1);
+  l.tile_bytes = P * kCols * 4;
+  l.xr = l.tile_bytes;
+  l.stage_bytes = (int)align_up((size_t)l.xr + (size_t)l.rmax * P * esz, 128);
+  l.gb_B = kGHdr;
+  l.gb_C = (int)align_up((size_t)l.gb_B + (size_t)l.rmax * kCols * esz, 16);
+  l.gb_dt = (int)align_up((size_t)l.gb_C + (size_t)l.no * kCols * esz, 16);
+  l.gb_bytes = (int)align_up((size_t)l.gb_dt + (size_t)kHG * dt_stride(L) * 4, 128);
+  // tables: g[no][rmax], coef[kHG][no][rmax], ao[kHG][no], wf[kHG][rmax], af[kHG], flags[8]
+  const int floats = l.no * l.rmax + kHG * l.no * l.rmax + kHG * l.no + kHG * l.rmax + kHG + 8;
+  l.tab_bytes = (int)align_up((size_t)floats * 4, 128);
+  return l;
 }
 
-constexpr int kTableFloats(int rmax, int no, int P) { return no * rmax + rmax + no + no * P; }
+// barriers: full[8], empty[8], gfull[2], gempty[2], tfull[2]; then armed phase per barrier (ints)
+constexpr int kBarBytes = 256;
+constexpr int kM2Threads = kConsumers + 64;  // + producer warp + prep warp
+constexpr int kProducerWarp = kConsumerWarps, kPrepWarp = kConsumerWarps + 1;
 
 template <typename TI, int NO>
-__global__ void __launch_bounds__(kThreads, 1) m2_replay_kernel(M2Args a) {
+__global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int esz = sizeof(TI);
-  const M2Stage lay = m2_stage_layout(a.P, a.L, a.tmax, esz, NO);
-  const int rmax = a.L + (a.tmax > 1 ? a.tmax : 1);
+  const M2Layout lay = m2_layout(a.P, a.L, a.tmax, esz);
+  const int NS = a.nstage;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *empty = full + a.nstage;
-  float *tab = reinterpret_cast<float *>(smem + 16 * a.nstage);
-  float *g_co = tab;                      // [NO][rmax] coefficient of record r in output j
-  float *w_f = g_co + NO * rmax;          // [rmax]   fold weight of record r
-  float *a_o = w_f + rmax;                // [NO]     checkpoint factor of output j
-  float *extra = a_o + NO;                // [NO][P]  buffered part of output j
-  float *a_f = extra + NO * a.P;          // [1]      checkpoint factor of the fold
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(a_f + 1);
-  volatile int *issued = abort_flag + 1;    // units whose copies the producer has issued
-  volatile int *consumed = abort_flag + 2;  // units the consumers have taken
-  unsigned char *stages = smem + a.stage_base;
+  uint64_t *empty = full + 8;
+  uint64_t *gfull = empty + 8;
+  uint64_t *gempty = gfull + 2;
+  uint64_t *tfull = gempty + 2;
+  volatile int *armed = reinterpret_cast<volatile int *>(tfull + 2);  // [10]: last armed phase of full[0..7], gfull[0..1]
+  volatile int *abort_flag = armed + 10;
+  const int rmax = lay.rmax;
+  unsigned char *tabs = smem + kBarBytes;  // two table buffers
+  unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
+  unsigned char *stages = gbuf + 2 * lay.gb_bytes;
+  struct Tables {
+    float *g, *coef, *ao, *wf, *af;
+  };
+  auto tables = [&](int which) {
+    Tables t;
+    t.g = reinterpret_cast<float *>(tabs + (size_t)which * lay.tab_bytes);  // [NO][rmax]   B_r . C_j
+    t.coef = t.g + NO * rmax;                                                // [kHG][NO][rmax]
+    t.ao = t.coef + kHG * NO * rmax;                                         // [kHG][NO]
+    t.wf = t.ao + kHG * NO;                                                  // [kHG][rmax]
+    t.af = t.wf + kHG * rmax;                                                // [kHG]
+    return t;
+  };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int u_begin = (int)(((long long)blockIdx.x * a.units) / gridDim.x);
-  const int u_end = (int)(((long long)(blockIdx.x + 1) * a.units) / gridDim.x);
   const int hpg = a.H / a.G;
+  const int chunks = (hpg + kHG - 1) / kHG;
+  const int units = a.Bt * a.G * chunks;
+  const int u_begin = (int)(((long long)blockIdx.x * units) / gridDim.x);
+  const int u_end = (int)(((long long)(blockIdx.x + 1) * units) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < a.nstage; ++s) {
+    for (int s = 0; s < 8; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&gfull[s], 1);
+      mbar_init(&gempty[s], kConsumerWarps);
+      mbar_init(&tfull[s], 1);
+    }
+    for (int s = 0; s < 10; ++s) armed[s] = -1;
     *abort_flag = 0;
-    *issued = 0;
-    *consumed = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------------ producer warp
+  if (warp == kProducerWarp) {
+    // ================================================================== producer warp
     const uint64_t pol_stream = policy_evict_first();
     const uint64_t pol_keep = policy_evict_last();
-    int cached_b = -1;
+    const uint32_t xrow = (uint32_t)a.P * esz, brow = (uint32_t)kCols * esz;
+    const int L = a.L, dts = dt_stride(L);
+    int cached_b = -1, msk = 1;
     int4 meta = make_int4(0, 0, 0, 0);
-    int msk = 1;
-    for (int u = u_begin, i = 0; u < u_end; ++u, ++i) {
-      const int s = i % a.nstage;
-      const uint32_t ph = (uint32_t)((i / a.nstage) & 1);
-      const int b = u / a.H, h = u % a.H, g = h / hpg;
+    int ti = 0;
+    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+      const int b = u / (a.G * chunks);
+      const int g = (u / chunks) % a.G;
+      const int ch = u % chunks;
+      const int h0 = g * hpg + ch * kHG;
+      const int nh = min(kHG, hpg - ch * kHG);
       if (b != cached_b) {
         if (lane == 0) {
           meta = a.meta_in[b];
@@ -123,24 +159,20 @@ __global__ void __launch_bounds__(kThreads, 1) m2_replay_kernel(M2Args a) {
         cached_b = b;
       }
       const int c = meta.x, e = meta.y, pend = meta.z;
-      const int L = a.L;
-      // ---- schedule of this unit (identical for every head of the sequence)
+      // ---- schedule of this sequence for this call
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
       int mc = c, me = e, mp = pend;
       const int base_e = (e & 1) * L, base_n = ((e + 1) & 1) * L;
       if (pend != 0) {
         active = 0;
-        if (h == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
+        if (h0 == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
       } else if (a.op == OP_STEP) {
         n_new = 1;
         t_out = 1;
         int c1;
-        if (c == L) {  // pre-fold of a window completed by a commit
-          n_ring = L; m = L; slot0 = base_n; c1 = 1; me = e + 1;
-        } else {
-          n_ring = c; m = 0; slot0 = base_e + c; c1 = c + 1;
-        }
-        if (c1 == L) { m = n_ring + 1; mc = 0; me = me + 1; }  // eager fold: the window is full
+        if (c == L) { n_ring = L; m = L; slot0 = base_n; c1 = 1; me = e + 1; }   // pre-fold after a commit
+        else { n_ring = c; m = 0; slot0 = base_e + c; c1 = c + 1; }
+        if (c1 == L) { m = n_ring + 1; mc = 0; me = me + 1; }                   // eager fold: window full
         else mc = c1;
       } else if (a.op == OP_VERIFY) {
         n_new = a.T;
@@ -153,252 +185,307 @@ __global__ void __launch_bounds__(kThreads, 1) m2_replay_kernel(M2Args a) {
         else { n_ring = c; m = c; mc = 0; me = e + 1; }
       }
       const int n_rec = n_ring + n_new;
-      if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, abort_flag)) {
+      // ---- group buffer
+      const int gs = gi & 1;
+      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
-      unsigned char *st = stages + (size_t)s * lay.bytes;
-      int *hi = reinterpret_cast<int *>(st);
-      float *hf = reinterpret_cast<float *>(st);
+      unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
+      int *gh = reinterpret_cast<int *>(gb);
+      float *gf = reinterpret_cast<float *>(gb);
       if (lane == 0) {
-        hi[H_FLAGS] = active | ((active && m > 0) ? 2 : 0) | (h == 0 ? 4 : 0);
-        hi[H_NREC] = n_rec; hi[H_M] = m; hi[H_NRING] = n_ring; hi[H_NNEW] = n_new; hi[H_TOUT] = t_out;
-        hi[H_SLOT0] = slot0; hi[H_MC] = mc; hi[H_ME] = me; hi[H_MP] = mp; hi[H_B] = b; hi[H_H] = h;
-        hi[H_BASE] = base_e;
-        hf[H_F + 8] = a.A[h];
-        hf[H_F + 9] = a.D[h];
+        gh[G_ACTIVE] = active; gh[G_NREC] = n_rec; gh[G_M] = m; gh[G_NRING] = n_ring; gh[G_NNEW] = n_new;
+        gh[G_TOUT] = t_out; gh[G_SLOT0] = slot0; gh[G_MC] = mc; gh[G_ME] = me; gh[G_MP] = mp;
+        gh[G_B] = b; gh[G_G] = g; gh[G_H0] = h0; gh[G_NH] = nh; gh[G_BASE] = base_e;
+        gh[G_WMETA] = (h0 == 0); gh[G_WB] = (ch == 0);
       }
-      if (active && lane < n_new) {
-        const TI *dtp = reinterpret_cast<const TI *>(a.dt) + ((size_t)b * a.T + lane) * a.H + h;
-        hf[H_F + lane] = to_f32(*dtp);
+      if (lane < nh) {
+        gf[G_A + lane] = a.A[h0 + lane];
+        gf[G_D + lane] = a.D[h0 + lane];
+      }
+      if (active) {
+        for (int q = lane; q < n_new * nh; q += 32) {
+          const int t = q / nh, i = q % nh;
+          gf[G_DT + t * kHG + i] = to_f32(reinterpret_cast<const TI *>(a.dt)[((size_t)b * a.T + t) * a.H + h0 + i]);
+        }
       }
       __syncwarp();
-      // ---- bulk copies
-      uint32_t bytes = 0;
-      const uint32_t tile_b = (uint32_t)a.P * kCols * 4;
-      const uint32_t xrow = (uint32_t)a.P * esz, brow = (uint32_t)kCols * esz;
-      if (active) bytes = tile_b + n_rec * (xrow + brow) + dt_stride(L) * 4 + t_out * brow;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
+      const uint32_t gbytes = active ? (uint32_t)(n_rec * brow + t_out * brow + nh * dts * 4) : 0u;
+      if (lane == 0) {
+        armed[8 + gs] = gi >> 1;
+        mbar_arrive_expect_tx(&gfull[gs], gbytes);
+      }
       __syncwarp();
       if (active) {
-        const size_t unit = (size_t)b * a.H + h;
-        // copy k is issued by lane k
-        if (lane == 0) bulk_g2s(st + lay.tile, a.hp + unit * a.P * kCols, tile_b, &full[s], pol_stream);
-        if (lane == 1 && n_ring)
-          bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + base_e) * xrow,
-                   n_ring * xrow, &full[s], pol_keep);
-        if (lane == 2 && n_ring)
-          bulk_g2s(st + lay.br,
+        if (lane == 0 && n_ring)
+          bulk_g2s(gb + lay.gb_B,
                    reinterpret_cast<const unsigned char *>(a.ring_B) + (((size_t)b * a.G + g) * 2 * L + base_e) * brow,
-                   n_ring * brow, &full[s], pol_keep);
-        if (lane == 3)
-          bulk_g2s(st + lay.dtr, a.ring_dt + unit * dt_stride(L), dt_stride(L) * 4, &full[s], pol_keep);
+                   n_ring * brow, &gfull[gs], pol_keep);
+        if (lane == 1)
+          bulk_g2s(gb + lay.gb_dt, a.ring_dt + ((size_t)b * a.H + h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
         if (lane >= 4 && lane < 4 + n_new) {
           const int t = lane - 4;
-          bulk_g2s(st + lay.xr + (n_ring + t) * xrow,
-                   reinterpret_cast<const unsigned char *>(a.x) + (((size_t)b * a.T + t) * a.H + h) * xrow, xrow,
-                   &full[s], pol_keep);
-        }
-        if (lane >= 12 && lane < 12 + n_new) {
-          const int t = lane - 12;
-          bulk_g2s(st + lay.br + (n_ring + t) * brow,
+          bulk_g2s(gb + lay.gb_B + (n_ring + t) * brow,
                    reinterpret_cast<const unsigned char *>(a.Bin) + (((size_t)b * a.T + t) * a.G + g) * brow, brow,
-                   &full[s], pol_keep);
+                   &gfull[gs], pol_keep);
         }
-        if (lane >= 20 && lane < 20 + t_out) {
-          const int t = lane - 20;
-          bulk_g2s(st + lay.cr + t * brow,
+        if (lane >= 12 && lane < 12 + t_out) {
+          const int t = lane - 12;
+          bulk_g2s(gb + lay.gb_C + t * brow,
                    reinterpret_cast<const unsigned char *>(a.C) + (((size_t)b * a.T + t) * a.G + g) * brow, brow,
-                   &full[s], pol_keep);
+                   &gfull[gs], pol_keep);
         }
-      }
-      if (lane == 0) *issued = i + 1;
-    }
-  } else {
-
-  // -------------------------------------------------------------------- consumer warps
-  const int tid = threadIdx.x;
-  for (int u = u_begin, i = 0; u < u_end; ++u, ++i) {
-    const int s = i % a.nstage;
-    const uint32_t ph = (uint32_t)((i / a.nstage) & 1);
-    if (!mbar_wait_or_abort(&full[s], ph, abort_flag) && lane == 0) {
-      record_error(a.err, u / a.H, RSSM_DEV_TIMEOUT);
-      *abort_flag = 1;
-    }
-    consumer_sync();  // a uniform decision: every consumer warp has waited (bounded) for this stage
-    if (*abort_flag) break;
-    if (tid == 0) *consumed = i + 1;
-    const unsigned char *st = stages + (size_t)s * lay.bytes;
-    const int *hi = reinterpret_cast<const int *>(st);
-    const float *hf = reinterpret_cast<const float *>(st);
-    const int flags = hi[H_FLAGS];
-    const int b = hi[H_B], h = hi[H_H];
-    if (flags & 4) {
-      if (tid == 0) a.meta_out[b] = make_int4(hi[H_MC], hi[H_ME], hi[H_MP], 0);
-    }
-    if (flags & 1) {
-      const int n_rec = hi[H_NREC], m = hi[H_M], n_ring = hi[H_NRING], n_new = hi[H_NNEW];
-      const int t_out = hi[H_TOUT];
-      const float A = hf[H_F + 8], Dh = hf[H_F + 9];
-      const TI *xr = reinterpret_cast<const TI *>(st + lay.xr);
-      const TI *br = reinterpret_cast<const TI *>(st + lay.br);
-      const TI *cr = reinterpret_cast<const TI *>(st + lay.cr);
-      const float *ring_dt = reinterpret_cast<const float *>(st + lay.dtr);
-      const int base_e = hi[H_BASE];
-      // dt of record r
-      auto dt_of = [&](int r) -> float { return r < n_ring ? ring_dt[base_e + r] : hf[H_F + (r - n_ring)]; };
-      // ---- P1: coefficients (pairs (j, r) with m <= r < e_j) and fold weights
-      const int npairs = NO * n_rec;
-      for (int pidx = warp; pidx < npairs; pidx += kConsumerWarps) {
-        const int j = pidx / n_rec, r = pidx % n_rec;
-        const int e_j = n_rec - t_out + j + 1;
-        if (j >= t_out || r < m || r >= e_j) {
-          if (lane == 0) g_co[j * rmax + r] = 0.f;
-          continue;
-        }
-        const float4 bv = load4(br + r * kCols + 4 * lane);
-        const float4 cv = load4(cr + j * kCols + 4 * lane);
-        float d = bv.x * cv.x + bv.y * cv.y + bv.z * cv.z + bv.w * cv.w;
-        d = warp_sum(d);
-        if (lane == 0) {
-          float sfx = 0.f;
-          for (int l = r + 1; l < e_j; ++l) sfx += dt_of(l);
-          g_co[j * rmax + r] = dt_of(r) * __expf(A * sfx) * d;
-        }
-      }
-      if (tid < NO) {
-        const int j = tid;
-        if (j < t_out) {
-          const int e_j = n_rec - t_out + j + 1;
-          float sm = 0.f;
-          for (int l = m; l < e_j; ++l) sm += dt_of(l);
-          a_o[j] = __expf(A * sm);
-        }
-      }
-      if (tid >= 64 && tid < 64 + m) {
-        const int r = tid - 64;
-        float sfx = 0.f;
-        for (int l = r + 1; l < m; ++l) sfx += dt_of(l);
-        w_f[r] = dt_of(r) * __expf(A * sfx);
-      }
-      if (tid == 128) {
-        float sm = 0.f;
-        for (int l = 0; l < m; ++l) sm += dt_of(l);
-        *a_f = __expf(A * sm);
-      }
-      consumer_sync();
-      // ---- P2: buffered part of each output row
-      for (int q = tid; q < NO * a.P; q += kConsumers) {
-        const int j = q / a.P, p = q % a.P;
-        if (j >= t_out) break;
-        const int e_j = n_rec - t_out + j + 1;
-        float acc = Dh * to_f32(xr[(e_j - 1) * a.P + p]);
-        for (int r = m; r < e_j; ++r) acc += g_co[j * rmax + r] * to_f32(xr[r * a.P + p]);
-        extra[j * a.P + p] = acc;
-      }
-      consumer_sync();
-      // ---- P3: stream the tile: fold (if any) and row dot products
-      const float *tile = reinterpret_cast<const float *>(st + lay.tile);
-      float4 cv[NO];
-#pragma unroll
-      for (int j = 0; j < NO; ++j) cv[j] = (j < t_out) ? load4(cr + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
-      const int row0 = warp * 8;
-      if (row0 < a.P) {
-        float4 sv[8];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) sv[rr] = *reinterpret_cast<const float4 *>(tile + (row0 + rr) * kCols + 4 * lane);
-        if (m > 0) {
-          const float af = *a_f;
-#pragma unroll
-          for (int rr = 0; rr < 8; ++rr) { sv[rr].x *= af; sv[rr].y *= af; sv[rr].z *= af; sv[rr].w *= af; }
-          for (int r = 0; r < m; ++r) {
-            const float4 bv = load4(br + r * kCols + 4 * lane);
-            const float wr = w_f[r];
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-              const float cx = wr * to_f32(xr[r * a.P + row0 + rr]);
-              sv[rr].x = fmaf(cx, bv.x, sv[rr].x);
-              sv[rr].y = fmaf(cx, bv.y, sv[rr].y);
-              sv[rr].z = fmaf(cx, bv.z, sv[rr].z);
-              sv[rr].w = fmaf(cx, bv.w, sv[rr].w);
-            }
+        // ---- tiles of the unit's heads
+        const uint32_t tbytes = (uint32_t)lay.tile_bytes + n_rec * xrow;
+        bool ok = true;
+        for (int i = 0; i < nh; ++i, ++ti) {
+          const int s = ti % NS;
+          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+            if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+            ok = false;
+            break;
           }
-          float *dst = a.hp + ((size_t)b * a.H + h) * a.P * kCols;
-#pragma unroll
-          for (int rr = 0; rr < 8; ++rr) __stcs(reinterpret_cast<float4 *>(dst + (row0 + rr) * kCols + 4 * lane), sv[rr]);
-        }
-        float part[8 * NO];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr)
-#pragma unroll
-          for (int j = 0; j < NO; ++j)
-            part[rr * NO + j] = sv[rr].x * cv[j].x + sv[rr].y * cv[j].y + sv[rr].z * cv[j].z + sv[rr].w * cv[j].w;
-        warp_transpose_reduce<8 * NO>(part, lane);
-        constexpr int V = 8 * NO;
-        constexpr int KEEP = V >= 32 ? V / 32 : 1;
-        constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
-        if ((lane % SPREAD) == 0) {
-#pragma unroll
-          for (int i2 = 0; i2 < KEEP; ++i2) {
-            const int idx = (V >= 32) ? lane * KEEP + i2 : lane / SPREAD;
-            const int rr = idx / NO, j = idx % NO;
-            if (j < t_out) {
-              const int p = row0 + rr;
-              a.y[(((size_t)b * a.T + j) * a.H + h) * a.P + p] = a_o[j] * part[i2] + extra[j * a.P + p];
-            }
+          unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          const size_t unit = (size_t)b * a.H + h0 + i;
+          if (lane == 0) {
+            armed[s] = ti / NS;
+            mbar_arrive_expect_tx(&full[s], tbytes);
+          }
+          __syncwarp();
+          if (lane == 0) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
+          if (lane == 1 && n_ring)
+            bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + base_e) * xrow,
+                     n_ring * xrow, &full[s], pol_keep);
+          if (lane >= 4 && lane < 4 + n_new) {
+            const int t = lane - 4;
+            bulk_g2s(st + lay.xr + (n_ring + t) * xrow,
+                     reinterpret_cast<const unsigned char *>(a.x) + (((size_t)b * a.T + t) * a.H + h0 + i) * xrow, xrow,
+                     &full[s], pol_keep);
           }
         }
+        if (!ok) break;
       }
-      // ---- P4: append the new tokens to the ring
-      if (n_new) {
-        const int slot0 = hi[H_SLOT0];
-        const size_t unit = (size_t)b * a.H + h;
-        const int xq = a.P * esz / 16;  // 16-byte chunks per x row
-        for (int q = tid; q < n_new * xq; q += kConsumers) {
-          const int t = q / xq, c16 = q % xq;
-          const uint4 v = *reinterpret_cast<const uint4 *>(st + lay.xr + (n_ring + t) * a.P * esz + c16 * 16);
-          *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
-                                     ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v;
+    }
+  } else if (warp == kPrepWarp) {
+    // ================================================================== prep warp
+    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+      const int gs = gi & 1;
+      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+        if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
+      const int *gh = reinterpret_cast<const int *>(gb);
+      const float *gf = reinterpret_cast<const float *>(gb);
+      const int b = gh[G_B], g = gh[G_G], nh = gh[G_NH];
+      if (gh[G_WMETA] && lane == 0) a.meta_out[b] = make_int4(gh[G_MC], gh[G_ME], gh[G_MP], 0);
+      if (gh[G_ACTIVE]) {
+        const Tables T = tables(gs);
+        const int n_rec = gh[G_NREC], m = gh[G_M], n_ring = gh[G_NRING], n_new = gh[G_NNEW], t_out = gh[G_TOUT];
+        const int slot0 = gh[G_SLOT0], base_e = gh[G_BASE];
+        const int dts = dt_stride(a.L);
+        const TI *Bg = reinterpret_cast<const TI *>(gb + lay.gb_B);
+        const TI *Cg = reinterpret_cast<const TI *>(gb + lay.gb_C);
+        const float *dtg = reinterpret_cast<const float *>(gb + lay.gb_dt);
+        auto dt_of = [&](int i, int r) -> float {
+          return r < n_ring ? dtg[i * dts + base_e + r] : gf[G_DT + (r - n_ring) * kHG + i];
+        };
+        // g[j][r] = B_r . C_j, eight records per task
+        const int rblocks = (n_rec + 7) / 8;
+        for (int task = 0; task < t_out * rblocks; ++task) {
+          const int j = task / rblocks, r0 = (task % rblocks) * 8;
+          const float4 cv = load4(Cg + j * kCols + 4 * lane);
+          float pd[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int r = r0 + q < n_rec ? r0 + q : n_rec - 1;
+            const float4 bv = load4(Bg + r * kCols + 4 * lane);
+            pd[q] = bv.x * cv.x + bv.y * cv.y + bv.z * cv.z + bv.w * cv.w;
+          }
+          warp_transpose_reduce<8>(pd, lane);
+          if ((lane & 3) == 0 && r0 + (lane >> 2) < n_rec) T.g[j * rmax + r0 + (lane >> 2)] = pd[0];
         }
-        if (tid < n_new) a.ring_dt[unit * dt_stride(a.L) + slot0 + tid] = hf[H_F + tid];
-        if (h % hpg == 0) {
-          const int g = h / hpg;
+        // B records of the new tokens go to the group's ring row (first chunk only)
+        if (gh[G_WB]) {
           const int bq = kCols * esz / 16;
-          for (int q = tid; q < n_new * bq; q += kConsumers) {
+          for (int q = lane; q < n_new * bq; q += 32) {
             const int t = q / bq, c16 = q % bq;
-            const uint4 v = *reinterpret_cast<const uint4 *>(st + lay.br + (n_ring + t) * kCols * esz + c16 * 16);
+            const uint4 v = *reinterpret_cast<const uint4 *>(gb + lay.gb_B + (n_ring + t) * kCols * esz + c16 * 16);
             *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_B) +
                                        ((((size_t)b * a.G + g) * 2 * a.L + slot0 + t) * kCols) * esz + c16 * 16) = v;
           }
         }
+        __syncwarp();
+        // per-head decay weights (log-space suffix sums of dt); pairs (head, output), then fold weights
+        for (int pr = lane; pr < nh * t_out; pr += 32) {
+          const int i = pr / t_out, j = pr % t_out;
+          const float A = gf[G_A + i];
+          const int e_j = n_rec - t_out + j + 1;
+          float sfx = 0.f;
+          for (int r = e_j - 1; r >= m; --r) {
+            const float d = dt_of(i, r);
+            T.coef[(i * NO + j) * rmax + r] = d * __expf(A * sfx) * T.g[j * rmax + r];
+            sfx += d;
+          }
+          T.ao[i * NO + j] = __expf(A * sfx);
+        }
+        if (m > 0 && lane < nh) {
+          const int i = lane;
+          const float A = gf[G_A + i];
+          float sfx = 0.f;
+          for (int r = m - 1; r >= 0; --r) {
+            const float d = dt_of(i, r);
+            T.wf[i * rmax + r] = d * __expf(A * sfx);
+            sfx += d;
+          }
+          T.af[i] = __expf(A * sfx);
+        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tfull[gs]);
     }
-    // release the stage (all reads of it above are done) and the tables for the next unit
-    consumer_sync();
-    if (lane == 0) mbar_arrive(&empty[s]);
-  }
+  } else {
+    // ================================================================== consumer warps
+    const int row0 = warp * 8;
+    int ti = 0;
+    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+      const int gs = gi & 1;
+      if (!mbar_wait_or_abort(&tfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+        if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
+      const int *gh = reinterpret_cast<const int *>(gb);
+      const float *gf = reinterpret_cast<const float *>(gb);
+      const int b = gh[G_B], h0 = gh[G_H0], nh = gh[G_NH];
+      if (gh[G_ACTIVE]) {
+        const Tables T = tables(gs);
+        const float *t_coef = T.coef, *t_ao = T.ao, *t_wf = T.wf, *t_af = T.af;
+        const int n_rec = gh[G_NREC], m = gh[G_M], n_ring = gh[G_NRING], n_new = gh[G_NNEW], t_out = gh[G_TOUT];
+        const int slot0 = gh[G_SLOT0];
+        const int dts = dt_stride(a.L);
+        const TI *Bg = reinterpret_cast<const TI *>(gb + lay.gb_B);
+        const TI *Cg = reinterpret_cast<const TI *>(gb + lay.gb_C);
+        // ---- stream the heads' tiles; each warp works and releases on its own
+        float4 cv[NO];
+#pragma unroll
+        for (int j = 0; j < NO; ++j) cv[j] = (j < t_out) ? load4(Cg + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
+        constexpr int V = 8 * NO;
+        constexpr int KEEP = V >= 32 ? V / 32 : 1;
+        constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
+        for (int i = 0; i < nh; ++i, ++ti) {
+          const int s = ti % NS;
+          if (!mbar_wait_or_abort(&full[s], (uint32_t)((ti / NS) & 1), abort_flag)) {
+            if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+            break;
+          }
+          const unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          const float *tile = reinterpret_cast<const float *>(st);
+          const TI *xr = reinterpret_cast<const TI *>(st + lay.xr);
+          const int h = h0 + i;
+          const size_t unit = (size_t)b * a.H + h;
+          if (row0 < a.P) {
+            float4 sv[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) sv[rr] = *reinterpret_cast<const float4 *>(tile + (row0 + rr) * kCols + 4 * lane);
+            if (m > 0) {
+              const float af = t_af[i];
+#pragma unroll
+              for (int rr = 0; rr < 8; ++rr) { sv[rr].x *= af; sv[rr].y *= af; sv[rr].z *= af; sv[rr].w *= af; }
+              for (int r = 0; r < m; ++r) {
+                const float4 bv = load4(Bg + r * kCols + 4 * lane);
+                const float wr = t_wf[i * rmax + r];
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                  const float cx = wr * to_f32(xr[r * a.P + row0 + rr]);
+                  sv[rr].x = fmaf(cx, bv.x, sv[rr].x);
+                  sv[rr].y = fmaf(cx, bv.y, sv[rr].y);
+                  sv[rr].z = fmaf(cx, bv.z, sv[rr].z);
+                  sv[rr].w = fmaf(cx, bv.w, sv[rr].w);
+                }
+              }
+              float *dst = a.hp + unit * a.P * kCols;
+#pragma unroll
+              for (int rr = 0; rr < 8; ++rr)
+                __stcs(reinterpret_cast<float4 *>(dst + (row0 + rr) * kCols + 4 * lane), sv[rr]);
+            }
+            float part[V];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+              for (int j = 0; j < NO; ++j)
+                part[rr * NO + j] = sv[rr].x * cv[j].x + sv[rr].y * cv[j].y + sv[rr].z * cv[j].z + sv[rr].w * cv[j].w;
+            warp_transpose_reduce<V>(part, lane);
+            const float Dh = gf[G_D + i];
+#pragma unroll
+            for (int k2 = 0; k2 < KEEP; ++k2) {
+              const int idx = (V >= 32) ? lane * KEEP + k2 : lane / SPREAD;
+              const int rr = idx / NO, j = idx % NO;
+              const int p = row0 + rr;
+              const int e_j = n_rec - t_out + j + 1;
+              float acc = 0.f;
+              if (j < t_out) {
+                const float *co = t_coef + (i * NO + j) * rmax;
+                for (int r = m + (lane % SPREAD); r < e_j; r += SPREAD) acc = fmaf(co[r], to_f32(xr[r * a.P + p]), acc);
+              }
+#pragma unroll
+              for (int off = 1; off < SPREAD; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+              if (j < t_out && (lane % SPREAD) == 0)
+                a.y[(((size_t)b * a.T + j) * a.H + h) * a.P + p] =
+                    t_ao[i * NO + j] * part[k2] + acc + Dh * to_f32(xr[(e_j - 1) * a.P + p]);
+            }
+          }
+          if (warp == 0 && n_new) {  // append this head's new tokens (x rows, dt) to its ring row
+            const int xq = a.P * esz / 16;
+            for (int q = lane; q < n_new * xq; q += 32) {
+              const int t = q / xq, c16 = q % xq;
+              const uint4 v = *reinterpret_cast<const uint4 *>(st + lay.xr + (n_ring + t) * a.P * esz + c16 * 16);
+              *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
+                                         ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v;
+            }
+            if (lane < n_new) a.ring_dt[unit * dts + slot0 + lane] = gf[G_DT + lane * kHG + i];
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+        }
+      }
+      if (*abort_flag) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gempty[gs]);  // this warp is done with the group buffer and the tables
+    }
   }
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
-    // do not leave bulk copies in flight into shared memory of an exiting block
-    for (int i = *consumed; i < *issued; ++i)
-      if (!mbar_wait(&full[i % a.nstage], (uint32_t)((i / a.nstage) & 1))) break;
+    // do not leave bulk copies in flight into the shared memory of an exiting block
+    for (int s = 0; s < 8; ++s)
+      if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1));
+    for (int s = 0; s < 2; ++s)
+      if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
   }
 }
 
 }  // namespace
 
-int m2_stage_bytes(int P, int L, int tmax, int esz, int no) { return m2_stage_layout(P, L, tmax, esz, no).bytes; }
+int m2_smem_bytes(int P, int L, int tmax, int esz, int nstage) {
+  const M2Layout l = m2_layout(P, L, tmax, esz);
+  return kBarBytes + 2 * l.tab_bytes + 2 * l.gb_bytes + nstage * l.stage_bytes;
+}
 
-int m2_table_bytes(int P, int L, int tmax, int no) {
-  const int rmax = L + (tmax > 1 ? tmax : 1);
-  return (int)align_up((size_t)(kTableFloats(rmax, no, P) + 4) * 4, 128);
+int m2_max_stages(int P, int L, int tmax, int esz, int smem_budget) {
+  int n = 8;
+  while (n > 2 && m2_smem_bytes(P, L, tmax, esz, n) > smem_budget) --n;
+  return n;
+}
+
+int m2_units(int Bt, int H, int G) {
+  const int hpg = H / G;
+  return Bt * G * ((hpg + kHG - 1) / kHG);
 }
 
 cudaError_t launch_m2_replay(M2Args a, int esz, cudaStream_t stream) {
   const int no = a.tmax <= 1 ? 1 : a.tmax <= 2 ? 2 : a.tmax <= 4 ? 4 : 8;
-  a.stage_base = (int)align_up(16 * a.nstage + m2_table_bytes(a.P, a.L, a.tmax, no), 128);
-  const size_t smem = a.stage_base + (size_t)a.nstage * m2_stage_bytes(a.P, a.L, a.tmax, esz, no);
+  const size_t smem = m2_smem_bytes(a.P, a.L, a.tmax, esz, a.nstage);
   void (*kern)(M2Args) = nullptr;
 #define RSSM_PICK(TI, NOV) \
   if (no == NOV) kern = m2_replay_kernel<TI, NOV>;
@@ -410,7 +497,7 @@ cudaError_t launch_m2_replay(M2Args a, int esz, cudaStream_t stream) {
 #undef RSSM_PICK
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<a.grid, kThreads, smem, stream>>>(a);
+  kern<<<a.grid, kM2Threads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
