@@ -33,7 +33,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import MAMBA2_120B, mamba2_initial_state, mamba2_params, mamba2_step_inputs  # noqa: E402
+from synth import (GDN_B256, MAMBA2_120B, SPEC_MAMBA2_B512, accepted_lengths, gdn_initial_state,  # noqa: E402
+                   gdn_step_inputs, mamba2_draft_inputs, mamba2_initial_state, mamba2_params, mamba2_step_inputs)
 
 WL = MAMBA2_120B
 METRIC = "SSM decode tokens/s & achieved HBM GB/s at B=256, L=16 vs step-by-step kernel"
@@ -317,13 +318,139 @@ def run_gpu(args, rank, world):
     return res
 
 
+def gdn_traffic(wl, count_before: int) -> int:
+    """Algorithmic bytes of one GDN replay step (same terms as the Mamba-2 model)."""
+    Bt, H, dk, dv, L = wl.batch, wl.nheads, wl.dk, wl.dv, wl.window
+    esz = 2 if wl.in_dtype == "bf16" else 4
+    state = Bt * H * dv * dk * 4
+    rec = Bt * H * (dk * esz + dv * esz + 8)
+    tok = Bt * H * (2 * dk * esz + dv * esz + 8)
+    fold = count_before + 1 == L
+    return state + (state if fold else 0) + count_before * rec + tok + rec + Bt * H * dv * 4
+
+
+def timed(fn, n, stream):
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def gdn_section(steps: int) -> dict:
+    """Gated DeltaNet layer (batch 256, 32 heads, d_k = d_v = 128, L 16): replay vs conventional."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM, conv_gdn_step, make_config
+    wl, dev = GDN_B256, torch.device("cuda")
+    bf = torch.bfloat16
+    layer = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, wl.dk, 1, wl.window, 0, bf)
+    S0 = torch.from_numpy(gdn_initial_state(wl)).to(dev)
+    layer.load_checkpoint(S0)
+    pool = []
+    for t in range(16):
+        inp = gdn_step_inputs(wl, t)
+        pool.append({k: torch.from_numpy(v).to(dev).to(torch.float32 if k in ("alpha", "beta") else bf)
+                     for k, v in inp.items()})
+    y = torch.empty(wl.batch, wl.nheads, wl.dv, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        t = pool[i % 16]
+        layer.gdn_step(t["q"], t["k"], t["v"], t["alpha"], t["beta"], y)
+
+    for i in range(2 * wl.window):
+        step(i)
+    K = max(wl.window, steps // wl.window * wl.window)
+    ms = timed(step, K, stream)
+    bytes_avg = sum(gdn_traffic(wl, i % wl.window) for i in range(K)) / K
+    cfg = make_config("gdn", wl.batch, wl.nheads, wl.dv, wl.dk, 1, wl.window, 0, bf)
+    S = S0.clone()
+
+    def conv(i):
+        t = pool[i % 16]
+        conv_gdn_step(cfg, S, t["q"], t["k"], t["v"], t["alpha"], t["beta"], y)
+
+    for i in range(4):
+        conv(i)
+    ms_conv = timed(conv, max(16, K // 4), stream)
+    conv_bytes = 2 * S0.numel() * 4 + wl.batch * wl.nheads * (2 * wl.dk * 2 + wl.dv * 2 + 8 + wl.dv * 4)
+    hbm, _ = load_peaks()
+    return {"workload": "gdn replay decode, batch 256, 32 heads, d_k = d_v = 128, L 16, bf16 inputs, fp32 checkpoint",
+            "tokens_per_s": wl.batch / (ms * 1e-3), "ms_per_step": ms, "GBps": bytes_avg / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": bytes_avg / (ms * 1e-3) / 1e9 / hbm, "bytes_per_step": bytes_avg,
+            "conventional_tokens_per_s": wl.batch / (ms_conv * 1e-3), "conventional_ms_per_step": ms_conv,
+            "conventional_GBps": conv_bytes / (ms_conv * 1e-3) / 1e9, "replay_speedup": ms_conv / ms,
+            "steps": K, "device_error": layer.get_error()}
+
+
+def verify_section(rounds: int) -> dict:
+    """Speculative verify + commit on the Mamba-2 shape at batch 512 (T = 4, 8) vs snapshot-per-draft."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM, make_config, snap_commit, snap_verify
+    wl, dev, bf = SPEC_MAMBA2_B512, torch.device("cuda"), torch.bfloat16
+    p = mamba2_params(wl)
+    A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
+    stream = torch.cuda.current_stream()
+    S0 = torch.from_numpy(mamba2_initial_state(wl)).to(dev)
+    out = {"workload": "mamba2 speculative verify + commit, batch 512, 128 heads, P 64, N 128, 8 groups, L 16"}
+    for T in (4, 8):
+        layer = ReplaySSM("mamba2", wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window, T, bf,
+                          A=A, D=D)
+        layer.load_checkpoint(S0)
+        drafts = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in mamba2_draft_inputs(wl, r, T).items()}
+                  for r in range(4)]
+        accs = [torch.from_numpy(accepted_lengths(wl, r, T)).to(dev) for r in range(rounds)]
+        acc_total = sum(int(a.sum()) for a in accs)
+        y = torch.empty(wl.batch, T, wl.nheads, wl.headdim, device=dev)
+
+        def rnd(i):
+            d = drafts[i % 4]
+            layer.verify(T, y=y, x=d["x"], B=d["B"], C=d["C"], dt=d["dt"])
+            layer.commit(accs[i])
+
+        for i in range(min(8, rounds)):
+            rnd(i)
+        layer.load_checkpoint(S0)
+        ms = timed(rnd, rounds, stream)
+        err = layer.get_error()
+        del layer
+        # snapshot-per-draft comparison: one state read, T state writes per round
+        cfg = make_config("mamba2", wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window, T, bf, A=A, D=D)
+        snaps = torch.empty(wl.batch, T + 1, wl.nheads, wl.headdim, wl.dstate, device=dev)
+        snaps[:, 0].copy_(S0)
+        cur = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+
+        def snap(i):
+            d = drafts[i % 4]
+            snap_verify(cfg, snaps, cur, T, y, x=d["x"], B=d["B"], C=d["C"], dt=d["dt"])
+            snap_commit(cfg, cur, accs[i])
+
+        for i in range(min(4, rounds)):
+            snap(i)
+        ms_snap = timed(snap, rounds, stream)
+        del snaps
+        out[f"T{T}"] = {"ms_per_round": ms, "verified_tokens_per_s": wl.batch * T / (ms * 1e-3),
+                        "committed_tokens_per_s": acc_total / rounds / (ms * 1e-3),
+                        "snapshot_ms_per_round": ms_snap,
+                        "snapshot_committed_tokens_per_s": acc_total / rounds / (ms_snap * 1e-3),
+                        "speedup_vs_snapshot": ms_snap / ms, "rounds": rounds, "device_error": err}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--steps", type=int, default=4096)
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the GDN and speculative-verify sections")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -342,6 +469,9 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_gpu(args, rank, world)
+    if rank == 0 and world == 1 and not args.no_extra:
+        res["gdn"] = gdn_section(min(args.steps, 1024))
+        res["verify"] = verify_section(64)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -160,7 +160,7 @@ class ReplaySSM:
         dev, Bt, H, R = self.device, self.batch, self.nheads, self.rows
         codes = torch.empty(Bt, H, R, 64, dtype=torch.uint8, device=dev)
         scales = torch.empty(Bt, H, R, 8, dtype=torch.uint8, device=dev)
-        g = torch.empty(Bt, H, dtype=torch.float32, device=dev)
+        g = torch.empty(Bt, H, (R + 63) // 64, dtype=torch.float32, device=dev)
         abi.check(self.lib.rssm_export_read_copy(self.handle, _ptr(codes), _ptr(scales), _ptr(g), _stream()),
                   "rssm_export_read_copy")
         return {"packed": codes, "scales": scales, "g": g}

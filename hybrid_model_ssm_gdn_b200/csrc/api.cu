@@ -58,19 +58,9 @@ rssm_status validate(const rssm_config *c) {
   return RSSM_OK;
 }
 
-int pow2_outputs(int t) { return t <= 1 ? 1 : t <= 2 ? 2 : t <= 4 ? 4 : 8; }
-
 const int4 *meta_cur(rssm_ctx *x) { return reinterpret_cast<const int4 *>(x->arena + x->lay.meta) + x->parity * x->cfg.batch; }
 int4 *meta_next(rssm_ctx *x) { return reinterpret_cast<int4 *>(x->arena + x->lay.meta) + (1 - x->parity) * x->cfg.batch; }
 int *err_word(rssm_ctx *x) { return reinterpret_cast<int *>(x->arena + x->lay.err); }
-
-int pick_stages(rssm_ctx *x, int stage_bytes, int table_bytes) {
-  if (x->nstage_override > 0) return x->nstage_override;
-  const int budget = x->smem_optin - 1024;
-  int n = 8;
-  while (n > 2 && 16 * n + table_bytes + n * stage_bytes > budget) --n;
-  return n;
-}
 
 rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, const void *C, const void *dt,
                    const unsigned char *mask, float *y, cudaStream_t stream) {
@@ -100,13 +90,12 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   GArgs a{};
   a.Bt = c.batch; a.H = c.nheads; a.DV = c.headdim; a.L = c.window;
   a.T = T; a.tmax = op == OP_VERIFY ? T : 1; a.op = op;
-  a.units = c.batch * c.nheads;
+  a.units = g_units(c.batch, c.nheads, a.tmax);
   a.grid = a.units < x->num_sms ? a.units : x->num_sms;
   a.hp_mode = c.hp; a.read_mode = c.read; a.seed = c.seed; a.q_scale = c.q_scale;
   const int esz = esize(c);
-  const int sb = g_stage_bytes(a, esz), tb = g_table_bytes(a);
-  a.nstage = pick_stages(x, sb, tb);
-  if (16 * a.nstage + tb + a.nstage * sb > x->smem_optin) return RSSM_ERR_SHAPE;
+  a.nstage = x->nstage_override > 0 ? x->nstage_override : g_max_stages(a.DV, a.L, a.tmax, esz, x->smem_optin - 1024);
+  if (a.nstage < 2 || a.nstage > 8 || g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) > x->smem_optin) return RSSM_ERR_SHAPE;
   a.meta_in = meta_cur(x); a.meta_out = meta_next(x); a.err = err_word(x);
   a.hp = x->arena + x->lay.hp;
   a.rq = x->arena + x->lay.rq; a.rs = x->arena + x->lay.rs; a.rg = reinterpret_cast<float *>(x->arena + x->lay.rg);
@@ -301,7 +290,8 @@ rssm_status rssm_export_read_copy(rssm_ctx *x, unsigned char *codes, unsigned ch
   if (codes) e = cudaMemcpyAsync(codes, x->arena + x->lay.rq, elems / 2, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess && scales) e = cudaMemcpyAsync(scales, x->arena + x->lay.rs, elems / 16, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess && g)
-    e = cudaMemcpyAsync(g, x->arena + x->lay.rg, (size_t)c.batch * c.nheads * 4, cudaMemcpyDeviceToDevice, st);
+    e = cudaMemcpyAsync(g, x->arena + x->lay.rg, (size_t)c.batch * c.nheads * ((c.headdim + 63) / 64) * 4,
+                        cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return RSSM_OK;
 }

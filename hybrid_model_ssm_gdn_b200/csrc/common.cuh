@@ -42,7 +42,7 @@ struct ArenaLayout {
   size_t hp;       // checkpoint: fp32 or fp16 [Bt][H][R][128]
   size_t rq;       // NVFP4 codes u8 [Bt][H][R][64]
   size_t rs;       // NVFP4 block scales u8 [Bt][H][R][8]
-  size_t rg;       // NVFP4 tile scale fp32 [Bt][H]
+  size_t rg;       // NVFP4 tile scale fp32 [Bt][H][ceil(R/64)] (padded to 16 bytes)
   size_t ring_a;   // Mamba-2 x [Bt][H][2L][P] / GDN k [Bt][H][2L][128]   (input dtype)
   size_t ring_b;   // Mamba-2 B [Bt][G][2L][128] / GDN v [Bt][H][2L][d_v] (input dtype)
   size_t ring_c;   // Mamba-2 dt / GDN alpha: fp32 [Bt][H][dt_stride(L)]
@@ -64,7 +64,8 @@ inline ArenaLayout make_layout(const rssm_config &c) {
   const bool fp4 = c.read != RSSM_READ_SAME;
   a.rq = take(fp4 ? units * R * kCols / 2 : 0);
   a.rs = take(fp4 ? units * R * kCols / 16 : 0);
-  a.rg = take(fp4 ? units * 4 : 0);
+  const size_t nrb = (R + 63) / 64;  // NVFP4 tiles (64-row blocks) per head
+  a.rg = take(fp4 ? align_up(units * nrb, 4) * 4 : 0);
   if (c.kind == RSSM_MAMBA2) {
     a.ring_a = take(units * 2 * L * R * esz);
     a.ring_b = take(Bt * c.ngroups * 2 * L * kCols * esz);
@@ -96,6 +97,19 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
   r.z = __uint_as_float(u.y << 16);
   r.w = __uint_as_float(u.y & 0xffff0000u);
   return r;
+}
+
+// 8 consecutive elements starting at p (16-byte aligned for bf16, 32-byte for float)
+__device__ __forceinline__ void load8(const float *p, float (&o)[8]) {
+  const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&o)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  o[0] = __uint_as_float(u.x << 16); o[1] = __uint_as_float(u.x & 0xffff0000u);
+  o[2] = __uint_as_float(u.y << 16); o[3] = __uint_as_float(u.y & 0xffff0000u);
+  o[4] = __uint_as_float(u.z << 16); o[5] = __uint_as_float(u.z & 0xffff0000u);
+  o[6] = __uint_as_float(u.w << 16); o[7] = __uint_as_float(u.w & 0xffff0000u);
 }
 
 __device__ __forceinline__ void record_error(int *err, int seq, int code) { atomicMin(err, seq * 16 + code); }

@@ -1,8 +1,706 @@
-// gdn.cu -- Gated DeltaNet replay kernels (placeholder until the kernel lands).
+// gdn.cu -- ReplaySSM decode kernels for Gated DeltaNet layers (sm_100a).
+//
+// Per (sequence b, head h) the state S in R^{d_v x 128} follows the gated delta rule
+//     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   y_t = q_scale S_t q_t
+// and is held as a checkpoint plus the inputs (k, v, alpha, beta) of the tokens since it
+// ("SSM decoding stops writing state every step", Synopsis and Interpretation, second
+// paragraph).  With the call's records r = 0..n_rec-1 (buffered, then new), the first m
+// are folded into the state and output j replays records m..e_j-1.  The replay walks q
+// back through the buffered factors, newest first:
+//     u <- q_j;  for r = e_j-1 .. m:  c_r = k_r . u;  u <- alpha_r (u - beta_r c_r k_r)
+//     y_j = q_scale (S' u + sum_r beta_r c_r v_r)
+// so the checkpoint enters through one matrix-vector product per output.  The fold is
+// row-local: each row s of S takes, record by record,
+//     s <- alpha_r s + beta_r (v_r[row] - alpha_r (s . k_r)) k_r.
+//
+// Precision modes ("Hybrid-model decoding has a new bottleneck", Interpretation, fourth
+// paragraph, Perspective, second paragraph): the checkpoint is fp32 or fp16 written with
+// stochastic rounding; the copy read by non-fold outputs is the checkpoint itself, a
+// separate NVFP4 copy re-quantised from the fp32 fold result, or (contrast) an NVFP4 copy
+// that is also the state the recurrence continues from.  Outputs of a call that folds
+// come from the fp32 fold result.
+//
+// Block roles (one block per SM, persistent):
+//  * producer warp: TMA bulk copies (cp.async.bulk) of each unit's k records, q and
+//    alpha/beta rows into a double-buffered group buffer, and of each 64-row tile of a
+//    head's state (in its stored format) plus the head's v records into a ring of stages;
+//  * two prep warps: 8-lane subgroups walk q back for every (head, draft) pair of the
+//    unit, writing u_0 and the coefficients beta_r c_r into double-buffered tables;
+//    they also append k, alpha, beta of the new tokens and write the bookkeeping word;
+//  * two groups of four consumer warps take alternate tiles.  Non-fold tiles: lane l owns
+//    columns 4l..4l+3 of 16 rows, row dot products with u_0 finish in a warp transpose
+//    reduction.  Fold tiles: two lanes own one row (64 columns each) and run the
+//    sequential row update with one shuffle per record; then the new state is written
+//    in the checkpoint format and, in NVFP4 modes, quantised (tile maximum over the
+//    group through a named barrier).
+// Work unit: (sequence, chunk of HG heads), HG = 4, 4, 2, 1 for 1, 2, 4, 8 outputs.
+#include "common.cuh"
 #include "kernels.h"
+#include "lowprec.cuh"
 
 namespace rssm {
-int g_stage_bytes(const GArgs &, int) { return 1 << 30; }
-int g_table_bytes(const GArgs &) { return 0; }
-cudaError_t launch_gdn_replay(GArgs, int, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+constexpr int kGHdrBytes = 1024;
+enum {
+  Q_ACTIVE = 0, Q_NREC, Q_M, Q_NRING, Q_NNEW, Q_TOUT, Q_SLOT0, Q_MC, Q_ME, Q_MP, Q_B, Q_H0, Q_NH, Q_BASE,
+  Q_WMETA,
+  Q_F = 32,                // floats: alpha of new tokens [8][8] (token, head)
+  Q_FB = Q_F + 64          // beta of new tokens [8][8]
+};
+constexpr int kGdnThreads = kConsumers + 96;  // + producer + two prep warps
+constexpr int kGProducer = kConsumerWarps, kGPrep0 = kConsumerWarps + 1;
+constexpr int kTileMaxBytes = kFp4Rows * kCols * 4;  // a 64-row fp32 tile
+
+__host__ __device__ inline int g_heads_per_unit(int no) { return no == 1 ? 4 : no == 2 ? 4 : no == 4 ? 2 : 1; }
+
+struct GLayout {
+  int no, rmax, hg, nrb, dts;
+  int gb_k, gb_q, gb_a, gb_b, gb_bytes;   // group buffer
+  int tb_u0, tb_coef, tb_amax, tab_bytes; // tables (per buffer)
+  int st_g, st_v, stage_bytes;            // tile stage: [tile 32 KiB][g chunk 16 B][v records]
+};
+
+__host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz) {
+  GLayout l;
+  l.no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
+  l.rmax = L + (tmax > 1 ? tmax : 1);
+  l.hg = g_heads_per_unit(l.no);
+  l.nrb = (R + kFp4Rows - 1) / kFp4Rows;
+  l.dts = dt_stride(L);
+  l.gb_k = kGHdrBytes;
+  l.gb_q = (int)align_up((size_t)l.gb_k + (size_t)l.hg * l.rmax * kCols * esz, 16);
+  l.gb_a = (int)align_up((size_t)l.gb_q + (size_t)l.hg * l.no * kCols * esz, 16);
+  l.gb_b = l.gb_a + l.hg * l.dts * 4;
+  l.gb_bytes = (int)align_up((size_t)l.gb_b + (size_t)l.hg * l.dts * 4, 128);
+  l.tb_u0 = 0;
+  l.tb_coef = l.hg * l.no * kCols * 4;
+  l.tb_amax = (int)align_up((size_t)l.tb_coef + (size_t)l.hg * l.no * l.rmax * 4, 16);
+  l.tab_bytes = (int)align_up((size_t)l.tb_amax + 2 * 2 * 4 * 4, 128);   // amax[group][slot][warp]
+  l.st_g = kTileMaxBytes;
+  l.st_v = l.st_g + 16;
+  l.stage_bytes = (int)align_up((size_t)l.st_v + (size_t)l.rmax * R * esz, 128);
+  return l;
+}
+
+constexpr int kBarBytesG = 256;
+
+// tile source formats
+enum { SRC_F32 = 0, SRC_F16 = 1, SRC_FP4 = 2 };
+
+template <typename TI>
+__device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 consecutive elements
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 v = load4(p + 4 * q);
+    o[4 * q] = v.x; o[4 * q + 1] = v.y; o[4 * q + 2] = v.z; o[4 * q + 3] = v.w;
+  }
+}
+
+template <typename TI, int NO>
+__global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int esz = sizeof(TI);
+  const GLayout lay = g_layout(a.DV, a.L, a.tmax, esz);
+  const int NS = a.nstage, R = a.DV, L = a.L, HG = lay.hg, nrb = lay.nrb, dts = lay.dts;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + 8;
+  uint64_t *gfull = empty + 8;
+  uint64_t *gempty = gfull + 2;
+  uint64_t *tfull = gempty + 2;
+  uint64_t *psync = tfull + 2;   // rendezvous of the two prep warps (count 2)
+  uint64_t *csync = psync + 1;   // [2] rendezvous of the four warps of a consumer group (count 4)
+  volatile int *armed = reinterpret_cast<volatile int *>(csync + 2);  // [10]
+  volatile int *abort_flag = armed + 10;
+  unsigned char *tabs = smem + kBarBytesG;
+  unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
+  unsigned char *stages = gbuf + 2 * lay.gb_bytes;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunks = (a.H + HG - 1) / HG;
+  const int units = a.Bt * chunks;
+  const int u_begin = (int)(((long long)blockIdx.x * units) / gridDim.x);
+  const int u_end = (int)(((long long)(blockIdx.x + 1) * units) / gridDim.x);
+  const bool fp4_read = a.read_mode != RSSM_READ_SAME;
+  const bool shared_fp4 = a.read_mode == RSSM_READ_SHARED_NVFP4;
+  const bool hp16 = a.hp_mode == RSSM_HP_F16_SR;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);  // one consumer group of four warps per tile
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&gfull[s], 1);
+      mbar_init(&gempty[s], kConsumerWarps);
+      mbar_init(&tfull[s], 1);
+    }
+    mbar_init(psync, 2);
+    mbar_init(&csync[0], 4);
+    mbar_init(&csync[1], 4);
+    for (int s = 0; s < 10; ++s) armed[s] = -1;
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kGProducer) {
+    // ================================================================== producer warp
+    const uint64_t pol_stream = policy_evict_first();
+    const uint64_t pol_keep = policy_evict_last();
+    const uint32_t krow = (uint32_t)kCols * esz, vrow = (uint32_t)R * esz;
+    const int b_first = u_begin / chunks;
+    int mw_base = -1, mk = 1;
+    int4 mw = make_int4(0, 0, 0, 0);
+    int ti = 0;
+    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+      const int b = u / chunks, ch = u % chunks;
+      const int h0 = ch * HG, nh = min(HG, a.H - h0);
+      const int base32 = b_first + ((b - b_first) & ~31);
+      if (base32 != mw_base) {
+        const int bq = base32 + lane;
+        if (bq < a.Bt) {
+          mw = a.meta_in[bq];
+          mk = (a.mask == nullptr) ? 1 : (int)a.mask[bq];
+        }
+        mw_base = base32;
+      }
+      const int src = b - base32;
+      const int c = __shfl_sync(0xffffffffu, mw.x, src), e = __shfl_sync(0xffffffffu, mw.y, src);
+      const int pend = __shfl_sync(0xffffffffu, mw.z, src), msk = __shfl_sync(0xffffffffu, mk, src);
+      // ---- schedule (identical for every head of the sequence)
+      int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
+      int mc = c, me = e, mp = pend;
+      const int base_e = (e & 1) * L, base_n = ((e + 1) & 1) * L;
+      if (pend != 0) {
+        active = 0;
+        if (h0 == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
+      } else if (a.op == OP_STEP) {
+        n_new = 1;
+        t_out = 1;
+        int c1;
+        if (c == L) { n_ring = L; m = L; slot0 = base_n; c1 = 1; me = e + 1; }
+        else { n_ring = c; m = 0; slot0 = base_e + c; c1 = c + 1; }
+        if (c1 == L) { m = n_ring + 1; mc = 0; me = me + 1; }
+        else mc = c1;
+      } else if (a.op == OP_VERIFY) {
+        n_new = a.T;
+        t_out = a.T;
+        mp = a.T;
+        if (c + a.T > L) { n_ring = c; m = c; slot0 = base_n; mc = 0; me = e + 1; }
+        else { n_ring = c; m = 0; slot0 = base_e + c; }
+      } else {
+        if (!msk || c == 0) active = 0;
+        else { n_ring = c; m = c; mc = 0; me = e + 1; }
+      }
+      const int n_rec = n_ring + n_new;
+      const int gs = gi & 1;
+      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
+        if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
+      int *gh = reinterpret_cast<int *>(gb);
+      if (lane == 0) {
+        gh[Q_ACTIVE] = active; gh[Q_NREC] = n_rec; gh[Q_M] = m; gh[Q_NRING] = n_ring; gh[Q_NNEW] = n_new;
+        gh[Q_TOUT] = t_out; gh[Q_SLOT0] = slot0; gh[Q_MC] = mc; gh[Q_ME] = me; gh[Q_MP] = mp;
+        gh[Q_B] = b; gh[Q_H0] = h0; gh[Q_NH] = nh; gh[Q_BASE] = base_e; gh[Q_WMETA] = (h0 == 0);
+      }
+      __syncwarp();
+      const uint32_t gbytes =
+          active ? (uint32_t)(nh * (n_rec * krow + t_out * krow) + 2 * nh * dts * 4) : 0u;
+      if (lane == 0) {
+        armed[8 + gs] = gi >> 1;
+        mbar_arrive_expect_tx(&gfull[gs], gbytes);
+      }
+      __syncwarp();
+      if (active) {
+        // copies: per head: k ring range, k of each new token, q of each output; alpha rows, beta rows
+        const int per_head = 1 + n_new + t_out;
+        const int ncopy = nh * per_head + 2;
+        for (int q = lane; q < ncopy; q += 32) {
+          if (q == ncopy - 2) {
+            bulk_g2s(gb + lay.gb_a, a.ring_a + ((size_t)b * a.H + h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
+          } else if (q == ncopy - 1) {
+            bulk_g2s(gb + lay.gb_b, a.ring_b + ((size_t)b * a.H + h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
+          } else {
+            const int i = q / per_head, w = q % per_head;
+            const size_t unit = (size_t)b * a.H + h0 + i;
+            unsigned char *kd = gb + lay.gb_k + (size_t)i * lay.rmax * krow;
+            if (w == 0) {
+              if (n_ring)
+                bulk_g2s(kd, reinterpret_cast<const unsigned char *>(a.ring_k) + (unit * 2 * L + base_e) * krow,
+                         n_ring * krow, &gfull[gs], pol_keep);
+            } else if (w <= n_new) {
+              const int t = w - 1;
+              bulk_g2s(kd + (n_ring + t) * krow,
+                       reinterpret_cast<const unsigned char *>(a.k) + (((size_t)b * a.T + t) * a.H + h0 + i) * krow,
+                       krow, &gfull[gs], pol_keep);
+            } else {
+              const int t = w - 1 - n_new;
+              bulk_g2s(gb + lay.gb_q + ((size_t)i * lay.no + t) * krow,
+                       reinterpret_cast<const unsigned char *>(a.q) + (((size_t)b * a.T + t) * a.H + h0 + i) * krow,
+                       krow, &gfull[gs], pol_keep);
+            }
+          }
+        }
+        // ---- tiles: (head, 64-row block)
+        const bool fold = m > 0;
+        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
+                                : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
+        bool ok = true;
+        for (int tt = 0; tt < nh * nrb; ++tt, ++ti) {
+          const int i = tt / nrb, t = tt % nrb;
+          const int rows = min(kFp4Rows, R - kFp4Rows * t);
+          const size_t unit = (size_t)b * a.H + h0 + i;
+          const size_t row_abs = unit * R + (size_t)kFp4Rows * t;  // first state row of the tile
+          const int s = ti % NS;
+          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+            if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+            ok = false;
+            break;
+          }
+          unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          uint32_t tb = (uint32_t)n_rec * vrow;
+          if (srcfmt == SRC_F32) tb += rows * kCols * 4;
+          else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
+          else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
+          if (lane == 0) {
+            armed[s] = ti / NS;
+            mbar_arrive_expect_tx(&full[s], tb);
+          }
+          __syncwarp();
+          if (lane == 0) {
+            if (srcfmt == SRC_F32)
+              bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
+            else if (srcfmt == SRC_F16)
+              bulk_g2s(st, reinterpret_cast<const __half *>(a.hp) + row_abs * kCols, rows * kCols * 2, &full[s], pol_stream);
+            else
+              bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
+          }
+          if (lane == 1 && srcfmt == SRC_FP4)
+            bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
+          if (lane == 2 && srcfmt == SRC_FP4) {
+            const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
+            bulk_g2s(st + lay.st_g, a.rg + gi4, 16, &full[s], pol_keep);
+          }
+          if (lane == 3 && n_ring)
+            bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + base_e) * vrow,
+                     n_ring * vrow, &full[s], pol_keep);
+          if (lane >= 4 && lane < 4 + n_new) {
+            const int tk = lane - 4;
+            bulk_g2s(st + lay.st_v + (n_ring + tk) * vrow,
+                     reinterpret_cast<const unsigned char *>(a.v) + (((size_t)b * a.T + tk) * a.H + h0 + i) * vrow,
+                     vrow, &full[s], pol_keep);
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == kGPrep0 || warp == kGPrep0 + 1) {
+    // ================================================================== prep warps
+    const int pw = warp - kGPrep0;
+    const int sg = pw * 4 + (lane >> 3), sl = lane & 7;       // 8 subgroups of 8 lanes
+    const unsigned smask = 0xFFu << (lane & 24);
+    int rdv = 0;  // rendezvous count (both prep warps take the same ones)
+    auto prep_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(psync);
+      const bool ok = mbar_wait_or_abort(psync, (uint32_t)(rdv & 1), abort_flag);
+      ++rdv;
+      return ok;
+    };
+    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+      const int gs = gi & 1;
+      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+        if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
+      const int *gh = reinterpret_cast<const int *>(gb);
+      float *gf = reinterpret_cast<float *>(gb);
+      const int b = gh[Q_B], h0 = gh[Q_H0], nh = gh[Q_NH];
+      if (pw == 0 && gh[Q_WMETA] && lane == 0) a.meta_out[b] = make_int4(gh[Q_MC], gh[Q_ME], gh[Q_MP], 0);
+      const int active = gh[Q_ACTIVE];
+      const int n_rec = gh[Q_NREC], m = gh[Q_M], n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], t_out = gh[Q_TOUT];
+      const int slot0 = gh[Q_SLOT0], base_e = gh[Q_BASE];
+      if (active) {
+        // alpha, beta of the new tokens (global loads) -> header; append k, alpha, beta to the ring
+        for (int q = pw * 32 + lane; q < n_new * nh; q += 64) {
+          const int t = q / nh, i = q % nh;
+          const size_t tok = ((size_t)b * a.T + t) * a.H + h0 + i;
+          const float al = a.alpha[tok], be = a.beta[tok];
+          gf[Q_F + t * 8 + i] = al;
+          gf[Q_FB + t * 8 + i] = be;
+          const size_t unit = (size_t)b * a.H + h0 + i;
+          a.ring_a[unit * dts + slot0 + t] = al;
+          a.ring_b[unit * dts + slot0 + t] = be;
+        }
+        const int kq = kCols * esz / 16;
+        for (int q = pw * 32 + lane; q < n_new * nh * kq; q += 64) {
+          const int c16 = q % kq, ti2 = q / kq, t = ti2 / nh, i = ti2 % nh;
+          const size_t unit = (size_t)b * a.H + h0 + i;
+          const uint4 v = *reinterpret_cast<const uint4 *>(gb + lay.gb_k + ((size_t)i * lay.rmax + n_ring + t) * kCols * esz + c16 * 16);
+          *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_k) + ((unit * 2 * L + slot0 + t) * kCols) * esz +
+                                     c16 * 16) = v;
+        }
+      }
+      if (!prep_sync()) {  // both prep warps see the header floats
+        if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      if (active) {
+        float *u0t = reinterpret_cast<float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_u0);
+        float *cot = reinterpret_cast<float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_coef);
+        const TI *kg = reinterpret_cast<const TI *>(gb + lay.gb_k);
+        const TI *qg = reinterpret_cast<const TI *>(gb + lay.gb_q);
+        const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
+        const float *bg = reinterpret_cast<const float *>(gb + lay.gb_b);
+        for (int p = sg; p < nh * t_out; p += 8) {
+          const int i = p / t_out, j = p % t_out;
+          const int e_j = n_rec - t_out + j + 1;
+          float u[16];
+          load_k16(qg + ((size_t)i * lay.no + j) * kCols + sl * 16, u);
+          float *co = cot + ((size_t)i * lay.no + j) * lay.rmax;
+          for (int r = sl; r < n_rec; r += 8)
+            if (r < m || r >= e_j) co[r] = 0.f;
+          for (int r = e_j - 1; r >= m; --r) {
+            float kv[16];
+            load_k16(kg + ((size_t)i * lay.rmax + r) * kCols + sl * 16, kv);
+            float c = 0.f;
+#pragma unroll
+            for (int z = 0; z < 16; ++z) c = fmaf(u[z], kv[z], c);
+            c += __shfl_xor_sync(smask, c, 1);
+            c += __shfl_xor_sync(smask, c, 2);
+            c += __shfl_xor_sync(smask, c, 4);
+            const float al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
+            const float be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
+            if (sl == 0) co[r] = a.q_scale * be * c;
+            const float bc = be * c;
+#pragma unroll
+            for (int z = 0; z < 16; ++z) u[z] = al * fmaf(-bc, kv[z], u[z]);
+          }
+          float *ud = u0t + ((size_t)i * lay.no + j) * kCols + sl * 16;
+          const float qs = a.q_scale;
+#pragma unroll
+          for (int z = 0; z < 16; z += 4)
+            *reinterpret_cast<float4 *>(ud + z) = make_float4(qs * u[z], qs * u[z + 1], qs * u[z + 2], qs * u[z + 3]);
+        }
+      }
+      if (!prep_sync()) {  // tables complete
+        if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      if (pw == 0 && lane == 0) mbar_arrive(&tfull[gs]);
+    }
+  } else {
+    // ================================================================== consumer warps
+    const int cg = warp >> 2, wid = warp & 3;
+    int ti = 0, group_rdv = 0;
+    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+      const int gs = gi & 1;
+      if (!mbar_wait_or_abort(&tfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+        if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+        break;
+      }
+      const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
+      const int *gh = reinterpret_cast<const int *>(gb);
+      const float *gf = reinterpret_cast<const float *>(gb);
+      const int b = gh[Q_B], h0 = gh[Q_H0], nh = gh[Q_NH];
+      if (gh[Q_ACTIVE]) {
+        const int n_rec = gh[Q_NREC], m = gh[Q_M], n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], t_out = gh[Q_TOUT];
+        const int slot0 = gh[Q_SLOT0], base_e = gh[Q_BASE], me = gh[Q_ME];
+        const bool fold = m > 0;
+        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
+                                : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
+        const float *u0t = reinterpret_cast<const float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_u0);
+        const float *cot = reinterpret_cast<const float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_coef);
+        float *amx = reinterpret_cast<float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_amax);
+        const TI *kg = reinterpret_cast<const TI *>(gb + lay.gb_k);
+        const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
+        const float *bg = reinterpret_cast<const float *>(gb + lay.gb_b);
+        int fold_tiles = 0;
+        for (int tt = 0; tt < nh * nrb; ++tt, ++ti) {
+          if ((ti & 1) != cg) continue;
+          const int i = tt / nrb, t = tt % nrb;
+          const int rows = min(kFp4Rows, R - kFp4Rows * t);
+          const int h = h0 + i;
+          const size_t unit = (size_t)b * a.H + h;
+          const int s = ti % NS;
+          if (!mbar_wait_or_abort(&full[s], (uint32_t)((ti / NS) & 1), abort_flag)) {
+            if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+            break;
+          }
+          const unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          const TI *vr = reinterpret_cast<const TI *>(st + lay.st_v);
+          const float g_tile = reinterpret_cast<const float *>(st + lay.st_g)[(unit * nrb + t) & 3];
+          const float *co_h = cot + (size_t)i * lay.no * lay.rmax;
+          const float *u0_h = u0t + (size_t)i * lay.no * kCols;
+          if (!fold) {
+            // ---------------- non-fold tile: lane owns columns 4l..4l+3 of 16 rows
+            float4 uv[NO];
+#pragma unroll
+            for (int j = 0; j < NO; ++j)
+              uv[j] = (j < t_out) ? *reinterpret_cast<const float4 *>(u0_h + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
+            constexpr int V = 8 * NO;
+            constexpr int KEEP = V >= 32 ? V / 32 : 1;
+            constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
+#pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
+              const int r0 = wid * 16 + pass * 8;
+              if (r0 >= rows) break;
+              float part[V];
+#pragma unroll
+              for (int rr = 0; rr < 8; ++rr) {
+                const int row = r0 + rr;
+                float4 sv;
+                if (srcfmt == SRC_F32) {
+                  sv = *reinterpret_cast<const float4 *>(st + (row * kCols + 4 * lane) * 4);
+                } else if (srcfmt == SRC_F16) {
+                  const uint2 hv = *reinterpret_cast<const uint2 *>(st + (row * kCols + 4 * lane) * 2);
+                  const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.x));
+                  const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.y));
+                  sv = make_float4(f0.x, f0.y, f1.x, f1.y);
+                } else {
+                  const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + 2 * lane);
+                  const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + (lane >> 2)];
+                  const float d_b = __fmul_rn(e4m3_value(sc), g_tile);
+                  sv = make_float4(nvfp4_value(cw & 15u, d_b), nvfp4_value((cw >> 4) & 15u, d_b),
+                                   nvfp4_value((cw >> 8) & 15u, d_b), nvfp4_value((cw >> 12) & 15u, d_b));
+                }
+#pragma unroll
+                for (int j = 0; j < NO; ++j)
+                  part[rr * NO + j] = sv.x * uv[j].x + sv.y * uv[j].y + sv.z * uv[j].z + sv.w * uv[j].w;
+              }
+              // buffered part: lane r adds coef_{j,r} v_r[row] for the 8 rows (one 16-byte load of v_r)
+              for (int r = lane; r < n_rec; r += 32) {
+                float vv[8];
+                load8(vr + r * R + kFp4Rows * t + r0, vv);
+#pragma unroll
+                for (int j = 0; j < NO; ++j) {
+                  const float co = (j < t_out) ? co_h[j * lay.rmax + r] : 0.f;
+#pragma unroll
+                  for (int rr = 0; rr < 8; ++rr) part[rr * NO + j] = fmaf(co, vv[rr], part[rr * NO + j]);
+                }
+              }
+              warp_transpose_reduce<V>(part, lane);
+#pragma unroll
+              for (int k2 = 0; k2 < KEEP; ++k2) {
+                const int idx = (V >= 32) ? lane * KEEP + k2 : lane / SPREAD;
+                const int rr = idx / NO, j = idx % NO;
+                const int row = r0 + rr;
+                if (j < t_out && row < rows && (lane % SPREAD) == 0)
+                  a.y[(((size_t)b * a.T + j) * a.H + h) * R + kFp4Rows * t + row] = part[k2];
+              }
+            }
+          } else {
+            // ---------------- fold tile: two lanes per row, 64 columns each (chunks rotated by lane)
+            const int row = wid * 16 + (lane >> 1), half = lane & 1;
+            const bool live = row < rows;
+            const int rowg = kFp4Rows * t + row;  // row within the head's state
+            float4 sv[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const int ch2 = (q + lane) & 15;
+              const int col = half * 64 + ch2 * 4;
+              float4 v4 = make_float4(0, 0, 0, 0);
+              if (live) {
+                if (srcfmt == SRC_F32) {
+                  v4 = *reinterpret_cast<const float4 *>(st + (row * kCols + col) * 4);
+                } else if (srcfmt == SRC_F16) {
+                  const uint2 hv = *reinterpret_cast<const uint2 *>(st + (row * kCols + col) * 2);
+                  const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.x));
+                  const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.y));
+                  v4 = make_float4(f0.x, f0.y, f1.x, f1.y);
+                } else {
+                  const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + col / 2);
+                  const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + col / 16];
+                  const float d_b = __fmul_rn(e4m3_value(sc), g_tile);
+                  v4 = make_float4(nvfp4_value(cw & 15u, d_b), nvfp4_value((cw >> 4) & 15u, d_b),
+                                   nvfp4_value((cw >> 8) & 15u, d_b), nvfp4_value((cw >> 12) & 15u, d_b));
+                }
+              }
+              sv[q] = v4;
+            }
+            // sequential row update over the folded records
+            for (int r = 0; r < m; ++r) {
+              const TI *kr = kg + ((size_t)i * lay.rmax + r) * kCols + half * 64;
+              float d = 0.f;
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const float4 kv = load4(kr + ((q + lane) & 15) * 4);
+                d = fmaf(sv[q].x, kv.x, fmaf(sv[q].y, kv.y, fmaf(sv[q].z, kv.z, fmaf(sv[q].w, kv.w, d))));
+              }
+              d += __shfl_xor_sync(0xffffffffu, d, 1);
+              const float al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
+              const float be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
+              const float vrow = live ? to_f32(vr[r * R + rowg]) : 0.f;
+              const float coef = be * (vrow - al * d);
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const float4 kv = load4(kr + ((q + lane) & 15) * 4);
+                sv[q].x = fmaf(al, sv[q].x, coef * kv.x);
+                sv[q].y = fmaf(al, sv[q].y, coef * kv.y);
+                sv[q].z = fmaf(al, sv[q].z, coef * kv.z);
+                sv[q].w = fmaf(al, sv[q].w, coef * kv.w);
+              }
+            }
+            // outputs from the fp32 fold result
+            for (int j = 0; j < t_out; ++j) {
+              const float *uj = u0_h + j * kCols + half * 64;
+              float z = 0.f;
+#pragma unroll
+              for (int q = 0; q < 16; ++q) {
+                const float4 uv = *reinterpret_cast<const float4 *>(uj + ((q + lane) & 15) * 4);
+                z = fmaf(sv[q].x, uv.x, fmaf(sv[q].y, uv.y, fmaf(sv[q].z, uv.z, fmaf(sv[q].w, uv.w, z))));
+              }
+              z += __shfl_xor_sync(0xffffffffu, z, 1);
+              const int e_j = n_rec - t_out + j + 1;
+              float acc = 0.f;
+              if (live)
+                for (int r = m + half; r < e_j; r += 2) acc = fmaf(co_h[j * lay.rmax + r], to_f32(vr[r * R + rowg]), acc);
+              acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+              if (live && half == 0) a.y[(((size_t)b * a.T + j) * a.H + h) * R + rowg] = z + acc;
+            }
+            // write the new state: checkpoint format, then the NVFP4 copy
+            if (live && !shared_fp4) {
+              if (!hp16) {
+                float *dst = reinterpret_cast<float *>(a.hp) + (unit * R + rowg) * kCols + half * 64;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) __stcs(reinterpret_cast<float4 *>(dst + ((q + lane) & 15) * 4), sv[q]);
+              } else {
+                __half *dst = reinterpret_cast<__half *>(a.hp) + (unit * R + rowg) * kCols + half * 64;
+                const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                  const int ch2 = (q + lane) & 15;
+                  const uint32_t elem = (uint32_t)(rowg * kCols + half * 64 + ch2 * 4);
+                  const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
+                  const __half h0v = fp16_sr(sv[q].x, rw.x), h1v = fp16_sr(sv[q].y, rw.y);
+                  const __half h2v = fp16_sr(sv[q].z, rw.z), h3v = fp16_sr(sv[q].w, rw.w);
+                  uint2 pk;
+                  pk.x = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
+                  pk.y = (uint32_t)__half_as_ushort(h2v) | ((uint32_t)__half_as_ushort(h3v) << 16);
+                  *reinterpret_cast<uint2 *>(dst + ch2 * 4) = pk;
+                }
+              }
+            }
+            if (fp4_read) {
+              float am = 0.f;
+#pragma unroll
+              for (int q = 0; q < 16; ++q)
+                am = fmaxf(am, fmaxf(fmaxf(fabsf(sv[q].x), fabsf(sv[q].y)), fmaxf(fabsf(sv[q].z), fabsf(sv[q].w))));
+#pragma unroll
+              for (int off = 16; off >= 1; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+              const int slot = fold_tiles & 1;
+              if (lane == 0) amx[(cg * 2 + slot) * 4 + wid] = am;
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&csync[cg]);  // the group's four warps have posted their maxima
+              if (!mbar_wait_or_abort(&csync[cg], (uint32_t)(group_rdv & 1), abort_flag)) {
+                if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+                break;
+              }
+              ++group_rdv;
+              const float tmax = fmaxf(fmaxf(amx[(cg * 2 + slot) * 4 + 0], amx[(cg * 2 + slot) * 4 + 1]),
+                                       fmaxf(amx[(cg * 2 + slot) * 4 + 2], amx[(cg * 2 + slot) * 4 + 3]));
+              const float g = nvfp4_tile_scale(tmax);
+              if (wid == 0 && lane == 0) a.rg[unit * nrb + t] = g;
+              if (live) {
+                // blocks of 16 columns = 4 chunks; this lane holds blocks half*4 .. half*4+3
+                float bam[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                  const int ch2 = (q + lane) & 15;
+                  const float mq = fmaxf(fmaxf(fabsf(sv[q].x), fabsf(sv[q].y)), fmaxf(fabsf(sv[q].z), fabsf(sv[q].w)));
+#pragma unroll
+                  for (int blk = 0; blk < 4; ++blk)
+                    if ((ch2 >> 2) == blk) bam[blk] = fmaxf(bam[blk], mq);
+                }
+                float db[4];
+                uint32_t scw = 0;
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) scw |= nvfp4_block_scale(bam[blk], g, &db[blk]) << (8 * blk);
+                *reinterpret_cast<uint32_t *>(a.rs + (unit * R + rowg) * (kCols / 16) + half * 4) = scw;
+                unsigned char *cd = a.rq + (unit * R + rowg) * (kCols / 2) + half * 32;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                  const int ch2 = (q + lane) & 15;
+                  float d_b = db[0];
+#pragma unroll
+                  for (int blk = 1; blk < 4; ++blk)
+                    if ((ch2 >> 2) == blk) d_b = db[blk];
+                  const uint32_t cw = nvfp4_code(sv[q].x, d_b) | (nvfp4_code(sv[q].y, d_b) << 4) |
+                                      (nvfp4_code(sv[q].z, d_b) << 8) | (nvfp4_code(sv[q].w, d_b) << 12);
+                  *reinterpret_cast<uint16_t *>(cd + ch2 * 2) = (uint16_t)cw;
+                }
+              }
+              ++fold_tiles;
+            }
+          }
+          // append this head's new v rows (once per head, by the group that owns its first tile)
+          if (t == 0 && wid == 0 && n_new) {
+            const int vq = R * esz / 16;
+            for (int q = lane; q < n_new * vq; q += 32) {
+              const int tk = q / vq, c16 = q % vq;
+              const uint4 v = *reinterpret_cast<const uint4 *>(st + lay.st_v + (n_ring + tk) * R * esz + c16 * 16);
+              *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_v) +
+                                         ((unit * 2 * L + slot0 + tk) * R) * esz + c16 * 16) = v;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+        }
+      }
+      if (*abort_flag) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gempty[gs]);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int s = 0; s < 8; ++s)
+      if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1));
+    for (int s = 0; s < 2; ++s)
+      if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
+  }
+}
+
+}  // namespace
+
+int g_smem_bytes(int R, int L, int tmax, int esz, int nstage) {
+  const GLayout l = g_layout(R, L, tmax, esz);
+  return kBarBytesG + 2 * l.tab_bytes + 2 * l.gb_bytes + nstage * l.stage_bytes;
+}
+
+int g_max_stages(int R, int L, int tmax, int esz, int budget) {
+  int n = 8;
+  while (n > 2 && g_smem_bytes(R, L, tmax, esz, n) > budget) --n;
+  return n;
+}
+
+int g_units(int Bt, int H, int tmax) {
+  const int no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
+  const int hg = g_heads_per_unit(no);
+  return Bt * ((H + hg - 1) / hg);
+}
+
+cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream) {
+  const int no = a.tmax <= 1 ? 1 : a.tmax <= 2 ? 2 : a.tmax <= 4 ? 4 : 8;
+  const size_t smem = g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage);
+  void (*kern)(GArgs) = nullptr;
+#define RSSM_PICK(TI, NOV) \
+  if (no == NOV) kern = gdn_replay_kernel<TI, NOV>;
+  if (esz == 2) {
+    RSSM_PICK(__nv_bfloat16, 1) RSSM_PICK(__nv_bfloat16, 2) RSSM_PICK(__nv_bfloat16, 4) RSSM_PICK(__nv_bfloat16, 8)
+  } else {
+    RSSM_PICK(float, 1) RSSM_PICK(float, 2) RSSM_PICK(float, 4) RSSM_PICK(float, 8)
+  }
+#undef RSSM_PICK
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  kern<<<a.grid, kGdnThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace rssm

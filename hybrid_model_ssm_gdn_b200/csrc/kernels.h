@@ -43,7 +43,7 @@ struct GArgs {
   int *err;
   void *hp;                       // fp32 or fp16 [Bt][H][DV][128]
   unsigned char *rq, *rs;         // NVFP4 codes [Bt][H][DV][64], scales [Bt][H][DV][8]
-  float *rg;                      // tile scales [Bt][H]
+  float *rg;                      // tile scales [Bt][H][ceil(DV/64)]
   void *ring_k, *ring_v;          // input dtype [Bt][H][2L][128], [Bt][H][2L][DV]
   float *ring_a, *ring_b;         // alpha, beta [Bt][H][dt_stride(L)]
   const void *q, *k, *v;          // [Bt][T][H][128], [Bt][T][H][128], [Bt][T][H][DV]
@@ -51,8 +51,9 @@ struct GArgs {
   const unsigned char *mask;
   float *y;                       // [Bt][T][H][DV]
 };
-int g_stage_bytes(const GArgs &a, int esz);
-int g_table_bytes(const GArgs &a);
+int g_smem_bytes(int R, int L, int tmax, int esz, int nstage);
+int g_max_stages(int R, int L, int tmax, int esz, int budget);
+int g_units(int Bt, int H, int tmax);  // work units: (sequence, chunk of heads)
 cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream);
 
 // small kernels (bookkeeping, load, export)

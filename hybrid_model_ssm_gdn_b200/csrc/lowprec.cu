@@ -1,13 +1,111 @@
-// lowprec.cu -- precision converters (placeholder until the converters land).
+// lowprec.cu -- stand-alone precision converters: write a loaded fp32 checkpoint in the
+// stored formats (fp32 or fp16 with stochastic rounding at epoch 0, plus the NVFP4 read
+// copy) and widen the stored checkpoint back to fp32 for export.  The rounding rules are
+// those of lowprec.cuh.  One block of 64 threads per 64-row tile of a head's state;
+// thread r owns row r (128 columns).
 #include "kernels.h"
+#include "lowprec.cuh"
 
 namespace rssm {
-cudaError_t launch_store_state(const float *, void *, int, unsigned char *, unsigned char *, float *, int, int, int,
-                               unsigned long long, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+namespace {
+
+__global__ void store_state_kernel(const float *S, void *hp, int hp_mode, unsigned char *rq, unsigned char *rs,
+                                   float *rg, int read_mode, int rows_per_head, unsigned long long seed) {
+  const int nrb = (rows_per_head + kFp4Rows - 1) / kFp4Rows;
+  const size_t unit = blockIdx.x / nrb;
+  const int t = blockIdx.x % nrb;
+  const int rows = min(kFp4Rows, rows_per_head - kFp4Rows * t);
+  const int row = threadIdx.x;
+  const bool live = row < rows;
+  const int rowg = kFp4Rows * t + row;
+  const float *src = S + (unit * rows_per_head + rowg) * kCols;
+  __shared__ float red[64];
+  float am = 0.f;
+  if (live)
+    for (int c = 0; c < kCols; ++c) am = fmaxf(am, fabsf(src[c]));
+  if (read_mode != RSSM_READ_SHARED_NVFP4 && live) {
+    if (hp_mode == RSSM_HP_F32) {
+      float *dst = reinterpret_cast<float *>(hp) + (unit * rows_per_head + rowg) * kCols;
+      for (int c = 0; c < kCols; ++c) dst[c] = src[c];
+    } else {
+      __half *dst = reinterpret_cast<__half *>(hp) + (unit * rows_per_head + rowg) * kCols;
+      for (int c = 0; c < kCols; c += 4) {
+        const uint32_t elem = (uint32_t)(rowg * kCols + c);
+        const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, 0u, elem >> 2, 0u), (uint32_t)seed,
+                                       (uint32_t)(seed >> 32));
+        dst[c] = fp16_sr(src[c], rw.x);
+        dst[c + 1] = fp16_sr(src[c + 1], rw.y);
+        dst[c + 2] = fp16_sr(src[c + 2], rw.z);
+        dst[c + 3] = fp16_sr(src[c + 3], rw.w);
+      }
+    }
+  }
+  if (read_mode == RSSM_READ_SAME) return;
+  red[row] = am;
+  __syncthreads();
+  float tmax = 0.f;
+  for (int r = 0; r < kFp4Rows; ++r) tmax = fmaxf(tmax, red[r]);
+  const float g = nvfp4_tile_scale(tmax);
+  if (row == 0) rg[unit * nrb + t] = g;
+  if (!live) return;
+  for (int blk = 0; blk < kCols / 16; ++blk) {
+    float bam = 0.f;
+    for (int c = 0; c < 16; ++c) bam = fmaxf(bam, fabsf(src[blk * 16 + c]));
+    float d_b;
+    rs[(unit * rows_per_head + rowg) * (kCols / 16) + blk] = (unsigned char)nvfp4_block_scale(bam, g, &d_b);
+    for (int c = 0; c < 16; c += 2) {
+      const uint32_t lo = nvfp4_code(src[blk * 16 + c], d_b), hi = nvfp4_code(src[blk * 16 + c + 1], d_b);
+      rq[(unit * rows_per_head + rowg) * (kCols / 2) + (blk * 16 + c) / 2] = (unsigned char)(lo | (hi << 4));
+    }
+  }
 }
-cudaError_t launch_widen_state(const void *, int, const unsigned char *, const unsigned char *, const float *, int,
-                               float *, int, int, cudaStream_t) {
-  return cudaErrorNotSupported;
+
+__global__ void widen_state_kernel(const void *hp, int hp_mode, const unsigned char *rq, const unsigned char *rs,
+                                   const float *rg, int read_mode, float *out, int rows_per_head) {
+  const int nrb = (rows_per_head + kFp4Rows - 1) / kFp4Rows;
+  const size_t unit = blockIdx.x / nrb;
+  const int t = blockIdx.x % nrb;
+  const int rows = min(kFp4Rows, rows_per_head - kFp4Rows * t);
+  const int row = threadIdx.x;
+  if (row >= rows) return;
+  const size_t r = unit * rows_per_head + kFp4Rows * t + row;
+  float *dst = out + r * kCols;
+  if (read_mode == RSSM_READ_SHARED_NVFP4) {
+    const float g = rg[unit * nrb + t];
+    for (int blk = 0; blk < kCols / 16; ++blk) {
+      const float d_b = __fmul_rn(e4m3_value(rs[r * (kCols / 16) + blk]), g);
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t byte = rq[r * (kCols / 2) + (blk * 16 + c) / 2];
+        dst[blk * 16 + c] = nvfp4_value(((c & 1) ? (byte >> 4) : byte) & 15u, d_b);
+      }
+    }
+  } else if (hp_mode == RSSM_HP_F16_SR) {
+    const __half *src = reinterpret_cast<const __half *>(hp) + r * kCols;
+    for (int c = 0; c < kCols; ++c) dst[c] = __half2float(src[c]);
+  } else {
+    const float *src = reinterpret_cast<const float *>(hp) + r * kCols;
+    for (int c = 0; c < kCols; ++c) dst[c] = src[c];
+  }
 }
+
+}  // namespace
+
+cudaError_t launch_store_state(const float *S, void *hp, int hp_mode, unsigned char *rq, unsigned char *rs, float *rg,
+                               int read_mode, int units, int rows, unsigned long long seed, int /*H*/,
+                               cudaStream_t stream) {
+  const int nrb = (rows + kFp4Rows - 1) / kFp4Rows;
+  store_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(S, hp, hp_mode, rq, rs, rg, read_mode,
+                                                                                 rows, seed);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_widen_state(const void *hp, int hp_mode, const unsigned char *rq, const unsigned char *rs,
+                               const float *rg, int read_mode, float *out, int units, int rows, cudaStream_t stream) {
+  const int nrb = (rows + kFp4Rows - 1) / kFp4Rows;
+  widen_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(hp, hp_mode, rq, rs, rg, read_mode, out,
+                                                                                 rows);
+  return cudaGetLastError();
+}
+
 }  // namespace rssm

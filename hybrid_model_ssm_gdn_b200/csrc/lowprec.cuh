@@ -1,0 +1,128 @@
+// lowprec.cuh -- device-side number formats of the separate-precision mode.
+//
+// The recurrence checkpoint and the copy read for outputs may use different
+// precisions so that the read copy's rounding never re-enters the recurrence
+// ("Hybrid-model decoding has a new bottleneck", Interpretation, fourth paragraph);
+// the pages name an FP16 recurrence with stochastic rounding (same page, Perspective,
+// second paragraph) and NVFP4 reads (E2M1 values, an E4M3 scale per 16-element
+// block).  Rounding rules, all exact integer or IEEE-fp32 procedures:
+//
+// * FP16 stochastic rounding of fp32 x with a 32-bit word r: with u the fp16 spacing
+//   at |x| (2^(floor(log2|x|)-10), or 2^-24 below 2^-14) and |x| = (q + f) u, round
+//   up to (q+1) u iff r < floor(f * 2^32); keep the sign; saturate at 65504.
+// * E4M3 (OCP FP8 E4M3FN) and E2M1 (OCP FP4): round to nearest, ties to even,
+//   saturating at 448 and 6.
+// * NVFP4 tile (64 consecutive rows x 128 columns of one head's state), blocks of 16
+//   columns: g = amax(tile)/2688 (1 if amax = 0); s_b = E4M3(amax_b / (6 g));
+//   d_b = s_b g; code = sign | E2M1(|x| / d_b) (all zero if s_b = 0); value = E2M1 * d_b.
+// * Random words: Philox4x32-10 (Salmon, Moraes, Dror & Shaw, SC'11), counter
+//   (sequence*H + head, epoch written, element/4, 0), key = the 64-bit seed; element e
+//   uses output word e % 4.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace rssm {
+
+constexpr int kFp4Rows = 64;  // rows of one NVFP4 tile (one row block of a head's state)
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Stochastic rounding of fp32 x to fp16 with the uniform word r (see the rule above).
+__device__ __forceinline__ __half fp16_sr(float x, uint32_t r) {
+  const uint32_t bits = __float_as_uint(x);
+  const uint32_t sign = bits >> 31;
+  const int E = (int)((bits >> 23) & 0xFFu);
+  const uint32_t mant = bits & 0x7FFFFFu;
+  if (E == 255) return mant ? __ushort_as_half(0x7E00) : __ushort_as_half(sign ? 0xFBFF : 0x7BFF);
+  const uint32_t M = E ? (mant | 0x800000u) : mant;  // |x| = M * 2^(Eeff - 150)
+  const int Eeff = E ? E : 1;
+  const int s = max(13, 126 - Eeff);                  // fp32 bits below the fp16 spacing
+  uint32_t q, F;
+  if (s >= 24) { q = 0; F = M; } else { q = M >> s; F = M & ((1u << s) - 1u); }
+  uint64_t thr;
+  if (s <= 32) thr = (uint64_t)F << (32 - s);
+  else if (s - 32 < 24) thr = (uint64_t)(F >> (s - 32));
+  else thr = 0;
+  const uint32_t up = ((uint64_t)r < thr) ? 1u : 0u;
+  const int ulp_exp = max(Eeff - 127, -14) - 10;
+  float mag = ldexpf((float)(q + up), ulp_exp);     // exact: an integer <= 2^11 times a power of two
+  mag = fminf(mag, 65504.f);
+  return __float2half_rn(sign ? -mag : mag);          // exact: the value lies on the fp16 grid
+}
+
+// E4M3FN round-to-nearest-even of v >= 0, saturating at 448 (value, not code).
+__device__ __forceinline__ float e4m3_round(float v) {
+  if (v >= 448.f) return 448.f;
+  if (v < 0.015625f) return rintf(v * 512.f) * (1.f / 512.f);  // subnormal spacing 2^-9
+  int e;
+  frexpf(v, &e);                                                 // v = m 2^e, m in [0.5, 1)
+  return ldexpf(rintf(ldexpf(v, 4 - e)), e - 4);                 // spacing 2^(floor(log2 v) - 3)
+}
+
+__device__ __forceinline__ uint32_t e4m3_code(float q) {  // q >= 0 on the E4M3 grid
+  if (q < 0.015625f) return (uint32_t)(q * 512.f);
+  int e;
+  frexpf(q, &e);
+  const int E = e - 1 + 7;
+  const uint32_t m = (uint32_t)ldexpf(q, 4 - e) - 8u;
+  return ((uint32_t)E << 3) | m;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const uint32_t ef = (code >> 3) & 0xFu, m = code & 7u;
+  return ef == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8u + m), (int)ef - 10);
+}
+
+// E2M1 magnitude index (0..7 for {0, .5, 1, 1.5, 2, 3, 4, 6}) of y >= 0, ties to even index.
+__device__ __forceinline__ uint32_t e2m1_index(float y) {
+  uint32_t n;
+  if (y < 2.f) n = (uint32_t)rintf(y * 2.f);
+  else if (y < 4.f) n = (uint32_t)rintf(y) + 2u;
+  else n = (uint32_t)rintf(y * 0.5f) + 4u;
+  return n > 7u ? 7u : n;
+}
+
+__device__ __forceinline__ float e2m1_value(uint32_t idx) {
+  // {0, .5, 1, 1.5, 2, 3, 4, 6}
+  const float lo = (float)idx * 0.5f;           // exact for idx <= 4
+  return idx <= 4u ? lo : (idx == 5u ? 3.f : (idx == 6u ? 4.f : 6.f));
+}
+
+// NVFP4 tile scale from the tile's largest magnitude.
+__device__ __forceinline__ float nvfp4_tile_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f; }
+
+// Block scale code and the block's dequantisation step d_b = s_b * g.
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax_b, float g, float *d_b) {
+  const float t = __fmul_rn(6.f, g);
+  const float sb = e4m3_round(__fdiv_rn(amax_b, t));
+  *d_b = __fmul_rn(sb, g);
+  return e4m3_code(sb);
+}
+
+// 4-bit code of x in a block with step d_b (d_b == 0 when the block scale is zero).
+__device__ __forceinline__ uint32_t nvfp4_code(float x, float d_b) {
+  if (d_b == 0.f) return 0u;
+  const uint32_t idx = e2m1_index(__fdiv_rn(fabsf(x), d_b));
+  return idx | (x < 0.f ? 8u : 0u);
+}
+
+__device__ __forceinline__ float nvfp4_value(uint32_t code, float d_b) {
+  const float v = __fmul_rn(e2m1_value(code & 7u), d_b);
+  return (code & 8u) ? -v : v;
+}
+
+}  // namespace rssm

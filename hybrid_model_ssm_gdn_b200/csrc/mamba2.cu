@@ -74,8 +74,9 @@ __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
   return l;
 }
 
-// barriers: full[8], empty[8], gfull[2], gempty[2], tfull[2]; then armed phase per barrier (ints)
+// barriers: full[8], empty[8], gfull[3], gempty[3], tfull[2], tempty[2]; then armed phases (ints)
 constexpr int kBarBytes = 256;
+constexpr int kGB = 3;  // group buffers: the producer loads a unit's group data one unit ahead
 constexpr int kM2Threads = kConsumers + 64;  // + producer warp + prep warp
 constexpr int kProducerWarp = kConsumerWarps, kPrepWarp = kConsumerWarps + 1;
 
@@ -87,15 +88,16 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   const int NS = a.nstage;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + 8;
-  uint64_t *gfull = empty + 8;
-  uint64_t *gempty = gfull + 2;
-  uint64_t *tfull = gempty + 2;
-  volatile int *armed = reinterpret_cast<volatile int *>(tfull + 2);  // [10]: last armed phase of full[0..7], gfull[0..1]
-  volatile int *abort_flag = armed + 10;
+  uint64_t *gfull = empty + 8;    // [kGB] group data landed
+  uint64_t *gempty = gfull + kGB; // [kGB] consumers done with a unit's group data
+  uint64_t *tfull = gempty + kGB; // [2] tables ready
+  uint64_t *tempty = tfull + 2;   // [2] consumers done with the tables
+  volatile int *armed = reinterpret_cast<volatile int *>(tempty + 2);  // last armed phase of full[0..7], gfull[..]
+  volatile int *abort_flag = armed + 8 + kGB;
   const int rmax = lay.rmax;
   unsigned char *tabs = smem + kBarBytes;  // two table buffers
   unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
-  unsigned char *stages = gbuf + 2 * lay.gb_bytes;
+  unsigned char *stages = gbuf + kGB * lay.gb_bytes;
   struct Tables {
     float *g, *coef, *ao, *wf, *af;
   };
@@ -121,12 +123,15 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kGB; ++s) {
       mbar_init(&gfull[s], 1);
       mbar_init(&gempty[s], kConsumerWarps);
-      mbar_init(&tfull[s], 1);
     }
-    for (int s = 0; s < 10; ++s) armed[s] = -1;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], kConsumerWarps);
+    }
+    for (int s = 0; s < 8 + kGB; ++s) armed[s] = -1;
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -138,34 +143,38 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     const uint64_t pol_keep = policy_evict_last();
     const uint32_t xrow = (uint32_t)a.P * esz, brow = (uint32_t)kCols * esz;
     const int L = a.L, dts = dt_stride(L);
-    int cached_b = -1, msk = 1;
-    int4 meta = make_int4(0, 0, 0, 0);
-    int ti = 0;
-    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
-      const int b = u / (a.G * chunks);
-      const int g = (u / chunks) % a.G;
-      const int ch = u % chunks;
-      const int h0 = g * hpg + ch * kHG;
-      const int nh = min(kHG, hpg - ch * kHG);
-      if (b != cached_b) {
-        if (lane == 0) {
-          meta = a.meta_in[b];
-          msk = (a.mask == nullptr) ? 1 : (int)a.mask[b];
+    // bookkeeping words: lane q holds sequence (first + q) of the block's range, loaded up front
+    // (and refreshed every 32 sequences) so the issue loop never waits on a global load
+    const int b_first = u_begin / (a.G * chunks);
+    int mw_base = -1;
+    int4 mw = make_int4(0, 0, 0, 0);
+    int mk = 1;
+    struct Sched {
+      int b, g, h0, nh, active, n_ring, n_new, m, t_out, slot0, base_e;
+    };
+    // schedule of unit u (identical for every head of the sequence); loads nothing but the
+    // prefetched bookkeeping words
+    auto schedule = [&](int u, Sched &S, int *hdr) {
+      const int b = u / (a.G * chunks), g = (u / chunks) % a.G, ch = u % chunks;
+      S.b = b; S.g = g; S.h0 = g * hpg + ch * kHG; S.nh = min(kHG, hpg - ch * kHG);
+      const int base32 = b_first + ((b - b_first) & ~31);
+      if (base32 != mw_base) {
+        const int bq = base32 + lane;
+        if (bq < a.Bt) {
+          mw = a.meta_in[bq];
+          mk = (a.mask == nullptr) ? 1 : (int)a.mask[bq];
         }
-        meta.x = __shfl_sync(0xffffffffu, meta.x, 0);
-        meta.y = __shfl_sync(0xffffffffu, meta.y, 0);
-        meta.z = __shfl_sync(0xffffffffu, meta.z, 0);
-        msk = __shfl_sync(0xffffffffu, msk, 0);
-        cached_b = b;
+        mw_base = base32;
       }
-      const int c = meta.x, e = meta.y, pend = meta.z;
-      // ---- schedule of this sequence for this call
+      const int src = b - base32;
+      const int c = __shfl_sync(0xffffffffu, mw.x, src), e = __shfl_sync(0xffffffffu, mw.y, src);
+      const int pend = __shfl_sync(0xffffffffu, mw.z, src), msk = __shfl_sync(0xffffffffu, mk, src);
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
       int mc = c, me = e, mp = pend;
       const int base_e = (e & 1) * L, base_n = ((e + 1) & 1) * L;
       if (pend != 0) {
         active = 0;
-        if (h0 == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
+        if (S.h0 == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
       } else if (a.op == OP_STEP) {
         n_new = 1;
         t_out = 1;
@@ -184,104 +193,123 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         if (!msk || c == 0) active = 0;
         else { n_ring = c; m = c; mc = 0; me = e + 1; }
       }
-      const int n_rec = n_ring + n_new;
-      // ---- group buffer
-      const int gs = gi & 1;
-      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
-        if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
-        break;
+      S.active = active; S.n_ring = n_ring; S.n_new = n_new; S.m = m; S.t_out = t_out; S.slot0 = slot0;
+      S.base_e = base_e;
+      if (hdr != nullptr && lane == 0) {
+        hdr[G_ACTIVE] = active; hdr[G_NREC] = n_ring + n_new; hdr[G_M] = m; hdr[G_NRING] = n_ring;
+        hdr[G_NNEW] = n_new; hdr[G_TOUT] = t_out; hdr[G_SLOT0] = slot0; hdr[G_MC] = mc; hdr[G_ME] = me;
+        hdr[G_MP] = mp; hdr[G_B] = b; hdr[G_G] = g; hdr[G_H0] = S.h0; hdr[G_NH] = S.nh; hdr[G_BASE] = base_e;
+        hdr[G_WMETA] = (S.h0 == 0); hdr[G_WB] = (ch == 0);
       }
+    };
+    // group data of unit u into buffer u % kGB (B records, B and C of the new tokens, dt rows)
+    auto issue_group = [&](int u, int gi) -> bool {
+      const int gs = gi % kGB;
+      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGB) & 1) ^ 1), abort_flag)) return false;
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
-      int *gh = reinterpret_cast<int *>(gb);
-      float *gf = reinterpret_cast<float *>(gb);
-      if (lane == 0) {
-        gh[G_ACTIVE] = active; gh[G_NREC] = n_rec; gh[G_M] = m; gh[G_NRING] = n_ring; gh[G_NNEW] = n_new;
-        gh[G_TOUT] = t_out; gh[G_SLOT0] = slot0; gh[G_MC] = mc; gh[G_ME] = me; gh[G_MP] = mp;
-        gh[G_B] = b; gh[G_G] = g; gh[G_H0] = h0; gh[G_NH] = nh; gh[G_BASE] = base_e;
-        gh[G_WMETA] = (h0 == 0); gh[G_WB] = (ch == 0);
-      }
-      if (lane < nh) {
-        gf[G_A + lane] = a.A[h0 + lane];
-        gf[G_D + lane] = a.D[h0 + lane];
-      }
-      if (active) {
-        for (int q = lane; q < n_new * nh; q += 32) {
-          const int t = q / nh, i = q % nh;
-          gf[G_DT + t * kHG + i] = to_f32(reinterpret_cast<const TI *>(a.dt)[((size_t)b * a.T + t) * a.H + h0 + i]);
-        }
-      }
+      Sched S;
+      schedule(u, S, reinterpret_cast<int *>(gb));
       __syncwarp();
-      const uint32_t gbytes = active ? (uint32_t)(n_rec * brow + t_out * brow + nh * dts * 4) : 0u;
+      const int n_rec = S.n_ring + S.n_new;
+      const uint32_t gbytes = S.active ? (uint32_t)(n_rec * brow + S.t_out * brow + S.nh * dts * 4) : 0u;
       if (lane == 0) {
-        armed[8 + gs] = gi >> 1;
+        armed[8 + gs] = gi / kGB;
         mbar_arrive_expect_tx(&gfull[gs], gbytes);
       }
       __syncwarp();
-      if (active) {
-        if (lane == 0 && n_ring)
+      if (S.active) {
+        if (lane == 0 && S.n_ring)
           bulk_g2s(gb + lay.gb_B,
-                   reinterpret_cast<const unsigned char *>(a.ring_B) + (((size_t)b * a.G + g) * 2 * L + base_e) * brow,
-                   n_ring * brow, &gfull[gs], pol_keep);
+                   reinterpret_cast<const unsigned char *>(a.ring_B) + (((size_t)S.b * a.G + S.g) * 2 * L + S.base_e) * brow,
+                   S.n_ring * brow, &gfull[gs], pol_keep);
         if (lane == 1)
-          bulk_g2s(gb + lay.gb_dt, a.ring_dt + ((size_t)b * a.H + h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
-        if (lane >= 4 && lane < 4 + n_new) {
+          bulk_g2s(gb + lay.gb_dt, a.ring_dt + ((size_t)S.b * a.H + S.h0) * dts, S.nh * dts * 4, &gfull[gs], pol_keep);
+        if (lane >= 4 && lane < 4 + S.n_new) {
           const int t = lane - 4;
-          bulk_g2s(gb + lay.gb_B + (n_ring + t) * brow,
-                   reinterpret_cast<const unsigned char *>(a.Bin) + (((size_t)b * a.T + t) * a.G + g) * brow, brow,
+          bulk_g2s(gb + lay.gb_B + (S.n_ring + t) * brow,
+                   reinterpret_cast<const unsigned char *>(a.Bin) + (((size_t)S.b * a.T + t) * a.G + S.g) * brow, brow,
                    &gfull[gs], pol_keep);
         }
-        if (lane >= 12 && lane < 12 + t_out) {
+        if (lane >= 12 && lane < 12 + S.t_out) {
           const int t = lane - 12;
           bulk_g2s(gb + lay.gb_C + t * brow,
-                   reinterpret_cast<const unsigned char *>(a.C) + (((size_t)b * a.T + t) * a.G + g) * brow, brow,
+                   reinterpret_cast<const unsigned char *>(a.C) + (((size_t)S.b * a.T + t) * a.G + S.g) * brow, brow,
                    &gfull[gs], pol_keep);
         }
-        // ---- tiles of the unit's heads
-        const uint32_t tbytes = (uint32_t)lay.tile_bytes + n_rec * xrow;
-        bool ok = true;
-        for (int i = 0; i < nh; ++i, ++ti) {
-          const int s = ti % NS;
-          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
-            if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
-            ok = false;
-            break;
-          }
-          unsigned char *st = stages + (size_t)s * lay.stage_bytes;
-          const size_t unit = (size_t)b * a.H + h0 + i;
-          if (lane == 0) {
-            armed[s] = ti / NS;
-            mbar_arrive_expect_tx(&full[s], tbytes);
-          }
-          __syncwarp();
-          if (lane == 0) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
-          if (lane == 1 && n_ring)
-            bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + base_e) * xrow,
-                     n_ring * xrow, &full[s], pol_keep);
-          if (lane >= 4 && lane < 4 + n_new) {
-            const int t = lane - 4;
-            bulk_g2s(st + lay.xr + (n_ring + t) * xrow,
-                     reinterpret_cast<const unsigned char *>(a.x) + (((size_t)b * a.T + t) * a.H + h0 + i) * xrow, xrow,
-                     &full[s], pol_keep);
-          }
-        }
-        if (!ok) break;
       }
+      return true;
+    };
+    bool ok = true;
+    if (u_begin < u_end) ok = issue_group(u_begin, 0);
+    int ti = 0;
+    for (int u = u_begin, gi = 0; ok && u < u_end; ++u, ++gi) {
+      if (u + 1 < u_end && !issue_group(u + 1, gi + 1)) {
+        ok = false;
+        break;
+      }
+      Sched S;
+      schedule(u, S, nullptr);
+      if (!S.active) continue;
+      const int n_rec = S.n_ring + S.n_new;
+      const uint32_t tbytes = (uint32_t)lay.tile_bytes + n_rec * xrow;
+      for (int i = 0; i < S.nh; ++i, ++ti) {
+        const int s = ti % NS;
+        if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+        const size_t unit = (size_t)S.b * a.H + S.h0 + i;
+        if (lane == 0) {
+          armed[s] = ti / NS;
+          mbar_arrive_expect_tx(&full[s], tbytes);
+        }
+        __syncwarp();
+        if (lane == 0) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
+        if (lane == 1 && S.n_ring)
+          bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + S.base_e) * xrow,
+                   S.n_ring * xrow, &full[s], pol_keep);
+        if (lane >= 4 && lane < 4 + S.n_new) {
+          const int t = lane - 4;
+          bulk_g2s(st + lay.xr + (S.n_ring + t) * xrow,
+                   reinterpret_cast<const unsigned char *>(a.x) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * xrow, xrow,
+                   &full[s], pol_keep);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      record_error(a.err, 0, RSSM_DEV_TIMEOUT);
+      *abort_flag = 1;
     }
   } else if (warp == kPrepWarp) {
     // ================================================================== prep warp
     for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
-      const int gs = gi & 1;
-      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+      const int gs = gi % kGB, tsl = gi & 1;
+      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGB) & 1), abort_flag) ||
+          !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
       const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
       const float *gf = reinterpret_cast<const float *>(gb);
-      const int b = gh[G_B], g = gh[G_G], nh = gh[G_NH];
+      const int b = gh[G_B], g = gh[G_G], nh = gh[G_NH], h0 = gh[G_H0];
       if (gh[G_WMETA] && lane == 0) a.meta_out[b] = make_int4(gh[G_MC], gh[G_ME], gh[G_MP], 0);
+      // per-head parameters and the new tokens' dt (global loads, kept off the producer's path)
+      float *gfw = reinterpret_cast<float *>(gbuf + (size_t)gs * lay.gb_bytes);
+      if (lane < nh) {
+        gfw[G_A + lane] = a.A[h0 + lane];
+        gfw[G_D + lane] = a.D[h0 + lane];
+      }
       if (gh[G_ACTIVE]) {
-        const Tables T = tables(gs);
+        for (int q = lane; q < gh[G_NNEW] * nh; q += 32) {
+          const int t = q / nh, i = q % nh;
+          gfw[G_DT + t * kHG + i] = to_f32(reinterpret_cast<const TI *>(a.dt)[((size_t)b * a.T + t) * a.H + h0 + i]);
+        }
+      }
+      __syncwarp();
+      if (gh[G_ACTIVE]) {
+        const Tables T = tables(tsl);
         const int n_rec = gh[G_NREC], m = gh[G_M], n_ring = gh[G_NRING], n_new = gh[G_NNEW], t_out = gh[G_TOUT];
         const int slot0 = gh[G_SLOT0], base_e = gh[G_BASE];
         const int dts = dt_stride(a.L);
@@ -317,17 +345,23 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
           }
         }
         __syncwarp();
-        // per-head decay weights (log-space suffix sums of dt); pairs (head, output), then fold weights
+        // per-head weights of every record in every output (log-space suffix sums of dt):
+        // coef[r] = dt_r exp(A s(r+1, e_j)) (B_r . C_j) for m <= r < e_j, plus D on the output's
+        // own token r = e_j - 1, and 0 elsewhere; ao = exp(A s(m, e_j)) scales S' C_j
         for (int pr = lane; pr < nh * t_out; pr += 32) {
           const int i = pr / t_out, j = pr % t_out;
           const float A = gf[G_A + i];
           const int e_j = n_rec - t_out + j + 1;
+          float *co = T.coef + (i * NO + j) * rmax;
+          for (int r = e_j; r < n_rec; ++r) co[r] = 0.f;
           float sfx = 0.f;
           for (int r = e_j - 1; r >= m; --r) {
             const float d = dt_of(i, r);
-            T.coef[(i * NO + j) * rmax + r] = d * __expf(A * sfx) * T.g[j * rmax + r];
+            co[r] = d * __expf(A * sfx) * T.g[j * rmax + r];
             sfx += d;
           }
+          for (int r = 0; r < m; ++r) co[r] = 0.f;
+          co[e_j - 1] += gf[G_D + i];
           T.ao[i * NO + j] = __expf(A * sfx);
         }
         if (m > 0 && lane < nh) {
@@ -343,15 +377,15 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tfull[gs]);
+      if (lane == 0) mbar_arrive(&tfull[tsl]);
     }
   } else {
     // ================================================================== consumer warps
     const int row0 = warp * 8;
     int ti = 0;
     for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
-      const int gs = gi & 1;
-      if (!mbar_wait_or_abort(&tfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+      const int gs = gi % kGB, tsl = gi & 1;
+      if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -360,7 +394,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       const float *gf = reinterpret_cast<const float *>(gb);
       const int b = gh[G_B], h0 = gh[G_H0], nh = gh[G_NH];
       if (gh[G_ACTIVE]) {
-        const Tables T = tables(gs);
+        const Tables T = tables(tsl);
         const float *t_coef = T.coef, *t_ao = T.ao, *t_wf = T.wf, *t_af = T.af;
         const int n_rec = gh[G_NREC], m = gh[G_M], n_ring = gh[G_NRING], n_new = gh[G_NNEW], t_out = gh[G_TOUT];
         const int slot0 = gh[G_SLOT0];
@@ -396,9 +430,11 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
               for (int r = 0; r < m; ++r) {
                 const float4 bv = load4(Bg + r * kCols + 4 * lane);
                 const float wr = t_wf[i * rmax + r];
+                float xv[8];
+                load8(xr + r * a.P + row0, xv);
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
-                  const float cx = wr * to_f32(xr[r * a.P + row0 + rr]);
+                  const float cx = wr * xv[rr];
                   sv[rr].x = fmaf(cx, bv.x, sv[rr].x);
                   sv[rr].y = fmaf(cx, bv.y, sv[rr].y);
                   sv[rr].z = fmaf(cx, bv.z, sv[rr].z);
@@ -410,30 +446,34 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
               for (int rr = 0; rr < 8; ++rr)
                 __stcs(reinterpret_cast<float4 *>(dst + (row0 + rr) * kCols + 4 * lane), sv[rr]);
             }
+            // S'[row] . (ao_j C_j) over this lane's 4 columns, plus the buffered part: lane r
+            // (< n_rec) adds coef_{j,r} x_r[row] for the warp's 8 rows (one 16-byte load of x_r)
             float part[V];
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr)
+            for (int j = 0; j < NO; ++j) {
+              const float ao = (j < t_out) ? t_ao[i * NO + j] : 0.f;
+              const float4 c4 = make_float4(ao * cv[j].x, ao * cv[j].y, ao * cv[j].z, ao * cv[j].w);
 #pragma unroll
-              for (int j = 0; j < NO; ++j)
-                part[rr * NO + j] = sv[rr].x * cv[j].x + sv[rr].y * cv[j].y + sv[rr].z * cv[j].z + sv[rr].w * cv[j].w;
+              for (int rr = 0; rr < 8; ++rr)
+                part[rr * NO + j] = sv[rr].x * c4.x + sv[rr].y * c4.y + sv[rr].z * c4.z + sv[rr].w * c4.w;
+            }
+            for (int r = lane; r < n_rec; r += 32) {
+              float xv[8];
+              load8(xr + r * a.P + row0, xv);
+#pragma unroll
+              for (int j = 0; j < NO; ++j) {
+                const float co = (j < t_out) ? t_coef[(i * NO + j) * rmax + r] : 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) part[rr * NO + j] = fmaf(co, xv[rr], part[rr * NO + j]);
+              }
+            }
             warp_transpose_reduce<V>(part, lane);
-            const float Dh = gf[G_D + i];
 #pragma unroll
             for (int k2 = 0; k2 < KEEP; ++k2) {
               const int idx = (V >= 32) ? lane * KEEP + k2 : lane / SPREAD;
               const int rr = idx / NO, j = idx % NO;
-              const int p = row0 + rr;
-              const int e_j = n_rec - t_out + j + 1;
-              float acc = 0.f;
-              if (j < t_out) {
-                const float *co = t_coef + (i * NO + j) * rmax;
-                for (int r = m + (lane % SPREAD); r < e_j; r += SPREAD) acc = fmaf(co[r], to_f32(xr[r * a.P + p]), acc);
-              }
-#pragma unroll
-              for (int off = 1; off < SPREAD; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
               if (j < t_out && (lane % SPREAD) == 0)
-                a.y[(((size_t)b * a.T + j) * a.H + h) * a.P + p] =
-                    t_ao[i * NO + j] * part[k2] + acc + Dh * to_f32(xr[(e_j - 1) * a.P + p]);
+                a.y[(((size_t)b * a.T + j) * a.H + h) * a.P + row0 + rr] = part[k2];
             }
           }
           if (warp == 0 && n_new) {  // append this head's new tokens (x rows, dt) to its ring row
@@ -452,7 +492,10 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       if (*abort_flag) break;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&gempty[gs]);  // this warp is done with the group buffer and the tables
+      if (lane == 0) {  // this warp is done with the unit's group buffer and tables
+        mbar_arrive(&gempty[gs]);
+        mbar_arrive(&tempty[tsl]);
+      }
     }
   }
   __syncthreads();
@@ -460,7 +503,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     // do not leave bulk copies in flight into the shared memory of an exiting block
     for (int s = 0; s < 8; ++s)
       if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1));
-    for (int s = 0; s < 2; ++s)
+    for (int s = 0; s < kGB; ++s)
       if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
   }
 }
@@ -469,7 +512,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
 
 int m2_smem_bytes(int P, int L, int tmax, int esz, int nstage) {
   const M2Layout l = m2_layout(P, L, tmax, esz);
-  return kBarBytes + 2 * l.tab_bytes + 2 * l.gb_bytes + nstage * l.stage_bytes;
+  return kBarBytes + 2 * l.tab_bytes + kGB * l.gb_bytes + nstage * l.stage_bytes;
 }
 
 int m2_max_stages(int P, int L, int tmax, int esz, int smem_budget) {

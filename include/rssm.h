@@ -40,7 +40,7 @@
  *     call that changes the bookkeeping.
  *   - Token inputs are row-major with the leading dimensions named, and must
  *     start on 16-byte boundaries; rows of length P, N, d_k or d_v in the
- *     input dtype must be multiples of 16 bytes, and so must H * sizeof(dt).
+ *     input dtype must be multiples of 16 bytes.
  */
 #ifndef RSSM_H
 #define RSSM_H
@@ -187,7 +187,8 @@ rssm_status rssm_ring_bytes(const rssm_config *cfg, size_t *bytes);
 rssm_status rssm_export(rssm_ctx *ctx, float *S_out, void *ring_out, int *meta_out, rssm_stream stream);
 
 /* Copy the NVFP4 read copy out (device destinations): codes uint8 [Bt][H][rows][cols/2]
- * (element 2j in the low nibble), scales uint8 [Bt][H][rows][cols/16] (E4M3), g fp32 [Bt][H].
+ * (element 2j in the low nibble), scales uint8 [Bt][H][rows][cols/16] (E4M3 of each
+ * 16-element block), g fp32 [Bt][H][ceil(rows/64)] (one scale per 64-row tile).
  * RSSM_ERR_UNSUPPORTED if the context has no read copy. */
 rssm_status rssm_export_read_copy(rssm_ctx *ctx, unsigned char *codes, unsigned char *scales, float *g,
                                   rssm_stream stream);

@@ -47,7 +47,8 @@ rounding, random words from Philox4x32-10 with counter (sequence*H + head,
 new epoch, element/4, 0) and the 64-bit seed as key); read = "same" (outputs
 read the checkpoint), "nvfp4" (separate NVFP4 read copy, re-quantised from the
 fp32 fold result at every fold) or "shared_nvfp4" (the NVFP4 copy is also the
-checkpoint the recurrence continues from; contrast mode).
+checkpoint the recurrence continues from; contrast mode).  The NVFP4 copy is
+quantised tile by tile, a tile being 64 consecutive rows of one head's state.
 
 Two outputs are produced per call: ``y`` mirrors the method (folds at the
 points above, state rounded to its stored formats, replay in float64) and
@@ -145,7 +146,7 @@ class ReplayOracle:
         return rc.gdn_step(S, rec["q"], rec["k"], rec["v"], rec["alpha"], rec["beta"], self.q_scale)
 
     def _read_copy(self, S32):
-        return lowprec.nvfp4_roundtrip(S32).astype(np.float64)
+        return lowprec.nvfp4_roundtrip_state(S32).astype(np.float64)
 
     def _store(self, b, S_new):
         """Write a fold result for sequence b into the stored formats."""

@@ -24,12 +24,13 @@ E2M1 (OCP FP4): magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}; round to nearest,
     ties to the even code; saturate at 6.  Code = sign << 3 | magnitude index,
     with the sign bit set iff x < 0.
 
-NVFP4 read copy of one state tile (one sequence and head), blocks of 16
+NVFP4 read copy.  A tile is 64 consecutive rows (fewer for the last rows) of
+one sequence's and head's state matrix, all 128 columns; blocks are 16
 consecutive elements along the contracted (contiguous) axis:
     g   = amax(tile) / 2688 in fp32 (2688 = 6 * 448), or 1 if amax = 0
     s_b = E4M3(amax(block) / (6 g))             (fp32 product, then fp32 divide)
     d_b = s_b * g                               (fp32)
-    q   = E2M1(|x| / d_b) with the sign of x     (fp32 divide); q = 0 if s_b = 0
+    q   = E2M1(|x| / d_b) with the sign of x     (fp32 divide); q = 0 if d_b = 0
     dequantised value = value(q) * d_b          (fp32)
 """
 
@@ -41,6 +42,7 @@ FP16_MAX = 65504.0
 E4M3_MAX = 448.0
 E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], np.float64)
 NVFP4_BLOCK = 16
+NVFP4_TILE_ROWS = 64
 
 
 # --------------------------------------------------------------------------- FP16 stochastic rounding
@@ -137,11 +139,11 @@ def nvfp4_quantize(tile) -> dict:
     sb_in = (amax_b / t[..., None, None]).astype(np.float32)
     s_b = e4m3_round(sb_in).astype(np.float32)
     d_b = (s_b * g[..., None, None]).astype(np.float32)
-    safe = np.where(s_b > 0, d_b, np.float32(1.0)).astype(np.float32)
+    safe = np.where(d_b > 0, d_b, np.float32(1.0)).astype(np.float32)
     yb = (blocks / safe[..., None]).astype(np.float32)
     mag = e2m1_magnitude_code(yb)
-    mag = np.where((s_b > 0)[..., None], mag, 0).astype(np.uint8)
-    neg = (x.reshape(blocks.shape) < 0) & (s_b > 0)[..., None]
+    mag = np.where((d_b > 0)[..., None], mag, 0).astype(np.uint8)
+    neg = (x.reshape(blocks.shape) < 0) & (d_b > 0)[..., None]
     codes = (mag | (neg.astype(np.uint8) << 3)).reshape(x.shape).astype(np.uint8)
     packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
     return {"codes": codes, "packed": packed, "scales": e4m3_code(s_b), "g": g}
@@ -162,3 +164,23 @@ def nvfp4_dequantize(codes, scales, g) -> np.ndarray:
 def nvfp4_roundtrip(tile) -> np.ndarray:
     q = nvfp4_quantize(tile)
     return nvfp4_dequantize(q["codes"], q["scales"], q["g"])
+
+
+def nvfp4_quantize_state(S) -> dict:
+    """Quantise states [..., rows, 128] tile by tile (64-row tiles).  Returns packed codes
+    [..., rows, 64], scales [..., rows, 8] and g [..., ceil(rows/64)]."""
+    S = np.ascontiguousarray(S, np.float32)
+    rows = S.shape[-2]
+    parts = [nvfp4_quantize(S[..., r0:r0 + NVFP4_TILE_ROWS, :]) for r0 in range(0, rows, NVFP4_TILE_ROWS)]
+    return {"codes": np.concatenate([p["codes"] for p in parts], axis=-2),
+            "packed": np.concatenate([p["packed"] for p in parts], axis=-2),
+            "scales": np.concatenate([p["scales"] for p in parts], axis=-2),
+            "g": np.stack([p["g"] for p in parts], axis=-1)}
+
+
+def nvfp4_roundtrip_state(S) -> np.ndarray:
+    """fp32 values of the read copy of states [..., rows, 128] (64-row tiles)."""
+    S = np.ascontiguousarray(S, np.float32)
+    rows = S.shape[-2]
+    return np.concatenate([nvfp4_roundtrip(S[..., r0:r0 + NVFP4_TILE_ROWS, :])
+                           for r0 in range(0, rows, NVFP4_TILE_ROWS)], axis=-2)

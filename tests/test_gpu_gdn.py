@@ -1,0 +1,161 @@
+"""Gated DeltaNet replay decode on the GPU vs the float64 oracle (parity tests; need a B200)."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_harness import TOL_F32, Pair, head_rel_err
+from oracle import lowprec as lp
+from oracle.philox import sr_words
+from synth import GDN_B256, GDN_LOWPREC, accepted_lengths, gdn_draft_inputs, gdn_step_inputs
+
+pytestmark = pytest.mark.gpu
+
+SMALL = GDN_B256.replace(batch=4, nheads=4)
+
+
+def run_steps(p, steps, start=0, check_every=1, tol=TOL_F32, ref="true"):
+    worst = 0.0
+    for t in range(start, start + steps):
+        y, y_ref, y_true = p.step(gdn_step_inputs(p.wl, t))
+        err = head_rel_err(y, y_true if ref == "true" else y_ref)
+        worst = max(worst, err.max())
+        assert err.max() <= tol, f"step {t}: rel err {err.max():.3e}"
+        if check_every and (t + 1) % check_every == 0:
+            p.check_bookkeeping()
+    return worst
+
+
+def test_small_every_step(cuda_ok):
+    p = Pair(SMALL)
+    run_steps(p, 48)
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
+@pytest.mark.parametrize("L", [1, 4, 8, 32])
+def test_window_sweep(cuda_ok, L):
+    p = Pair(SMALL.replace(window=L, batch=3))
+    run_steps(p, 40)
+    p.check_checkpoint()
+
+
+def test_ragged_rows_and_heads(cuda_ok):
+    """d_v = 40 (one partial 64-row tile), 6 heads (a partial unit), fp32 inputs, 5 sequences."""
+    wl = SMALL.replace(batch=5, nheads=6, dv=40, in_dtype="f32")
+    p = Pair(wl)
+    run_steps(p, 34, check_every=17)
+    p.check_checkpoint()
+
+
+def test_many_units(cuda_ok):
+    """More units than SMs, not a multiple of them (151 sequences x 2 units)."""
+    wl = SMALL.replace(batch=151, nheads=8)
+    p = Pair(wl, seq_ids=[0, 75, 150])
+    run_steps(p, 20, check_every=10)
+    p.check_checkpoint()
+
+
+@pytest.mark.parametrize("T", [1, 2, 4, 8])
+def test_verify_commit_random(cuda_ok, T):
+    wl = SMALL.replace(batch=5, nheads=3)
+    p = Pair(wl, max_draft=T)
+    step = 0
+    for rnd in range(10):
+        y, _, y_true = p.verify(T, gdn_draft_inputs(wl, rnd, T))
+        assert head_rel_err(y, y_true).max() <= TOL_F32
+        p.check_bookkeeping()
+        p.commit(accepted_lengths(wl, rnd, T))
+        p.check_bookkeeping()
+        if rnd % 3 == 1:
+            for _ in range(3):
+                y, _, y_true = p.step(gdn_step_inputs(wl, step))
+                step += 1
+                assert head_rel_err(y, y_true).max() <= TOL_F32
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
+def test_flush_mask(cuda_ok):
+    p = Pair(SMALL)
+    run_steps(p, 5)
+    p.flush(np.array([1, 0, 0, 1]))
+    p.check_bookkeeping()
+    p.check_checkpoint()
+    run_steps(p, 12, start=5)
+    p.flush()
+    p.check_bookkeeping()
+    p.check_checkpoint()
+
+
+# ------------------------------------------------------------------------------------ precision converters
+
+def _edge_state(shape, seed):
+    rng = np.random.default_rng(seed)
+    S = (rng.standard_normal(shape) * 10.0 ** rng.uniform(-7, 2, shape[:-1] + (1,))).astype(np.float32)
+    S[0, 0, 3] = 0.0                                             # a zero row
+    S[0, 0, 5, :16] = 0.0                                        # a zero block
+    S[0, 1, 7, :4] = [65504.0, -70000.0, 3e-6, -1e-8]            # saturation, fp16 subnormals
+    S[0, 1, 9] = np.float16(0.125).astype(np.float32)            # on the fp16 grid
+    return S
+
+
+@pytest.mark.parametrize("hp,read", [("f16sr", "nvfp4"), ("f32", "shared_nvfp4"), ("f16sr", "same")])
+def test_load_converters_bit_exact(cuda_ok, hp, read):
+    wl = SMALL.replace(batch=2, nheads=3, dv=128)
+    S = _edge_state((2, 3, 128, 128), 1)
+    p = Pair(wl, hp=hp, read=read, seed=0xABCDEF0123456789, S0=S)
+    ex = p.gpu.export(state=True, ring=False)["S"].cpu().numpy()
+    if read == "shared_nvfp4":
+        np.testing.assert_array_equal(ex, lp.nvfp4_roundtrip_state(S))
+    elif hp == "f16sr":
+        units = (np.arange(2)[:, None] * 3 + np.arange(3)[None, :])
+        words = sr_words(0xABCDEF0123456789, units, 0, 128 * 128).reshape(2, 3, 128, 128)
+        np.testing.assert_array_equal(ex, lp.fp16_stochastic_round(S, words).astype(np.float32))
+    if read != "same":
+        rc = p.gpu.export_read_copy()
+        q = lp.nvfp4_quantize_state(S)
+        np.testing.assert_array_equal(rc["packed"].cpu().numpy(), q["packed"])
+        np.testing.assert_array_equal(rc["scales"].cpu().numpy(), q["scales"])
+        np.testing.assert_array_equal(rc["g"].cpu().numpy(), q["g"])
+
+
+# ------------------------------------------------------------------------------------ separate precision
+
+# Bound for low-precision modes: GPU vs the oracle in the same mode.  The two fold in
+# different arithmetic (fp32 vs float64), so now and then one element lands on the other
+# side of an NVFP4 or stochastic-rounding decision boundary.  A flipped NVFP4 code moves
+# one element by one E2M1 step (at most a third of its block maximum), which moves that
+# head's output by up to ~1e-2 relative; a flipped fp16 rounding moves it by one fp16
+# ulp.  So: every head within TOL_FLIP, and all but a small fraction of (step, sequence,
+# head) outputs within the fp32 bound.
+TOL_FLIP = 2e-2
+FLIP_FRACTION = 0.02
+
+
+@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f16sr", "same"), ("f32", "shared_nvfp4")])
+def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
+    wl = GDN_LOWPREC.replace(batch=4, nheads=4, window=8)
+    p = Pair(wl, hp=hp, read=read, seed=7)
+    errs = []
+    for t in range(48):
+        y, y_ref, y_true = p.step(gdn_step_inputs(wl, t))
+        err = head_rel_err(y, y_ref)
+        errs.append(err.ravel())
+        assert err.max() <= TOL_FLIP, f"step {t}: {err.max():.3e}"
+        p.check_bookkeeping(ring=(t % 8 == 7))
+    errs = np.concatenate(errs)
+    frac = float(np.mean(errs > TOL_F32))
+    print(f"{hp}/{read}: max {errs.max():.3e}, median {np.median(errs):.3e}, fraction above 1e-4 {frac:.4f}")
+    assert frac <= FLIP_FRACTION
+
+
+@pytest.mark.slow
+def test_full_size_sampled(cuda_ok):
+    """The GDN layer (batch 256, 32 heads, d 128, L 16), 1024 steps, sampled sequences and heads."""
+    wl = GDN_B256
+    p = Pair(wl, seq_ids=[0, 128, 255], head_ids=[0, 5, 31])
+    worst = run_steps(p, wl.steps, check_every=101)
+    p.check_bookkeeping()
+    p.check_checkpoint()
+    print(f"worst rel err {worst:.3e}")

@@ -187,3 +187,16 @@ def test_nvfp4_error_bound_and_scale_choice():
     # each block maximum lands within a scale step of code 6 (i.e. value 6 after rounding)
     top = lp.E2M1_VALUES[(q["codes"] & 7).reshape(blocks.shape).max(-1)]
     assert np.all(top[amax_b[..., 0] > 1e-4 * np.abs(t).max()] >= 4.0)
+
+
+def test_nvfp4_state_tiles_are_64_rows():
+    rng = np.random.default_rng(9)
+    S = rng.standard_normal((2, 3, 128, 128)).astype(np.float32)
+    S[0, 0, 70] *= 1000.0                                      # a large row in the second tile only
+    q = lp.nvfp4_quantize_state(S)
+    assert q["g"].shape == (2, 3, 2) and q["packed"].shape == (2, 3, 128, 64)
+    np.testing.assert_allclose(q["g"][0, 0], [np.abs(S[0, 0, :64]).max() / 2688, np.abs(S[0, 0, 64:]).max() / 2688],
+                               rtol=1e-7)
+    np.testing.assert_array_equal(lp.nvfp4_roundtrip_state(S)[..., :64, :], lp.nvfp4_roundtrip(S[..., :64, :]))
+    S40 = S[..., :40, :]
+    assert lp.nvfp4_quantize_state(S40)["g"].shape == (2, 3, 1)
