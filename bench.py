@@ -63,6 +63,22 @@ def conventional_bytes(wl) -> int:
     return 2 * Bt * H * P * N * 4 + Bt * (H * P * esz + 2 * G * N * esz + H * esz) + Bt * H * P * 4
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of a list of floats over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def weak_scaling_value(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job tokens/s: every rank decodes its own batch shard; time is the slowest rank's."""
+    return tokens_per_rank_step * world * steps / (max_ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -233,11 +249,7 @@ def run_gpu(args, rank, world):
         torch.cuda.synchronize()
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
     total_ms = ev[0].elapsed_time(ev[K])
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks([total_ms], device=dev)[0]
     model = [traffic_model(WL, (count0 + i) % WL.window) for i in range(K)]
     bytes_avg = sum(sum(m.values()) for m in model) / K
     step_ms = total_ms / K
@@ -282,15 +294,12 @@ def run_gpu(args, rank, world):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / Ke
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_ms, conv_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms, conv_ms = float(tt[0].item()), float(tt[1].item())
+    e2e_ms, conv_ms = max_over_ranks([e2e_ms, conv_ms], device=dev)
 
     tokens = WL.batch * world
     res = {
-        "metric": METRIC, "value": tokens * K / (total_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": weak_scaling_value(WL.batch, world, K, total_ms), "unit": "tokens/s",
+        "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; bf16 token inputs, fp32 checkpoint)",
         "config": {"workload": "mamba2 replay decode, batch 256 per GPU, 128 heads, P 64, N 128, 8 groups, L 16, "
@@ -366,7 +375,17 @@ def gdn_section(steps: int) -> dict:
     for i in range(2 * wl.window):
         step(i)
     K = max(wl.window, steps // wl.window * wl.window)
-    ms = timed(step, K, stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(K):
+        step(i)
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    ms = ev[0].elapsed_time(ev[K]) / K
+    fold_ms = [d for i, d in enumerate(per) if (i + 1) % wl.window == 0]
+    plain_ms = [d for i, d in enumerate(per) if (i + 1) % wl.window != 0]
     bytes_avg = sum(gdn_traffic(wl, i % wl.window) for i in range(K)) / K
     cfg = make_config("gdn", wl.batch, wl.nheads, wl.dv, wl.dk, 1, wl.window, 0, bf)
     S = S0.clone()
@@ -383,6 +402,7 @@ def gdn_section(steps: int) -> dict:
     return {"workload": "gdn replay decode, batch 256, 32 heads, d_k = d_v = 128, L 16, bf16 inputs, fp32 checkpoint",
             "tokens_per_s": wl.batch / (ms * 1e-3), "ms_per_step": ms, "GBps": bytes_avg / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": bytes_avg / (ms * 1e-3) / 1e9 / hbm, "bytes_per_step": bytes_avg,
+            "plain_launch_ms": statistics.median(plain_ms), "fold_launch_ms": statistics.mean(fold_ms),
             "conventional_tokens_per_s": wl.batch / (ms_conv * 1e-3), "conventional_ms_per_step": ms_conv,
             "conventional_GBps": conv_bytes / (ms_conv * 1e-3) / 1e9, "replay_speedup": ms_conv / ms,
             "steps": K, "device_error": layer.get_error()}
@@ -451,6 +471,8 @@ def main():
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN and speculative-verify sections")
+    ap.add_argument("--only", choices=["gdn", "verify"], default=None,
+                    help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -461,6 +483,12 @@ def main():
         # the reference arm is the CPU oracle, on rank 0 only; other ranks exit without work
         if rank == 0:
             print(json.dumps(reference_arm(args)))
+        return
+
+    if args.only is not None:
+        if rank == 0:
+            out = gdn_section(args.steps) if args.only == "gdn" else verify_section(args.steps)
+            print(json.dumps(out))
         return
 
     if world > 1:

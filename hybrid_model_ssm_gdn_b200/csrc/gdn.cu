@@ -22,17 +22,19 @@
 //
 // Block roles (one block per SM, persistent):
 //  * producer warp: TMA bulk copies (cp.async.bulk) of each unit's k records, q and
-//    alpha/beta rows into a double-buffered group buffer, and of each 64-row tile of a
-//    head's state (in its stored format) plus the head's v records into a ring of stages;
+//    alpha/beta rows into one of three group buffers, one unit ahead of the unit whose
+//    tiles it is issuing, and of each 64-row tile of a head's state (in its stored
+//    format) plus the head's v records into a ring of stages;
 //  * two prep warps: 8-lane subgroups walk q back for every (head, draft) pair of the
 //    unit, writing u_0 and the coefficients beta_r c_r into double-buffered tables;
 //    they also append k, alpha, beta of the new tokens and write the bookkeeping word;
-//  * two groups of four consumer warps take alternate tiles.  Non-fold tiles: lane l owns
-//    columns 4l..4l+3 of 16 rows, row dot products with u_0 finish in a warp transpose
-//    reduction.  Fold tiles: two lanes own one row (64 columns each) and run the
-//    sequential row update with one shuffle per record; then the new state is written
-//    in the checkpoint format and, in NVFP4 modes, quantised (tile maximum over the
-//    group through a named barrier).
+//  * eight consumer warps take every tile, warp w rows 8w..8w+7.  Non-fold tiles: lane l
+//    owns columns 4l..4l+3, the row dot products with u_0 and the buffered term finish in
+//    one warp transpose reduction.  Fold tiles: four lanes own one row (32 columns each,
+//    in registers) and run the sequential row update with two shuffles per record; then
+//    the new state is written in the checkpoint format and, in NVFP4 modes, quantised
+//    (tile maximum over the eight warps through an mbarrier rendezvous with bounded
+//    waits).
 // Work unit: (sequence, chunk of HG heads), HG = 4, 4, 2, 1 for 1, 2, 4, 8 outputs.
 #include "common.cuh"
 #include "kernels.h"
@@ -77,14 +79,15 @@ __host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz) {
   l.tb_u0 = 0;
   l.tb_coef = l.hg * l.no * kCols * 4;
   l.tb_amax = (int)align_up((size_t)l.tb_coef + (size_t)l.hg * l.no * l.rmax * 4, 16);
-  l.tab_bytes = (int)align_up((size_t)l.tb_amax + 2 * 2 * 4 * 4, 128);   // amax[group][slot][warp]
+  l.tab_bytes = (int)align_up((size_t)l.tb_amax + 2 * 8 * 4, 128);   // amax[slot][warp]
   l.st_g = kTileMaxBytes;
   l.st_v = l.st_g + 16;
   l.stage_bytes = (int)align_up((size_t)l.st_v + (size_t)l.rmax * R * esz, 128);
   return l;
 }
 
-constexpr int kBarBytesG = 256;
+constexpr int kBarBytesG = 512;  // mbarriers (29 x 8 B) + armed phases + abort flag
+constexpr int kGBG = 3;  // group buffers: the producer loads a unit's group data one unit ahead
 
 // tile source formats
 enum { SRC_F32 = 0, SRC_F16 = 1, SRC_FP4 = 2 };
@@ -106,16 +109,17 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   const int NS = a.nstage, R = a.DV, L = a.L, HG = lay.hg, nrb = lay.nrb, dts = lay.dts;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + 8;
-  uint64_t *gfull = empty + 8;
-  uint64_t *gempty = gfull + 2;
-  uint64_t *tfull = gempty + 2;
-  uint64_t *psync = tfull + 2;   // rendezvous of the two prep warps (count 2)
-  uint64_t *csync = psync + 1;   // [2] rendezvous of the four warps of a consumer group (count 4)
-  volatile int *armed = reinterpret_cast<volatile int *>(csync + 2);  // [10]
-  volatile int *abort_flag = armed + 10;
+  uint64_t *gfull = empty + 8;       // [kGBG] group data landed
+  uint64_t *gempty = gfull + kGBG;   // [kGBG] consumers done with a unit's group data
+  uint64_t *tfull = gempty + kGBG;   // [2] tables ready
+  uint64_t *tempty = tfull + 2;      // [2] consumers done with the tables
+  uint64_t *psync = tempty + 2;      // rendezvous of the two prep warps (count 2)
+  uint64_t *fsync = psync + 1;       // rendezvous of the eight consumer warps (NVFP4 tile maximum)
+  volatile int *armed = reinterpret_cast<volatile int *>(fsync + 1);  // [8 + kGBG]
+  volatile int *abort_flag = armed + 8 + kGBG;
   unsigned char *tabs = smem + kBarBytesG;
   unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
-  unsigned char *stages = gbuf + 2 * lay.gb_bytes;
+  unsigned char *stages = gbuf + kGBG * lay.gb_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunks = (a.H + HG - 1) / HG;
@@ -129,17 +133,19 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 4);  // one consumer group of four warps per tile
+      mbar_init(&empty[s], kConsumerWarps);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kGBG; ++s) {
       mbar_init(&gfull[s], 1);
       mbar_init(&gempty[s], kConsumerWarps);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], kConsumerWarps);
     }
     mbar_init(psync, 2);
-    mbar_init(&csync[0], 4);
-    mbar_init(&csync[1], 4);
-    for (int s = 0; s < 10; ++s) armed[s] = -1;
+    mbar_init(fsync, kConsumerWarps);
+    for (int s = 0; s < 8 + kGBG; ++s) armed[s] = -1;
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -153,10 +159,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     const int b_first = u_begin / chunks;
     int mw_base = -1, mk = 1;
     int4 mw = make_int4(0, 0, 0, 0);
-    int ti = 0;
-    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+    struct Sched {
+      int b, h0, nh, active, n_ring, n_new, m, t_out, slot0, base_e;
+    };
+    auto schedule = [&](int u, Sched &S, int *hdr) {
       const int b = u / chunks, ch = u % chunks;
-      const int h0 = ch * HG, nh = min(HG, a.H - h0);
+      S.b = b; S.h0 = ch * HG; S.nh = min(HG, a.H - S.h0);
       const int base32 = b_first + ((b - b_first) & ~31);
       if (base32 != mw_base) {
         const int bq = base32 + lane;
@@ -169,13 +177,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       const int src = b - base32;
       const int c = __shfl_sync(0xffffffffu, mw.x, src), e = __shfl_sync(0xffffffffu, mw.y, src);
       const int pend = __shfl_sync(0xffffffffu, mw.z, src), msk = __shfl_sync(0xffffffffu, mk, src);
-      // ---- schedule (identical for every head of the sequence)
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
       int mc = c, me = e, mp = pend;
       const int base_e = (e & 1) * L, base_n = ((e + 1) & 1) * L;
       if (pend != 0) {
         active = 0;
-        if (h0 == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
+        if (S.h0 == 0 && lane == 0 && (a.op != OP_FLUSH || msk)) record_error(a.err, b, RSSM_DEV_PENDING);
       } else if (a.op == OP_STEP) {
         n_new = 1;
         t_out = 1;
@@ -194,109 +201,125 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         if (!msk || c == 0) active = 0;
         else { n_ring = c; m = c; mc = 0; me = e + 1; }
       }
-      const int n_rec = n_ring + n_new;
-      const int gs = gi & 1;
-      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
-        if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
-        break;
+      S.active = active; S.n_ring = n_ring; S.n_new = n_new; S.m = m; S.t_out = t_out; S.slot0 = slot0;
+      S.base_e = base_e;
+      if (hdr != nullptr && lane == 0) {
+        hdr[Q_ACTIVE] = active; hdr[Q_NREC] = n_ring + n_new; hdr[Q_M] = m; hdr[Q_NRING] = n_ring;
+        hdr[Q_NNEW] = n_new; hdr[Q_TOUT] = t_out; hdr[Q_SLOT0] = slot0; hdr[Q_MC] = mc; hdr[Q_ME] = me;
+        hdr[Q_MP] = mp; hdr[Q_B] = b; hdr[Q_H0] = S.h0; hdr[Q_NH] = S.nh; hdr[Q_BASE] = base_e;
+        hdr[Q_WMETA] = (S.h0 == 0);
       }
+    };
+    // group data of unit u: k records and q of every head, alpha / beta ring rows
+    auto issue_group = [&](int u, int gi) -> bool {
+      const int gs = gi % kGBG;
+      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGBG) & 1) ^ 1), abort_flag)) return false;
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
-      int *gh = reinterpret_cast<int *>(gb);
-      if (lane == 0) {
-        gh[Q_ACTIVE] = active; gh[Q_NREC] = n_rec; gh[Q_M] = m; gh[Q_NRING] = n_ring; gh[Q_NNEW] = n_new;
-        gh[Q_TOUT] = t_out; gh[Q_SLOT0] = slot0; gh[Q_MC] = mc; gh[Q_ME] = me; gh[Q_MP] = mp;
-        gh[Q_B] = b; gh[Q_H0] = h0; gh[Q_NH] = nh; gh[Q_BASE] = base_e; gh[Q_WMETA] = (h0 == 0);
-      }
+      Sched S;
+      schedule(u, S, reinterpret_cast<int *>(gb));
       __syncwarp();
-      const uint32_t gbytes =
-          active ? (uint32_t)(nh * (n_rec * krow + t_out * krow) + 2 * nh * dts * 4) : 0u;
+      const int n_rec = S.n_ring + S.n_new, nh = S.nh;
+      const uint32_t gbytes = S.active ? (uint32_t)(nh * (n_rec * krow + S.t_out * krow) + 2 * nh * dts * 4) : 0u;
       if (lane == 0) {
-        armed[8 + gs] = gi >> 1;
+        armed[8 + gs] = gi / kGBG;
         mbar_arrive_expect_tx(&gfull[gs], gbytes);
       }
       __syncwarp();
-      if (active) {
-        // copies: per head: k ring range, k of each new token, q of each output; alpha rows, beta rows
-        const int per_head = 1 + n_new + t_out;
+      if (S.active) {
+        const int per_head = 1 + S.n_new + S.t_out;
         const int ncopy = nh * per_head + 2;
         for (int q = lane; q < ncopy; q += 32) {
           if (q == ncopy - 2) {
-            bulk_g2s(gb + lay.gb_a, a.ring_a + ((size_t)b * a.H + h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
+            bulk_g2s(gb + lay.gb_a, a.ring_a + ((size_t)S.b * a.H + S.h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
           } else if (q == ncopy - 1) {
-            bulk_g2s(gb + lay.gb_b, a.ring_b + ((size_t)b * a.H + h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
+            bulk_g2s(gb + lay.gb_b, a.ring_b + ((size_t)S.b * a.H + S.h0) * dts, nh * dts * 4, &gfull[gs], pol_keep);
           } else {
             const int i = q / per_head, w = q % per_head;
-            const size_t unit = (size_t)b * a.H + h0 + i;
+            const size_t unit = (size_t)S.b * a.H + S.h0 + i;
             unsigned char *kd = gb + lay.gb_k + (size_t)i * lay.rmax * krow;
             if (w == 0) {
-              if (n_ring)
-                bulk_g2s(kd, reinterpret_cast<const unsigned char *>(a.ring_k) + (unit * 2 * L + base_e) * krow,
-                         n_ring * krow, &gfull[gs], pol_keep);
-            } else if (w <= n_new) {
+              if (S.n_ring)
+                bulk_g2s(kd, reinterpret_cast<const unsigned char *>(a.ring_k) + (unit * 2 * L + S.base_e) * krow,
+                         S.n_ring * krow, &gfull[gs], pol_keep);
+            } else if (w <= S.n_new) {
               const int t = w - 1;
-              bulk_g2s(kd + (n_ring + t) * krow,
-                       reinterpret_cast<const unsigned char *>(a.k) + (((size_t)b * a.T + t) * a.H + h0 + i) * krow,
+              bulk_g2s(kd + (S.n_ring + t) * krow,
+                       reinterpret_cast<const unsigned char *>(a.k) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * krow,
                        krow, &gfull[gs], pol_keep);
             } else {
-              const int t = w - 1 - n_new;
+              const int t = w - 1 - S.n_new;
               bulk_g2s(gb + lay.gb_q + ((size_t)i * lay.no + t) * krow,
-                       reinterpret_cast<const unsigned char *>(a.q) + (((size_t)b * a.T + t) * a.H + h0 + i) * krow,
+                       reinterpret_cast<const unsigned char *>(a.q) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * krow,
                        krow, &gfull[gs], pol_keep);
             }
           }
         }
-        // ---- tiles: (head, 64-row block)
-        const bool fold = m > 0;
-        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
-                                : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
-        bool ok = true;
-        for (int tt = 0; tt < nh * nrb; ++tt, ++ti) {
-          const int i = tt / nrb, t = tt % nrb;
-          const int rows = min(kFp4Rows, R - kFp4Rows * t);
-          const size_t unit = (size_t)b * a.H + h0 + i;
-          const size_t row_abs = unit * R + (size_t)kFp4Rows * t;  // first state row of the tile
-          const int s = ti % NS;
-          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
-            if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
-            ok = false;
-            break;
-          }
-          unsigned char *st = stages + (size_t)s * lay.stage_bytes;
-          uint32_t tb = (uint32_t)n_rec * vrow;
-          if (srcfmt == SRC_F32) tb += rows * kCols * 4;
-          else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
-          else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
-          if (lane == 0) {
-            armed[s] = ti / NS;
-            mbar_arrive_expect_tx(&full[s], tb);
-          }
-          __syncwarp();
-          if (lane == 0) {
-            if (srcfmt == SRC_F32)
-              bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
-            else if (srcfmt == SRC_F16)
-              bulk_g2s(st, reinterpret_cast<const __half *>(a.hp) + row_abs * kCols, rows * kCols * 2, &full[s], pol_stream);
-            else
-              bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
-          }
-          if (lane == 1 && srcfmt == SRC_FP4)
-            bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
-          if (lane == 2 && srcfmt == SRC_FP4) {
-            const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
-            bulk_g2s(st + lay.st_g, a.rg + gi4, 16, &full[s], pol_keep);
-          }
-          if (lane == 3 && n_ring)
-            bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + base_e) * vrow,
-                     n_ring * vrow, &full[s], pol_keep);
-          if (lane >= 4 && lane < 4 + n_new) {
-            const int tk = lane - 4;
-            bulk_g2s(st + lay.st_v + (n_ring + tk) * vrow,
-                     reinterpret_cast<const unsigned char *>(a.v) + (((size_t)b * a.T + tk) * a.H + h0 + i) * vrow,
-                     vrow, &full[s], pol_keep);
-          }
-        }
-        if (!ok) break;
       }
+      return true;
+    };
+    bool ok = true;
+    if (u_begin < u_end) ok = issue_group(u_begin, 0);
+    int ti = 0;
+    for (int u = u_begin, gi = 0; ok && u < u_end; ++u, ++gi) {
+      if (u + 1 < u_end && !issue_group(u + 1, gi + 1)) {
+        ok = false;
+        break;
+      }
+      Sched S;
+      schedule(u, S, nullptr);
+      if (!S.active) continue;
+      const int n_rec = S.n_ring + S.n_new;
+      const bool fold = S.m > 0;
+      const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
+                              : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
+      for (int tt = 0; tt < S.nh * nrb; ++tt, ++ti) {
+        const int i = tt / nrb, t = tt % nrb;
+        const int rows = min(kFp4Rows, R - kFp4Rows * t);
+        const size_t unit = (size_t)S.b * a.H + S.h0 + i;
+        const size_t row_abs = unit * R + (size_t)kFp4Rows * t;  // first state row of the tile
+        const int s = ti % NS;
+        if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+        uint32_t tb = (uint32_t)n_rec * vrow;
+        if (srcfmt == SRC_F32) tb += rows * kCols * 4;
+        else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
+        else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
+        if (lane == 0) {
+          armed[s] = ti / NS;
+          mbar_arrive_expect_tx(&full[s], tb);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if (srcfmt == SRC_F32)
+            bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
+          else if (srcfmt == SRC_F16)
+            bulk_g2s(st, reinterpret_cast<const __half *>(a.hp) + row_abs * kCols, rows * kCols * 2, &full[s], pol_stream);
+          else
+            bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
+        }
+        if (lane == 1 && srcfmt == SRC_FP4)
+          bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
+        if (lane == 2 && srcfmt == SRC_FP4) {
+          const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
+          bulk_g2s(st + lay.st_g, a.rg + gi4, 16, &full[s], pol_keep);
+        }
+        if (lane == 3 && S.n_ring)
+          bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + S.base_e) * vrow,
+                   S.n_ring * vrow, &full[s], pol_keep);
+        if (lane >= 4 && lane < 4 + S.n_new) {
+          const int tk = lane - 4;
+          bulk_g2s(st + lay.st_v + (S.n_ring + tk) * vrow,
+                   reinterpret_cast<const unsigned char *>(a.v) + (((size_t)S.b * a.T + tk) * a.H + S.h0 + i) * vrow,
+                   vrow, &full[s], pol_keep);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      record_error(a.err, 0, RSSM_DEV_TIMEOUT);
+      *abort_flag = 1;
     }
   } else if (warp == kGPrep0 || warp == kGPrep0 + 1) {
     // ================================================================== prep warps
@@ -312,8 +335,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       return ok;
     };
     for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
-      const int gs = gi & 1;
-      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+      const int gs = gi % kGBG, tsl = gi & 1;
+      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGBG) & 1), abort_flag) ||
+          !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -351,8 +375,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         break;
       }
       if (active) {
-        float *u0t = reinterpret_cast<float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_u0);
-        float *cot = reinterpret_cast<float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_coef);
+        float *u0t = reinterpret_cast<float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_u0);
+        float *cot = reinterpret_cast<float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_coef);
         const TI *kg = reinterpret_cast<const TI *>(gb + lay.gb_k);
         const TI *qg = reinterpret_cast<const TI *>(gb + lay.gb_q);
         const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
@@ -392,15 +416,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
-      if (pw == 0 && lane == 0) mbar_arrive(&tfull[gs]);
+      if (pw == 0 && lane == 0) mbar_arrive(&tfull[tsl]);
     }
   } else {
     // ================================================================== consumer warps
-    const int cg = warp >> 2, wid = warp & 3;
-    int ti = 0, group_rdv = 0;
+    // All eight take every tile; warp w owns rows 8w..8w+7 of the 64-row tile.
+    const int row0 = warp * 8;
+    int ti = 0, rdv = 0;
     for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
-      const int gs = gi & 1;
-      if (!mbar_wait_or_abort(&tfull[gs], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+      const int gs = gi % kGBG, tsl = gi & 1;
+      if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -414,15 +439,13 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         const bool fold = m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
                                 : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
-        const float *u0t = reinterpret_cast<const float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_u0);
-        const float *cot = reinterpret_cast<const float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_coef);
-        float *amx = reinterpret_cast<float *>(tabs + (size_t)gs * lay.tab_bytes + lay.tb_amax);
+        const float *u0t = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_u0);
+        const float *cot = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_coef);
+        float *amx = reinterpret_cast<float *>(tabs + lay.tb_amax);  // [2 slots][8 warps], table buffer 0
         const TI *kg = reinterpret_cast<const TI *>(gb + lay.gb_k);
         const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
         const float *bg = reinterpret_cast<const float *>(gb + lay.gb_b);
-        int fold_tiles = 0;
         for (int tt = 0; tt < nh * nrb; ++tt, ++ti) {
-          if ((ti & 1) != cg) continue;
           const int i = tt / nrb, t = tt % nrb;
           const int rows = min(kFp4Rows, R - kFp4Rows * t);
           const int h = h0 + i;
@@ -437,38 +460,35 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           const float g_tile = reinterpret_cast<const float *>(st + lay.st_g)[(unit * nrb + t) & 3];
           const float *co_h = cot + (size_t)i * lay.no * lay.rmax;
           const float *u0_h = u0t + (size_t)i * lay.no * kCols;
+          // 4 consecutive state values of tile row `row` starting at column `col`, from the stage
+          auto load_row4 = [&](int row, int col) -> float4 {
+            if (srcfmt == SRC_F32) return *reinterpret_cast<const float4 *>(st + (row * kCols + col) * 4);
+            if (srcfmt == SRC_F16) {
+              const uint2 hv = *reinterpret_cast<const uint2 *>(st + (row * kCols + col) * 2);
+              const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.x));
+              const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.y));
+              return make_float4(f0.x, f0.y, f1.x, f1.y);
+            }
+            const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + col / 2);
+            const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + col / 16];
+            const float d_b = __fmul_rn(e4m3_value(sc), g_tile);
+            return make_float4(nvfp4_value(cw & 15u, d_b), nvfp4_value((cw >> 4) & 15u, d_b),
+                               nvfp4_value((cw >> 8) & 15u, d_b), nvfp4_value((cw >> 12) & 15u, d_b));
+          };
           if (!fold) {
-            // ---------------- non-fold tile: lane owns columns 4l..4l+3 of 16 rows
-            float4 uv[NO];
+            // ---------------- non-fold tile: lane owns columns 4l..4l+3 of the warp's 8 rows
+            if (row0 < rows) {
+              constexpr int V = 8 * NO;
+              constexpr int KEEP = V >= 32 ? V / 32 : 1;
+              constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
+              float4 uv[NO];
 #pragma unroll
-            for (int j = 0; j < NO; ++j)
-              uv[j] = (j < t_out) ? *reinterpret_cast<const float4 *>(u0_h + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
-            constexpr int V = 8 * NO;
-            constexpr int KEEP = V >= 32 ? V / 32 : 1;
-            constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
-#pragma unroll 1
-            for (int pass = 0; pass < 2; ++pass) {
-              const int r0 = wid * 16 + pass * 8;
-              if (r0 >= rows) break;
+              for (int j = 0; j < NO; ++j)
+                uv[j] = (j < t_out) ? *reinterpret_cast<const float4 *>(u0_h + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
               float part[V];
 #pragma unroll
               for (int rr = 0; rr < 8; ++rr) {
-                const int row = r0 + rr;
-                float4 sv;
-                if (srcfmt == SRC_F32) {
-                  sv = *reinterpret_cast<const float4 *>(st + (row * kCols + 4 * lane) * 4);
-                } else if (srcfmt == SRC_F16) {
-                  const uint2 hv = *reinterpret_cast<const uint2 *>(st + (row * kCols + 4 * lane) * 2);
-                  const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.x));
-                  const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.y));
-                  sv = make_float4(f0.x, f0.y, f1.x, f1.y);
-                } else {
-                  const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + 2 * lane);
-                  const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + (lane >> 2)];
-                  const float d_b = __fmul_rn(e4m3_value(sc), g_tile);
-                  sv = make_float4(nvfp4_value(cw & 15u, d_b), nvfp4_value((cw >> 4) & 15u, d_b),
-                                   nvfp4_value((cw >> 8) & 15u, d_b), nvfp4_value((cw >> 12) & 15u, d_b));
-                }
+                const float4 sv = load_row4(row0 + rr, 4 * lane);
 #pragma unroll
                 for (int j = 0; j < NO; ++j)
                   part[rr * NO + j] = sv.x * uv[j].x + sv.y * uv[j].y + sv.z * uv[j].z + sv.w * uv[j].w;
@@ -476,7 +496,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               // buffered part: lane r adds coef_{j,r} v_r[row] for the 8 rows (one 16-byte load of v_r)
               for (int r = lane; r < n_rec; r += 32) {
                 float vv[8];
-                load8(vr + r * R + kFp4Rows * t + r0, vv);
+                load8(vr + r * R + kFp4Rows * t + row0, vv);
 #pragma unroll
                 for (int j = 0; j < NO; ++j) {
                   const float co = (j < t_out) ? co_h[j * lay.rmax + r] : 0.f;
@@ -489,157 +509,138 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               for (int k2 = 0; k2 < KEEP; ++k2) {
                 const int idx = (V >= 32) ? lane * KEEP + k2 : lane / SPREAD;
                 const int rr = idx / NO, j = idx % NO;
-                const int row = r0 + rr;
-                if (j < t_out && row < rows && (lane % SPREAD) == 0)
-                  a.y[(((size_t)b * a.T + j) * a.H + h) * R + kFp4Rows * t + row] = part[k2];
+                if (j < t_out && (lane % SPREAD) == 0)
+                  a.y[(((size_t)b * a.T + j) * a.H + h) * R + kFp4Rows * t + row0 + rr] = part[k2];
               }
             }
           } else {
-            // ---------------- fold tile: two lanes per row, 64 columns each (chunks rotated by lane)
-            const int row = wid * 16 + (lane >> 1), half = lane & 1;
+            // ---------------- fold tile: four lanes per row, 32 columns each, chunks rotated by lane
+            const int qtr = lane & 3;
+            const int row = row0 + (lane >> 2);
             const bool live = row < rows;
             const int rowg = kFp4Rows * t + row;  // row within the head's state
-            float4 sv[16];
+            float4 sv[8];
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const int ch2 = (q + lane) & 15;
-              const int col = half * 64 + ch2 * 4;
-              float4 v4 = make_float4(0, 0, 0, 0);
-              if (live) {
-                if (srcfmt == SRC_F32) {
-                  v4 = *reinterpret_cast<const float4 *>(st + (row * kCols + col) * 4);
-                } else if (srcfmt == SRC_F16) {
-                  const uint2 hv = *reinterpret_cast<const uint2 *>(st + (row * kCols + col) * 2);
-                  const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.x));
-                  const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.y));
-                  v4 = make_float4(f0.x, f0.y, f1.x, f1.y);
-                } else {
-                  const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + col / 2);
-                  const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + col / 16];
-                  const float d_b = __fmul_rn(e4m3_value(sc), g_tile);
-                  v4 = make_float4(nvfp4_value(cw & 15u, d_b), nvfp4_value((cw >> 4) & 15u, d_b),
-                                   nvfp4_value((cw >> 8) & 15u, d_b), nvfp4_value((cw >> 12) & 15u, d_b));
-                }
-              }
-              sv[q] = v4;
+            for (int c = 0; c < 8; ++c) {
+              const int ch = (c + lane) & 7;
+              sv[c] = live ? load_row4(row, qtr * 32 + ch * 4) : make_float4(0, 0, 0, 0);
             }
-            // sequential row update over the folded records
+            // s <- alpha s + beta (v[row] - alpha (s . k)) k, record by record
             for (int r = 0; r < m; ++r) {
-              const TI *kr = kg + ((size_t)i * lay.rmax + r) * kCols + half * 64;
-              float d = 0.f;
+              const TI *kr = kg + ((size_t)i * lay.rmax + r) * kCols + qtr * 32;
+              float4 kv[8];
 #pragma unroll
-              for (int q = 0; q < 16; ++q) {
-                const float4 kv = load4(kr + ((q + lane) & 15) * 4);
-                d = fmaf(sv[q].x, kv.x, fmaf(sv[q].y, kv.y, fmaf(sv[q].z, kv.z, fmaf(sv[q].w, kv.w, d))));
+              for (int c = 0; c < 8; ++c) kv[c] = load4(kr + ((c + lane) & 7) * 4);
+              float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                d0 = fmaf(sv[c].x, kv[c].x, d0);
+                d1 = fmaf(sv[c].y, kv[c].y, d1);
+                d2 = fmaf(sv[c].z, kv[c].z, d2);
+                d3 = fmaf(sv[c].w, kv[c].w, d3);
               }
+              float d = (d0 + d1) + (d2 + d3);
               d += __shfl_xor_sync(0xffffffffu, d, 1);
+              d += __shfl_xor_sync(0xffffffffu, d, 2);
               const float al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
               const float be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
               const float vrow = live ? to_f32(vr[r * R + rowg]) : 0.f;
               const float coef = be * (vrow - al * d);
 #pragma unroll
-              for (int q = 0; q < 16; ++q) {
-                const float4 kv = load4(kr + ((q + lane) & 15) * 4);
-                sv[q].x = fmaf(al, sv[q].x, coef * kv.x);
-                sv[q].y = fmaf(al, sv[q].y, coef * kv.y);
-                sv[q].z = fmaf(al, sv[q].z, coef * kv.z);
-                sv[q].w = fmaf(al, sv[q].w, coef * kv.w);
+              for (int c = 0; c < 8; ++c) {
+                sv[c].x = fmaf(al, sv[c].x, coef * kv[c].x);
+                sv[c].y = fmaf(al, sv[c].y, coef * kv[c].y);
+                sv[c].z = fmaf(al, sv[c].z, coef * kv[c].z);
+                sv[c].w = fmaf(al, sv[c].w, coef * kv[c].w);
               }
             }
-            // outputs from the fp32 fold result
+            // outputs from the fp32 fold result (u_0 and the coefficients carry q_scale)
             for (int j = 0; j < t_out; ++j) {
-              const float *uj = u0_h + j * kCols + half * 64;
+              const float *uj = u0_h + j * kCols + qtr * 32;
               float z = 0.f;
 #pragma unroll
-              for (int q = 0; q < 16; ++q) {
-                const float4 uv = *reinterpret_cast<const float4 *>(uj + ((q + lane) & 15) * 4);
-                z = fmaf(sv[q].x, uv.x, fmaf(sv[q].y, uv.y, fmaf(sv[q].z, uv.z, fmaf(sv[q].w, uv.w, z))));
+              for (int c = 0; c < 8; ++c) {
+                const float4 uv = *reinterpret_cast<const float4 *>(uj + ((c + lane) & 7) * 4);
+                z = fmaf(sv[c].x, uv.x, fmaf(sv[c].y, uv.y, fmaf(sv[c].z, uv.z, fmaf(sv[c].w, uv.w, z))));
               }
-              z += __shfl_xor_sync(0xffffffffu, z, 1);
               const int e_j = n_rec - t_out + j + 1;
-              float acc = 0.f;
               if (live)
-                for (int r = m + half; r < e_j; r += 2) acc = fmaf(co_h[j * lay.rmax + r], to_f32(vr[r * R + rowg]), acc);
-              acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-              if (live && half == 0) a.y[(((size_t)b * a.T + j) * a.H + h) * R + rowg] = z + acc;
+                for (int r = m + qtr; r < e_j; r += 4) z = fmaf(co_h[j * lay.rmax + r], to_f32(vr[r * R + rowg]), z);
+              z += __shfl_xor_sync(0xffffffffu, z, 1);
+              z += __shfl_xor_sync(0xffffffffu, z, 2);
+              if (live && qtr == 0) a.y[(((size_t)b * a.T + j) * a.H + h) * R + rowg] = z;
             }
             // write the new state: checkpoint format, then the NVFP4 copy
             if (live && !shared_fp4) {
               if (!hp16) {
-                float *dst = reinterpret_cast<float *>(a.hp) + (unit * R + rowg) * kCols + half * 64;
+                float *dst = reinterpret_cast<float *>(a.hp) + (unit * R + rowg) * kCols + qtr * 32;
 #pragma unroll
-                for (int q = 0; q < 16; ++q) __stcs(reinterpret_cast<float4 *>(dst + ((q + lane) & 15) * 4), sv[q]);
+                for (int c = 0; c < 8; ++c) __stcs(reinterpret_cast<float4 *>(dst + ((c + lane) & 7) * 4), sv[c]);
               } else {
-                __half *dst = reinterpret_cast<__half *>(a.hp) + (unit * R + rowg) * kCols + half * 64;
+                __half *dst = reinterpret_cast<__half *>(a.hp) + (unit * R + rowg) * kCols + qtr * 32;
                 const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                  const int ch2 = (q + lane) & 15;
-                  const uint32_t elem = (uint32_t)(rowg * kCols + half * 64 + ch2 * 4);
+                for (int c = 0; c < 8; ++c) {
+                  const int ch = (c + lane) & 7;
+                  const uint32_t elem = (uint32_t)(rowg * kCols + qtr * 32 + ch * 4);
                   const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
-                  const __half h0v = fp16_sr(sv[q].x, rw.x), h1v = fp16_sr(sv[q].y, rw.y);
-                  const __half h2v = fp16_sr(sv[q].z, rw.z), h3v = fp16_sr(sv[q].w, rw.w);
+                  const __half h0v = fp16_sr(sv[c].x, rw.x), h1v = fp16_sr(sv[c].y, rw.y);
+                  const __half h2v = fp16_sr(sv[c].z, rw.z), h3v = fp16_sr(sv[c].w, rw.w);
                   uint2 pk;
                   pk.x = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
                   pk.y = (uint32_t)__half_as_ushort(h2v) | ((uint32_t)__half_as_ushort(h3v) << 16);
-                  *reinterpret_cast<uint2 *>(dst + ch2 * 4) = pk;
+                  *reinterpret_cast<uint2 *>(dst + ch * 4) = pk;
                 }
               }
             }
             if (fp4_read) {
               float am = 0.f;
 #pragma unroll
-              for (int q = 0; q < 16; ++q)
-                am = fmaxf(am, fmaxf(fmaxf(fabsf(sv[q].x), fabsf(sv[q].y)), fmaxf(fabsf(sv[q].z), fabsf(sv[q].w))));
+              for (int c = 0; c < 8; ++c)
+                am = fmaxf(am, fmaxf(fmaxf(fabsf(sv[c].x), fabsf(sv[c].y)), fmaxf(fabsf(sv[c].z), fabsf(sv[c].w))));
 #pragma unroll
               for (int off = 16; off >= 1; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
-              const int slot = fold_tiles & 1;
-              if (lane == 0) amx[(cg * 2 + slot) * 4 + wid] = am;
+              const int slot = rdv & 1;
+              if (lane == 0) amx[slot * 8 + warp] = am;
               __syncwarp();
-              if (lane == 0) mbar_arrive(&csync[cg]);  // the group's four warps have posted their maxima
-              if (!mbar_wait_or_abort(&csync[cg], (uint32_t)(group_rdv & 1), abort_flag)) {
+              if (lane == 0) mbar_arrive(fsync);  // every consumer warp has posted its maximum
+              if (!mbar_wait_or_abort(fsync, (uint32_t)(rdv & 1), abort_flag)) {
                 if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
                 break;
               }
-              ++group_rdv;
-              const float tmax = fmaxf(fmaxf(amx[(cg * 2 + slot) * 4 + 0], amx[(cg * 2 + slot) * 4 + 1]),
-                                       fmaxf(amx[(cg * 2 + slot) * 4 + 2], amx[(cg * 2 + slot) * 4 + 3]));
+              ++rdv;
+              float tmax = 0.f;
+#pragma unroll
+              for (int w = 0; w < kConsumerWarps; ++w) tmax = fmaxf(tmax, amx[slot * 8 + w]);
               const float g = nvfp4_tile_scale(tmax);
-              if (wid == 0 && lane == 0) a.rg[unit * nrb + t] = g;
+              if (warp == 0 && lane == 0) a.rg[unit * nrb + t] = g;
               if (live) {
-                // blocks of 16 columns = 4 chunks; this lane holds blocks half*4 .. half*4+3
-                float bam[4] = {0.f, 0.f, 0.f, 0.f};
+                // this lane's 32 columns are blocks qtr*2 and qtr*2+1; chunk ch lies in block ch >> 2
+                float bam0 = 0.f, bam1 = 0.f;
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                  const int ch2 = (q + lane) & 15;
-                  const float mq = fmaxf(fmaxf(fabsf(sv[q].x), fabsf(sv[q].y)), fmaxf(fabsf(sv[q].z), fabsf(sv[q].w)));
-#pragma unroll
-                  for (int blk = 0; blk < 4; ++blk)
-                    if ((ch2 >> 2) == blk) bam[blk] = fmaxf(bam[blk], mq);
+                for (int c = 0; c < 8; ++c) {
+                  const int ch = (c + lane) & 7;
+                  const float mq = fmaxf(fmaxf(fabsf(sv[c].x), fabsf(sv[c].y)), fmaxf(fabsf(sv[c].z), fabsf(sv[c].w)));
+                  if (ch < 4) bam0 = fmaxf(bam0, mq); else bam1 = fmaxf(bam1, mq);
                 }
-                float db[4];
-                uint32_t scw = 0;
+                float db0, db1;
+                const uint32_t sc0 = nvfp4_block_scale(bam0, g, &db0), sc1 = nvfp4_block_scale(bam1, g, &db1);
+                *reinterpret_cast<uint16_t *>(a.rs + (unit * R + rowg) * (kCols / 16) + qtr * 2) =
+                    (uint16_t)(sc0 | (sc1 << 8));
+                unsigned char *cd = a.rq + (unit * R + rowg) * (kCols / 2) + qtr * 16;
 #pragma unroll
-                for (int blk = 0; blk < 4; ++blk) scw |= nvfp4_block_scale(bam[blk], g, &db[blk]) << (8 * blk);
-                *reinterpret_cast<uint32_t *>(a.rs + (unit * R + rowg) * (kCols / 16) + half * 4) = scw;
-                unsigned char *cd = a.rq + (unit * R + rowg) * (kCols / 2) + half * 32;
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                  const int ch2 = (q + lane) & 15;
-                  float d_b = db[0];
-#pragma unroll
-                  for (int blk = 1; blk < 4; ++blk)
-                    if ((ch2 >> 2) == blk) d_b = db[blk];
-                  const uint32_t cw = nvfp4_code(sv[q].x, d_b) | (nvfp4_code(sv[q].y, d_b) << 4) |
-                                      (nvfp4_code(sv[q].z, d_b) << 8) | (nvfp4_code(sv[q].w, d_b) << 12);
-                  *reinterpret_cast<uint16_t *>(cd + ch2 * 2) = (uint16_t)cw;
+                for (int c = 0; c < 8; ++c) {
+                  const int ch = (c + lane) & 7;
+                  const float d_b = ch < 4 ? db0 : db1;
+                  const uint32_t cw = nvfp4_code(sv[c].x, d_b) | (nvfp4_code(sv[c].y, d_b) << 4) |
+                                      (nvfp4_code(sv[c].z, d_b) << 8) | (nvfp4_code(sv[c].w, d_b) << 12);
+                  *reinterpret_cast<uint16_t *>(cd + ch * 2) = (uint16_t)cw;
                 }
               }
-              ++fold_tiles;
             }
           }
-          // append this head's new v rows (once per head, by the group that owns its first tile)
-          if (t == 0 && wid == 0 && n_new) {
+          // append this head's new v rows (once per head, with its first tile)
+          if (t == 0 && warp == 0 && n_new) {
             const int vq = R * esz / 16;
             for (int q = lane; q < n_new * vq; q += 32) {
               const int tk = q / vq, c16 = q % vq;
@@ -654,14 +655,17 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       if (*abort_flag) break;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&gempty[gs]);
+      if (lane == 0) {  // this warp is done with the unit's group buffer and tables
+        mbar_arrive(&gempty[gs]);
+        mbar_arrive(&tempty[tsl]);
+      }
     }
   }
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s)
       if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1));
-    for (int s = 0; s < 2; ++s)
+    for (int s = 0; s < kGBG; ++s)
       if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
   }
 }
@@ -670,7 +674,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
 
 int g_smem_bytes(int R, int L, int tmax, int esz, int nstage) {
   const GLayout l = g_layout(R, L, tmax, esz);
-  return kBarBytesG + 2 * l.tab_bytes + 2 * l.gb_bytes + nstage * l.stage_bytes;
+  return kBarBytesG + 2 * l.tab_bytes + kGBG * l.gb_bytes + nstage * l.stage_bytes;
 }
 
 int g_max_stages(int R, int L, int tmax, int esz, int budget) {

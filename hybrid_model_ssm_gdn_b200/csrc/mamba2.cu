@@ -75,7 +75,7 @@ __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
 }
 
 // barriers: full[8], empty[8], gfull[3], gempty[3], tfull[2], tempty[2]; then armed phases (ints)
-constexpr int kBarBytes = 256;
+constexpr int kBarBytes = 512;  // mbarriers (26 x 8 B) + armed phases + abort flag
 constexpr int kGB = 3;  // group buffers: the producer loads a unit's group data one unit ahead
 constexpr int kM2Threads = kConsumers + 64;  // + producer warp + prep warp
 constexpr int kProducerWarp = kConsumerWarps, kPrepWarp = kConsumerWarps + 1;
