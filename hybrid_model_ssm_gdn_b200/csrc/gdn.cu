@@ -60,7 +60,7 @@ __host__ __device__ inline int g_heads_per_unit(int no) { return no == 1 ? 4 : n
 struct GLayout {
   int no, rmax, hg, nrb, dts;
   int gb_k, gb_q, gb_a, gb_b, gb_bytes;   // group buffer
-  int tb_u0, tb_coef, tb_amax, tab_bytes; // tables (per buffer)
+  int tb_u0, tb_coef, tb_ab, tb_amax, tab_bytes; // tables (per buffer)
   int st_g, st_v, stage_bytes;            // tile stage: [tile 32 KiB][g chunk 16 B][v records]
 };
 
@@ -78,7 +78,8 @@ __host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz) {
   l.gb_bytes = (int)align_up((size_t)l.gb_b + (size_t)l.hg * l.dts * 4, 128);
   l.tb_u0 = 0;
   l.tb_coef = l.hg * l.no * kCols * 4;
-  l.tb_amax = (int)align_up((size_t)l.tb_coef + (size_t)l.hg * l.no * l.rmax * 4, 16);
+  l.tb_ab = (int)align_up((size_t)l.tb_coef + (size_t)l.hg * l.no * l.rmax * 4, 16);  // {a, b, 1/a, 0}[hg][rmax]
+  l.tb_amax = l.tb_ab + l.hg * l.rmax * 16;
   l.tab_bytes = (int)align_up((size_t)l.tb_amax + 2 * 8 * 4, 128);   // amax[slot][warp]
   l.st_g = kTileMaxBytes;
   l.st_v = l.st_g + 16;
@@ -412,6 +413,17 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             *reinterpret_cast<float4 *>(ud + z) = make_float4(qs * u[z], qs * u[z + 1], qs * u[z + 2], qs * u[z + 3]);
         }
       }
+      if (active && m > 0) {  // per-record scalars of the fold: {alpha, beta, 1/alpha}
+        float4 *abt = reinterpret_cast<float4 *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_ab);
+        const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
+        const float *bg = reinterpret_cast<const float *>(gb + lay.gb_b);
+        for (int q = pw * 32 + lane; q < nh * m; q += 64) {
+          const int i = q / m, r = q % m;
+          const float al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
+          const float be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
+          abt[i * lay.rmax + r] = make_float4(al, be, __frcp_rn(al), 0.f);
+        }
+      }
       if (!prep_sync()) {  // tables complete
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
@@ -422,6 +434,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     // ================================================================== consumer warps
     // All eight take every tile; warp w owns rows 8w..8w+7 of the 64-row tile.
     const int row0 = warp * 8;
+    const uint64_t pol_wr = policy_evict_first();
     int ti = 0, rdv = 0;
     for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
@@ -431,11 +444,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
-      const float *gf = reinterpret_cast<const float *>(gb);
       const int b = gh[Q_B], h0 = gh[Q_H0], nh = gh[Q_NH];
       if (gh[Q_ACTIVE]) {
         const int n_rec = gh[Q_NREC], m = gh[Q_M], n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], t_out = gh[Q_TOUT];
-        const int slot0 = gh[Q_SLOT0], base_e = gh[Q_BASE], me = gh[Q_ME];
+        const int slot0 = gh[Q_SLOT0], me = gh[Q_ME];
         const bool fold = m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
                                 : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
@@ -443,8 +455,6 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         const float *cot = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_coef);
         float *amx = reinterpret_cast<float *>(tabs + lay.tb_amax);  // [2 slots][8 warps], table buffer 0
         const TI *kg = reinterpret_cast<const TI *>(gb + lay.gb_k);
-        const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
-        const float *bg = reinterpret_cast<const float *>(gb + lay.gb_b);
         for (int tt = 0; tt < nh * nrb; ++tt, ++ti) {
           const int i = tt / nrb, t = tt % nrb;
           const int rows = min(kFp4Rows, R - kFp4Rows * t);
@@ -485,14 +495,21 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
 #pragma unroll
               for (int j = 0; j < NO; ++j)
                 uv[j] = (j < t_out) ? *reinterpret_cast<const float4 *>(u0_h + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
+              float4 sv[8];
+              if (srcfmt == SRC_F32) {
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr)
+                  sv[rr] = *reinterpret_cast<const float4 *>(st + ((row0 + rr) * kCols + 4 * lane) * 4);
+              } else {
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) sv[rr] = load_row4(row0 + rr, 4 * lane);
+              }
               float part[V];
 #pragma unroll
-              for (int rr = 0; rr < 8; ++rr) {
-                const float4 sv = load_row4(row0 + rr, 4 * lane);
+              for (int rr = 0; rr < 8; ++rr)
 #pragma unroll
                 for (int j = 0; j < NO; ++j)
-                  part[rr * NO + j] = sv.x * uv[j].x + sv.y * uv[j].y + sv.z * uv[j].z + sv.w * uv[j].w;
-              }
+                  part[rr * NO + j] = sv[rr].x * uv[j].x + sv[rr].y * uv[j].y + sv[rr].z * uv[j].z + sv[rr].w * uv[j].w;
               // buffered part: lane r adds coef_{j,r} v_r[row] for the 8 rows (one 16-byte load of v_r)
               for (int r = lane; r < n_rec; r += 32) {
                 float vv[8];
@@ -525,12 +542,20 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               const int ch = (c + lane) & 7;
               sv[c] = live ? load_row4(row, qtr * 32 + ch * 4) : make_float4(0, 0, 0, 0);
             }
-            // s <- alpha s + beta (v[row] - alpha (s . k)) k, record by record
+            // s <- alpha s + beta (v[row] - alpha (s . k)) k, record by record.  The row is kept as
+            // s = sig * s~ so that each record costs one FMA per element: s~ += (coef / sig') k with
+            // sig' = alpha sig, and s . k = sig (s~ . k); s~ is rescaled if sig gets small.
+            float sig = 1.f, isig = 1.f;
+            const float4 *abt = reinterpret_cast<const float4 *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_ab) +
+                                (size_t)i * lay.rmax;
             for (int r = 0; r < m; ++r) {
               const TI *kr = kg + ((size_t)i * lay.rmax + r) * kCols + qtr * 32;
               float4 kv[8];
 #pragma unroll
               for (int c = 0; c < 8; ++c) kv[c] = load4(kr + ((c + lane) & 7) * 4);
+              const float4 abr = abt[r];
+              const float al = abr.x, be = abr.y;
+              const float vrow = live ? to_f32(vr[r * R + rowg]) : 0.f;
               float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
@@ -542,17 +567,27 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               float d = (d0 + d1) + (d2 + d3);
               d += __shfl_xor_sync(0xffffffffu, d, 1);
               d += __shfl_xor_sync(0xffffffffu, d, 2);
-              const float al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
-              const float be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
-              const float vrow = live ? to_f32(vr[r * R + rowg]) : 0.f;
-              const float coef = be * (vrow - al * d);
+              const float coef = be * (vrow - al * (sig * d));
+              sig *= al;
+              isig *= abr.z;
+              if (sig < 9.3e-10f) {  // 2^-30: fold the scale back into the row
+#pragma unroll
+                for (int c = 0; c < 8; ++c) { sv[c].x *= sig; sv[c].y *= sig; sv[c].z *= sig; sv[c].w *= sig; }
+                sig = 1.f;
+                isig = 1.f;
+              }
+              const float cs = coef * isig;
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
-                sv[c].x = fmaf(al, sv[c].x, coef * kv[c].x);
-                sv[c].y = fmaf(al, sv[c].y, coef * kv[c].y);
-                sv[c].z = fmaf(al, sv[c].z, coef * kv[c].z);
-                sv[c].w = fmaf(al, sv[c].w, coef * kv[c].w);
+                sv[c].x = fmaf(cs, kv[c].x, sv[c].x);
+                sv[c].y = fmaf(cs, kv[c].y, sv[c].y);
+                sv[c].z = fmaf(cs, kv[c].z, sv[c].z);
+                sv[c].w = fmaf(cs, kv[c].w, sv[c].w);
               }
+            }
+            if (sig != 1.f) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) { sv[c].x *= sig; sv[c].y *= sig; sv[c].z *= sig; sv[c].w *= sig; }
             }
             // outputs from the fp32 fold result (u_0 and the coefficients carry q_scale)
             for (int j = 0; j < t_out; ++j) {
@@ -570,27 +605,40 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               z += __shfl_xor_sync(0xffffffffu, z, 2);
               if (live && qtr == 0) a.y[(((size_t)b * a.T + j) * a.H + h) * R + rowg] = z;
             }
-            // write the new state: checkpoint format, then the NVFP4 copy
-            if (live && !shared_fp4) {
-              if (!hp16) {
-                float *dst = reinterpret_cast<float *>(a.hp) + (unit * R + rowg) * kCols + qtr * 32;
+            // write the new state in the checkpoint format: each lane puts its values back where it
+            // read them in the stage, then one bulk store per warp moves the warp's rows (contiguous
+            // in shared and in global memory) with full-line writes
+            if (!shared_fp4) {
+              unsigned char *stw = stages + (size_t)s * lay.stage_bytes;
+              if (live) {
+                if (!hp16) {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) __stcs(reinterpret_cast<float4 *>(dst + ((c + lane) & 7) * 4), sv[c]);
-              } else {
-                __half *dst = reinterpret_cast<__half *>(a.hp) + (unit * R + rowg) * kCols + qtr * 32;
-                const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+                  for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4 *>(stw + (row * kCols + qtr * 32 + ((c + lane) & 7) * 4) * 4) = sv[c];
+                } else {
+                  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                  const int ch = (c + lane) & 7;
-                  const uint32_t elem = (uint32_t)(rowg * kCols + qtr * 32 + ch * 4);
-                  const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
-                  const __half h0v = fp16_sr(sv[c].x, rw.x), h1v = fp16_sr(sv[c].y, rw.y);
-                  const __half h2v = fp16_sr(sv[c].z, rw.z), h3v = fp16_sr(sv[c].w, rw.w);
-                  uint2 pk;
-                  pk.x = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
-                  pk.y = (uint32_t)__half_as_ushort(h2v) | ((uint32_t)__half_as_ushort(h3v) << 16);
-                  *reinterpret_cast<uint2 *>(dst + ch * 4) = pk;
+                  for (int c = 0; c < 8; ++c) {
+                    const int ch = (c + lane) & 7;
+                    const uint32_t elem = (uint32_t)(rowg * kCols + qtr * 32 + ch * 4);
+                    const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
+                    const __half h0v = fp16_sr(sv[c].x, rw.x), h1v = fp16_sr(sv[c].y, rw.y);
+                    const __half h2v = fp16_sr(sv[c].z, rw.z), h3v = fp16_sr(sv[c].w, rw.w);
+                    uint2 pk;
+                    pk.x = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
+                    pk.y = (uint32_t)__half_as_ushort(h2v) | ((uint32_t)__half_as_ushort(h3v) << 16);
+                    *reinterpret_cast<uint2 *>(stw + (row * kCols + qtr * 32 + ch * 4) * 2) = pk;
+                  }
                 }
+              }
+              fence_async_smem();
+              __syncwarp();
+              const int wrows = min(8, rows - row0);
+              if (lane == 0 && wrows > 0) {
+                const int esz_hp = hp16 ? 2 : 4;
+                bulk_s2g(static_cast<unsigned char *>(a.hp) + (unit * R + kFp4Rows * t + row0) * kCols * esz_hp,
+                         stw + row0 * kCols * esz_hp, (uint32_t)(wrows * kCols * esz_hp), pol_wr);
+                bulk_commit();
               }
             }
             if (fp4_read) {
@@ -649,6 +697,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                                          ((unit * 2 * L + slot0 + tk) * R) * esz + c16 * 16) = v;
             }
           }
+          if (lane == 0) bulk_wait_read();  // a bulk store of this stage must have read it before release
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[s]);
         }
@@ -660,6 +709,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         mbar_arrive(&tempty[tsl]);
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {

@@ -55,6 +55,7 @@ struct M2Layout {
   int stage_bytes;
   int gb_B, gb_C, gb_dt, gb_bytes;  // group buffer
   int tab_bytes;
+  int cx_bytes;              // fold scratch: per consumer warp, wf_r x_r[row] for its 8 rows
 };
 
 __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
@@ -71,6 +72,7 @@ __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
   // tables: g[no][rmax], coef[kHG][no][rmax], ao[kHG][no], wf[kHG][rmax], af[kHG], flags[8]
   const int floats = l.no * l.rmax + kHG * l.no * l.rmax + kHG * l.no + kHG * l.rmax + kHG + 8;
   l.tab_bytes = (int)align_up((size_t)floats * 4, 128);
+  l.cx_bytes = (int)align_up((size_t)kConsumerWarps * l.rmax * 8 * 4, 128);
   return l;
 }
 
@@ -96,7 +98,8 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   volatile int *abort_flag = armed + 8 + kGB;
   const int rmax = lay.rmax;
   unsigned char *tabs = smem + kBarBytes;  // two table buffers
-  unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
+  float *cx_scratch = reinterpret_cast<float *>(tabs + 2 * lay.tab_bytes);  // [8 warps][rmax][8 rows]
+  unsigned char *gbuf = tabs + 2 * lay.tab_bytes + lay.cx_bytes;
   unsigned char *stages = gbuf + kGB * lay.gb_bytes;
   struct Tables {
     float *g, *coef, *ao, *wf, *af;
@@ -427,20 +430,30 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
               const float af = t_af[i];
 #pragma unroll
               for (int rr = 0; rr < 8; ++rr) { sv[rr].x *= af; sv[rr].y *= af; sv[rr].z *= af; sv[rr].w *= af; }
-              for (int r = 0; r < m; ++r) {
-                const float4 bv = load4(Bg + r * kCols + 4 * lane);
-                const float wr = t_wf[i * rmax + r];
+              // lane r forms wf_r x_r[row] for the warp's 8 rows in its warp's scratch rows
+              float *cxw = cx_scratch + (size_t)warp * rmax * 8;
+              for (int r = lane; r < m; r += 32) {
                 float xv[8];
                 load8(xr + r * a.P + row0, xv);
+                const float wr = t_wf[i * rmax + r];
+                *reinterpret_cast<float4 *>(cxw + r * 8) = make_float4(wr * xv[0], wr * xv[1], wr * xv[2], wr * xv[3]);
+                *reinterpret_cast<float4 *>(cxw + r * 8 + 4) = make_float4(wr * xv[4], wr * xv[5], wr * xv[6], wr * xv[7]);
+              }
+              __syncwarp();
+              for (int r = 0; r < m; ++r) {
+                const float4 bv = load4(Bg + r * kCols + 4 * lane);
+                const float4 c0 = *reinterpret_cast<const float4 *>(cxw + r * 8);
+                const float4 c1 = *reinterpret_cast<const float4 *>(cxw + r * 8 + 4);
+                const float cx[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
-                  const float cx = wr * xv[rr];
-                  sv[rr].x = fmaf(cx, bv.x, sv[rr].x);
-                  sv[rr].y = fmaf(cx, bv.y, sv[rr].y);
-                  sv[rr].z = fmaf(cx, bv.z, sv[rr].z);
-                  sv[rr].w = fmaf(cx, bv.w, sv[rr].w);
+                  sv[rr].x = fmaf(cx[rr], bv.x, sv[rr].x);
+                  sv[rr].y = fmaf(cx[rr], bv.y, sv[rr].y);
+                  sv[rr].z = fmaf(cx[rr], bv.z, sv[rr].z);
+                  sv[rr].w = fmaf(cx[rr], bv.w, sv[rr].w);
                 }
               }
+              __syncwarp();
               float *dst = a.hp + unit * a.P * kCols;
 #pragma unroll
               for (int rr = 0; rr < 8; ++rr)
@@ -512,7 +525,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
 
 int m2_smem_bytes(int P, int L, int tmax, int esz, int nstage) {
   const M2Layout l = m2_layout(P, L, tmax, esz);
-  return kBarBytes + 2 * l.tab_bytes + kGB * l.gb_bytes + nstage * l.stage_bytes;
+  return kBarBytes + 2 * l.tab_bytes + l.cx_bytes + kGB * l.gb_bytes + nstage * l.stage_bytes;
 }
 
 int m2_max_stages(int P, int L, int tmax, int esz, int smem_budget) {

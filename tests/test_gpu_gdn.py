@@ -135,19 +135,36 @@ FLIP_FRACTION = 0.02
 
 @pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f16sr", "same"), ("f32", "shared_nvfp4")])
 def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
+    """With stochastic rounding the oracle's trajectory is one sample among many, so the GPU is held to
+    the spread between two oracle seeds (mean error at most twice the seed-to-seed mean, plus the fp32
+    bound); without it, to rare single-code NVFP4 flips."""
+    from oracle.decoder import ReplayOracle
     wl = GDN_LOWPREC.replace(batch=4, nheads=4, window=8)
     p = Pair(wl, hp=hp, read=read, seed=7)
-    errs = []
+    other = None
+    if hp == "f16sr":
+        from synth import gdn_initial_state
+        other = ReplayOracle("gdn", gdn_initial_state(wl), wl.window, nheads=wl.nheads, hp=hp, read=read, seed=8)
+    errs, spread = [], []
     for t in range(48):
-        y, y_ref, y_true = p.step(gdn_step_inputs(wl, t))
+        inp = gdn_step_inputs(wl, t)
+        y, y_ref, y_true = p.step(inp)
         err = head_rel_err(y, y_ref)
         errs.append(err.ravel())
         assert err.max() <= TOL_FLIP, f"step {t}: {err.max():.3e}"
+        if other is not None:
+            y_other, _ = other.step(inp)
+            spread.append(head_rel_err(y_other, y_ref).ravel())
         p.check_bookkeeping(ring=(t % 8 == 7))
     errs = np.concatenate(errs)
     frac = float(np.mean(errs > TOL_F32))
     print(f"{hp}/{read}: max {errs.max():.3e}, median {np.median(errs):.3e}, fraction above 1e-4 {frac:.4f}")
-    assert frac <= FLIP_FRACTION
+    if other is not None:
+        spread = np.concatenate(spread)
+        print(f"  seed-to-seed spread: mean {spread.mean():.3e}, GPU mean {errs.mean():.3e}")
+        assert errs.mean() <= 2 * spread.mean() + TOL_F32
+    else:
+        assert frac <= FLIP_FRACTION
 
 
 @pytest.mark.slow
