@@ -463,6 +463,39 @@ def verify_section(rounds: int) -> dict:
     return out
 
 
+def window_section(windows=(4, 8, 16, 32), windows_timed: int = 8) -> dict:
+    """Mamba-2 batch-256 layer at several windows L: amortised step time vs the traffic model."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    p = mamba2_params(WL)
+    A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
+    S0 = torch.from_numpy(mamba2_initial_state(WL)).to(dev)
+    pool = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in mamba2_step_inputs(WL, t).items()} for t in range(8)]
+    y = torch.empty(WL.batch, WL.nheads, WL.headdim, device=dev)
+    stream = torch.cuda.current_stream()
+    out = {"workload": "mamba2 replay decode, batch 256, 128 heads, P 64, N 128, 8 groups, bf16 inputs, fp32 checkpoint"}
+    for L in windows:
+        wl = WL.replace(window=L)
+        layer = ReplaySSM("mamba2", wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, L, 0, bf, A=A, D=D)
+        layer.load_checkpoint(S0)
+
+        def step(i):
+            t = pool[i % 8]
+            layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], y)
+
+        for i in range(2 * L):
+            step(i)
+        K = L * max(windows_timed, 64 // L)
+        ms = timed(step, K, stream)
+        model = sum(sum(traffic_model(wl, i % L).values()) for i in range(K)) / K
+        out[f"L{L}"] = {"ms_per_step": ms, "tokens_per_s": wl.batch / (ms * 1e-3), "model_bytes_per_step": model,
+                        "GBps": model / (ms * 1e-3) / 1e9, "device_error": layer.get_error()}
+        del layer
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -471,7 +504,7 @@ def main():
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN and speculative-verify sections")
-    ap.add_argument("--only", choices=["gdn", "verify"], default=None,
+    ap.add_argument("--only", choices=["gdn", "verify", "window"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -487,7 +520,8 @@ def main():
 
     if args.only is not None:
         if rank == 0:
-            out = gdn_section(args.steps) if args.only == "gdn" else verify_section(args.steps)
+            out = (gdn_section(args.steps) if args.only == "gdn" else
+                   verify_section(args.steps) if args.only == "verify" else window_section())
             print(json.dumps(out))
         return
 
