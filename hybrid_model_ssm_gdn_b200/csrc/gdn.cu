@@ -362,6 +362,15 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           a.ring_a[unit * dts + slot0 + t] = al;
           a.ring_b[unit * dts + slot0 + t] = be;
         }
+        const int vq = R * esz / 16;  // v rows of the new tokens, straight from the inputs
+        for (int q = pw * 32 + lane; q < n_new * nh * vq; q += 64) {
+          const int c16 = q % vq, ti2 = q / vq, t = ti2 / nh, i = ti2 % nh;
+          const size_t unit = (size_t)b * a.H + h0 + i;
+          const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.v) +
+                                                           (((size_t)b * a.T + t) * a.H + h0 + i) * R * esz + c16 * 16);
+          *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_v) + ((unit * 2 * L + slot0 + t) * R) * esz +
+                                     c16 * 16) = v;
+        }
         const int kq = kCols * esz / 16;
         for (int q = pw * 32 + lane; q < n_new * nh * kq; q += 64) {
           const int c16 = q % kq, ti2 = q / kq, t = ti2 / nh, i = ti2 % nh;
@@ -446,8 +455,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       const int *gh = reinterpret_cast<const int *>(gb);
       const int b = gh[Q_B], h0 = gh[Q_H0], nh = gh[Q_NH];
       if (gh[Q_ACTIVE]) {
-        const int n_rec = gh[Q_NREC], m = gh[Q_M], n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], t_out = gh[Q_TOUT];
-        const int slot0 = gh[Q_SLOT0], me = gh[Q_ME];
+        const int n_rec = gh[Q_NREC], m = gh[Q_M], t_out = gh[Q_TOUT];
+        const int me = gh[Q_ME];
         const bool fold = m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
                                 : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
@@ -685,16 +694,6 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                   *reinterpret_cast<uint16_t *>(cd + ch * 2) = (uint16_t)cw;
                 }
               }
-            }
-          }
-          // append this head's new v rows (once per head, with its first tile)
-          if (t == 0 && warp == 0 && n_new) {
-            const int vq = R * esz / 16;
-            for (int q = lane; q < n_new * vq; q += 32) {
-              const int tk = q / vq, c16 = q % vq;
-              const uint4 v = *reinterpret_cast<const uint4 *>(st + lay.st_v + (n_ring + tk) * R * esz + c16 * 16);
-              *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_v) +
-                                         ((unit * 2 * L + slot0 + tk) * R) * esz + c16 * 16) = v;
             }
           }
           if (lane == 0) bulk_wait_read();  // a bulk store of this stage must have read it before release

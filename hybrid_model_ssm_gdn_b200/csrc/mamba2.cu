@@ -347,6 +347,22 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
                                        ((((size_t)b * a.G + g) * 2 * a.L + slot0 + t) * kCols) * esz + c16 * 16) = v;
           }
         }
+        // x rows and dt of the new tokens go to each head's ring row, straight from the inputs
+        {
+          const int xq = a.P * esz / 16;
+          for (int q = lane; q < n_new * nh * xq; q += 32) {
+            const int c16 = q % xq, ti2 = q / xq, t = ti2 / nh, i = ti2 % nh;
+            const size_t unit = (size_t)b * a.H + h0 + i;
+            const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.x) +
+                                                             (((size_t)b * a.T + t) * a.H + h0 + i) * a.P * esz + c16 * 16);
+            *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
+                                       ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v;
+          }
+          for (int q = lane; q < n_new * nh; q += 32) {
+            const int t = q / nh, i = q % nh;
+            a.ring_dt[((size_t)b * a.H + h0 + i) * dts + slot0 + t] = gf[G_DT + t * kHG + i];
+          }
+        }
         __syncwarp();
         // per-head weights of every record in every output (log-space suffix sums of dt):
         // coef[r] = dt_r exp(A s(r+1, e_j)) (B_r . C_j) for m <= r < e_j, plus D on the output's
@@ -394,14 +410,11 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
-      const float *gf = reinterpret_cast<const float *>(gb);
       const int b = gh[G_B], h0 = gh[G_H0], nh = gh[G_NH];
       if (gh[G_ACTIVE]) {
         const Tables T = tables(tsl);
         const float *t_coef = T.coef, *t_ao = T.ao, *t_wf = T.wf, *t_af = T.af;
-        const int n_rec = gh[G_NREC], m = gh[G_M], n_ring = gh[G_NRING], n_new = gh[G_NNEW], t_out = gh[G_TOUT];
-        const int slot0 = gh[G_SLOT0];
-        const int dts = dt_stride(a.L);
+        const int n_rec = gh[G_NREC], m = gh[G_M], t_out = gh[G_TOUT];
         const TI *Bg = reinterpret_cast<const TI *>(gb + lay.gb_B);
         const TI *Cg = reinterpret_cast<const TI *>(gb + lay.gb_C);
         // ---- stream the heads' tiles; each warp works and releases on its own
@@ -488,16 +501,6 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
               if (j < t_out && (lane % SPREAD) == 0)
                 a.y[(((size_t)b * a.T + j) * a.H + h) * a.P + row0 + rr] = part[k2];
             }
-          }
-          if (warp == 0 && n_new) {  // append this head's new tokens (x rows, dt) to its ring row
-            const int xq = a.P * esz / 16;
-            for (int q = lane; q < n_new * xq; q += 32) {
-              const int t = q / xq, c16 = q % xq;
-              const uint4 v = *reinterpret_cast<const uint4 *>(st + lay.xr + (n_ring + t) * a.P * esz + c16 * 16);
-              *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
-                                         ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v;
-            }
-            if (lane < n_new) a.ring_dt[unit * dts + slot0 + lane] = gf[G_DT + lane * kHG + i];
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[s]);
