@@ -79,6 +79,24 @@ def weak_scaling_value(tokens_per_rank_step: int, world: int, steps: int, max_ms
     return tokens_per_rank_step * world * steps / (max_ms * 1e-3)
 
 
+def profiled_traffic(summary: str, sources) -> "float | None":
+    """DRAM bytes per launch from the committed ncu summary, or None if the kernel changed since it was taken."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = hashlib.sha1()
+    for f in sources:
+        m.update(open(os.path.join(ROOT, "hybrid_model_ssm_gdn_b200", "csrc", f), "rb").read())
+    h = re.search(r"Kernel source hash[^`]*`([0-9a-f]+)`", text)
+    t = re.search(r"traffic_bytes_per_launch_window_avg:\s*([0-9.]+)", text)
+    if not h or not t or h.group(1) != m.hexdigest():
+        return None
+    return float(t.group(1))
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -309,7 +327,9 @@ def run_gpu(args, rank, world):
                    "parallelism": f"replicas x{world} (batch shards, no collective)",
                    "l2": "checkpoint stream (1 GiB/step) exceeds L2; no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "peak_kind": peak_kind, "traffic": None,
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "traffic": profiled_traffic("m2_replay_kernel__mamba2_b256_L16.md",
+                                                 ("mamba2.cu", "common.cuh", "kernels.h")),
                      "kernel": "m2_replay_kernel", "bytes_per_launch": bytes_avg,
                      "mean_launch_ms": mean_launch_ms,
                      "fold_launch_ms": statistics.mean(fold_ms) if fold_ms else None,
