@@ -362,14 +362,30 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           a.ring_a[unit * dts + slot0 + t] = al;
           a.ring_b[unit * dts + slot0 + t] = be;
         }
-        const int vq = R * esz / 16;  // v rows of the new tokens, straight from the inputs
-        for (int q = pw * 32 + lane; q < n_new * nh * vq; q += 64) {
-          const int c16 = q % vq, ti2 = q / vq, t = ti2 / nh, i = ti2 % nh;
-          const size_t unit = (size_t)b * a.H + h0 + i;
-          const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.v) +
-                                                           (((size_t)b * a.T + t) * a.H + h0 + i) * R * esz + c16 * 16);
-          *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_v) + ((unit * 2 * L + slot0 + t) * R) * esz +
-                                     c16 * 16) = v;
+        {  // v rows of the new tokens, straight from the inputs: eight 16-byte loads in flight per lane
+          const int vq = R * esz / 16, nq = n_new * nh * vq;
+          for (int q0 = 0; q0 < nq; q0 += 512) {
+            uint4 v[8];
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+              const int q = q0 + k2 * 64 + pw * 32 + lane;
+              if (q < nq) {
+                const int c16 = q % vq, ti2 = q / vq, t = ti2 / nh, i = ti2 % nh;
+                v[k2] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.v) +
+                                                         (((size_t)b * a.T + t) * a.H + h0 + i) * R * esz + c16 * 16);
+              }
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+              const int q = q0 + k2 * 64 + pw * 32 + lane;
+              if (q < nq) {
+                const int c16 = q % vq, ti2 = q / vq, t = ti2 / nh, i = ti2 % nh;
+                const size_t unit = (size_t)b * a.H + h0 + i;
+                *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_v) +
+                                           ((unit * 2 * L + slot0 + t) * R) * esz + c16 * 16) = v[k2];
+              }
+            }
+          }
         }
         const int kq = kCols * esz / 16;
         for (int q = pw * 32 + lane; q < n_new * nh * kq; q += 64) {

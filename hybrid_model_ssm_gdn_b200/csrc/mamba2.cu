@@ -300,14 +300,23 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       if (gh[G_WMETA] && lane == 0) a.meta_out[b] = make_int4(gh[G_MC], gh[G_ME], gh[G_MP], 0);
       // per-head parameters and the new tokens' dt (global loads, kept off the producer's path)
       float *gfw = reinterpret_cast<float *>(gbuf + (size_t)gs * lay.gb_bytes);
-      if (lane < nh) {
-        gfw[G_A + lane] = a.A[h0 + lane];
-        gfw[G_D + lane] = a.D[h0 + lane];
-      }
-      if (gh[G_ACTIVE]) {
-        for (int q = lane; q < gh[G_NNEW] * nh; q += 32) {
-          const int t = q / nh, i = q % nh;
-          gfw[G_DT + t * kHG + i] = to_f32(reinterpret_cast<const TI *>(a.dt)[((size_t)b * a.T + t) * a.H + h0 + i]);
+      {  // all loads issued before any is used (at most 8 tokens x 16 heads = 4 per lane)
+        const int nq = gh[G_ACTIVE] ? gh[G_NNEW] * nh : 0;
+        float dtv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int q = lane + 32 * k, t = q / max(nh, 1), i = q % max(nh, 1);
+          dtv[k] = q < nq ? to_f32(reinterpret_cast<const TI *>(a.dt)[((size_t)b * a.T + t) * a.H + h0 + i]) : 0.f;
+        }
+        const float Av = lane < nh ? a.A[h0 + lane] : 0.f, Dv = lane < nh ? a.D[h0 + lane] : 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int q = lane + 32 * k;
+          if (q < nq) gfw[G_DT + (q / nh) * kHG + q % nh] = dtv[k];
+        }
+        if (lane < nh) {
+          gfw[G_A + lane] = Av;
+          gfw[G_D + lane] = Dv;
         }
       }
       __syncwarp();
@@ -347,21 +356,37 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
                                        ((((size_t)b * a.G + g) * 2 * a.L + slot0 + t) * kCols) * esz + c16 * 16) = v;
           }
         }
-        // x rows and dt of the new tokens go to each head's ring row, straight from the inputs
+        // x rows of the new tokens go to each head's ring row, straight from the inputs: eight
+        // 16-byte loads in flight per lane before the stores
         {
-          const int xq = a.P * esz / 16;
-          for (int q = lane; q < n_new * nh * xq; q += 32) {
-            const int c16 = q % xq, ti2 = q / xq, t = ti2 / nh, i = ti2 % nh;
-            const size_t unit = (size_t)b * a.H + h0 + i;
-            const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.x) +
-                                                             (((size_t)b * a.T + t) * a.H + h0 + i) * a.P * esz + c16 * 16);
-            *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
-                                       ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v;
+          const int xq = a.P * esz / 16, nq = n_new * nh * xq;
+          for (int q0 = 0; q0 < nq; q0 += 256) {
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int q = q0 + k * 32 + lane;
+              if (q < nq) {
+                const int c16 = q % xq, ti2 = q / xq, t = ti2 / nh, i = ti2 % nh;
+                v[k] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.x) +
+                                                        (((size_t)b * a.T + t) * a.H + h0 + i) * a.P * esz + c16 * 16);
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int q = q0 + k * 32 + lane;
+              if (q < nq) {
+                const int c16 = q % xq, ti2 = q / xq, t = ti2 / nh, i = ti2 % nh;
+                const size_t unit = (size_t)b * a.H + h0 + i;
+                *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
+                                           ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v[k];
+              }
+            }
           }
-          for (int q = lane; q < n_new * nh; q += 32) {
-            const int t = q / nh, i = q % nh;
-            a.ring_dt[((size_t)b * a.H + h0 + i) * dts + slot0 + t] = gf[G_DT + t * kHG + i];
-          }
+        }
+        // dt of the new tokens goes to each head's ring row
+        for (int q = lane; q < n_new * nh; q += 32) {
+          const int t = q / nh, i = q % nh;
+          a.ring_dt[((size_t)b * a.H + h0 + i) * dts + slot0 + t] = gf[G_DT + t * kHG + i];
         }
         __syncwarp();
         // per-head weights of every record in every output (log-space suffix sums of dt):
