@@ -33,7 +33,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import (GDN_B256, MAMBA2_120B, SPEC_MAMBA2_B512, accepted_lengths, gdn_initial_state,  # noqa: E402
+from synth import (GDN_B256, MAMBA2_120B, SPEC_MAMBA2_B512, accepted_lengths, gdn_draft_inputs,  # noqa: E402
+                   gdn_initial_state,
                    gdn_step_inputs, mamba2_draft_inputs, mamba2_initial_state, mamba2_params, mamba2_step_inputs)
 
 WL = MAMBA2_120B
@@ -55,6 +56,35 @@ def traffic_model(wl, count_before: int) -> dict:
     fold = count_before + 1 == L
     return {"state_read": state, "state_write": state if fold else 0, "ring_read": count_before * rec,
             "inputs": tok, "append": rec, "y": Bt * H * P * 4}
+
+
+def verify_traffic(wl, T: int, accepted) -> float:
+    """Algorithmic HBM bytes of the verify + commit rounds with the given accepted lengths, from count 0.
+
+    Per sequence and round: checkpoint read, plus its write and the window's records when the verify
+    pre-folds (count + T > L); buffered records read otherwise; T tokens' inputs read, T records appended,
+    T fp32 outputs written.  Commit moves bookkeeping words only.
+    """
+    Bt, H, L = wl.batch, wl.nheads, wl.window
+    esz = 2 if wl.in_dtype == "bf16" else 4
+    if wl.kind == "mamba2":
+        P, N, G = wl.headdim, wl.dstate, wl.ngroups
+        state, y = H * P * N * 4, H * P * 4
+        rec = H * P * esz + G * N * esz + H * 4                 # x, B, dt (fp32)
+        tok = H * P * esz + 2 * G * N * esz + H * esz            # x, B, C, dt
+    else:
+        dk, dv = wl.dk, wl.dv
+        state, y = H * dv * dk * 4, H * dv * 4
+        rec = H * (dk * esz + dv * esz + 8)                      # k, v, alpha, beta (fp32)
+        tok = H * (2 * dk * esz + dv * esz + 8)                  # q, k, v, alpha, beta
+    count = np.zeros(Bt, np.int64)
+    total = 0.0
+    for acc in accepted:
+        fold = count + T > L
+        total += Bt * state + int(fold.sum()) * state + int(count.sum()) * rec
+        total += Bt * T * (tok + rec + y)
+        count = np.where(fold, 0, count) + np.asarray(acc, np.int64)
+    return total
 
 
 def conventional_bytes(wl) -> int:
@@ -463,57 +493,69 @@ def gdn_section(steps: int) -> dict:
 
 
 def verify_section(rounds: int) -> dict:
-    """Speculative verify + commit on the Mamba-2 shape at batch 512 (T = 4, 8) vs snapshot-per-draft."""
+    """Speculative verify + commit (T = 4, 8) vs snapshot-per-draft: the Mamba-2 shape at batch 512 and the
+    Gated DeltaNet layer at batch 256."""
     import torch
 
     from hybrid_model_ssm_gdn_b200 import ReplaySSM, make_config, snap_commit, snap_verify
-    wl, dev, bf = SPEC_MAMBA2_B512, torch.device("cuda"), torch.bfloat16
-    p = mamba2_params(wl)
-    A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
-    stream = torch.cuda.current_stream()
-    S0 = torch.from_numpy(mamba2_initial_state(wl)).to(dev)
-    out = {"workload": "mamba2 speculative verify + commit, batch 512, 128 heads, P 64, N 128, 8 groups, L 16"}
-    for T in (4, 8):
-        layer = ReplaySSM("mamba2", wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window, T, bf,
-                          A=A, D=D)
-        layer.load_checkpoint(S0)
-        drafts = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in mamba2_draft_inputs(wl, r, T).items()}
-                  for r in range(4)]
-        accs = [torch.from_numpy(accepted_lengths(wl, r, T)).to(dev) for r in range(rounds)]
-        acc_total = sum(int(a.sum()) for a in accs)
-        y = torch.empty(wl.batch, T, wl.nheads, wl.headdim, device=dev)
+    dev, bf, stream = torch.device("cuda"), torch.bfloat16, torch.cuda.current_stream()
+    hbm = load_peaks()[0]
+    out = {"workload": "mamba2 speculative verify + commit, batch 512, 128 heads, P 64, N 128, 8 groups, L 16",
+           "gdn": {"workload": "gdn speculative verify + commit, batch 256, 32 heads, d_k = d_v = 128, L 16"}}
+    for kind, wl in (("mamba2", SPEC_MAMBA2_B512), ("gdn", GDN_B256)):
+        if kind == "mamba2":
+            p = mamba2_params(wl)
+            A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
+            S0 = torch.from_numpy(mamba2_initial_state(wl)).to(dev)
+            rows, cols, G, f32_keys = wl.headdim, wl.dstate, wl.ngroups, ()
+            draft_inputs = mamba2_draft_inputs
+        else:
+            A = D = None
+            S0 = torch.from_numpy(gdn_initial_state(wl)).to(dev)
+            rows, cols, G, f32_keys = wl.dv, wl.dk, 1, ("alpha", "beta")
+            draft_inputs = gdn_draft_inputs
+        dst = out if kind == "mamba2" else out["gdn"]
+        for T in (4, 8):
+            layer = ReplaySSM(kind, wl.batch, wl.nheads, rows, cols, G, wl.window, T, bf, A=A, D=D)
+            layer.load_checkpoint(S0)
+            drafts = [{k: torch.from_numpy(v).to(dev).to(torch.float32 if k in f32_keys else bf)
+                       for k, v in draft_inputs(wl, r, T).items()} for r in range(4)]
+            acc_np = [accepted_lengths(wl, r, T) for r in range(rounds)]
+            accs = [torch.from_numpy(a).to(dev) for a in acc_np]
+            acc_total = sum(int(a.sum()) for a in accs)
+            y = torch.empty(wl.batch, T, wl.nheads, rows, device=dev)
 
-        def rnd(i):
-            d = drafts[i % 4]
-            layer.verify(T, y=y, x=d["x"], B=d["B"], C=d["C"], dt=d["dt"])
-            layer.commit(accs[i])
+            def rnd(i):
+                layer.verify(T, y=y, **drafts[i % 4])
+                layer.commit(accs[i])
 
-        for i in range(min(8, rounds)):
-            rnd(i)
-        layer.load_checkpoint(S0)
-        ms = timed(rnd, rounds, stream)
-        err = layer.get_error()
-        del layer
-        # snapshot-per-draft comparison: one state read, T state writes per round
-        cfg = make_config("mamba2", wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window, T, bf, A=A, D=D)
-        snaps = torch.empty(wl.batch, T + 1, wl.nheads, wl.headdim, wl.dstate, device=dev)
-        snaps[:, 0].copy_(S0)
-        cur = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+            for i in range(min(8, rounds)):
+                rnd(i)
+            layer.load_checkpoint(S0)
+            ms = timed(rnd, rounds, stream)
+            err = layer.get_error()
+            del layer
+            # snapshot-per-draft comparison: one state read, T state writes per round
+            cfg = make_config(kind, wl.batch, wl.nheads, rows, cols, G, wl.window, T, bf, A=A, D=D)
+            snaps = torch.empty(wl.batch, T + 1, wl.nheads, rows, cols, device=dev)
+            snaps[:, 0].copy_(S0)
+            cur = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
 
-        def snap(i):
-            d = drafts[i % 4]
-            snap_verify(cfg, snaps, cur, T, y, x=d["x"], B=d["B"], C=d["C"], dt=d["dt"])
-            snap_commit(cfg, cur, accs[i])
+            def snap(i):
+                snap_verify(cfg, snaps, cur, T, y, **drafts[i % 4])
+                snap_commit(cfg, cur, accs[i])
 
-        for i in range(min(4, rounds)):
-            snap(i)
-        ms_snap = timed(snap, rounds, stream)
-        del snaps
-        out[f"T{T}"] = {"ms_per_round": ms, "verified_tokens_per_s": wl.batch * T / (ms * 1e-3),
-                        "committed_tokens_per_s": acc_total / rounds / (ms * 1e-3),
-                        "snapshot_ms_per_round": ms_snap,
-                        "snapshot_committed_tokens_per_s": acc_total / rounds / (ms_snap * 1e-3),
-                        "speedup_vs_snapshot": ms_snap / ms, "rounds": rounds, "device_error": err}
+            for i in range(min(4, rounds)):
+                snap(i)
+            ms_snap = timed(snap, rounds, stream)
+            del snaps
+            gbps = verify_traffic(wl, T, acc_np) / rounds / (ms * 1e-3) / 1e9
+            dst[f"T{T}"] = {"ms_per_round": ms, "verified_tokens_per_s": wl.batch * T / (ms * 1e-3),
+                            "GBps": gbps, "frac_of_measured_hbm": gbps / hbm,
+                            "committed_tokens_per_s": acc_total / rounds / (ms * 1e-3),
+                            "snapshot_ms_per_round": ms_snap,
+                            "snapshot_committed_tokens_per_s": acc_total / rounds / (ms_snap * 1e-3),
+                            "speedup_vs_snapshot": ms_snap / ms, "rounds": rounds, "device_error": err}
     return out
 
 
@@ -587,7 +629,7 @@ def main():
     res = run_gpu(args, rank, world)
     if rank == 0 and world == 1 and not args.no_extra:
         res["gdn"] = gdn_section(min(args.steps, 1024))
-        res["verify"] = verify_section(64)
+        res["verify"] = verify_section(512)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -18,6 +18,7 @@ struct rssm_ctx {
   int num_sms;
   int smem_optin;
   int nstage_override;
+  int loaded;    // set by the first successful rssm_load_checkpoint
 };
 
 namespace {
@@ -64,6 +65,7 @@ int *err_word(rssm_ctx *x) { return reinterpret_cast<int *>(x->arena + x->lay.er
 
 rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, const void *C, const void *dt,
                    const unsigned char *mask, float *y, cudaStream_t stream) {
+  if (!x->loaded) return RSSM_ERR_UNSUPPORTED;
   const rssm_config &c = x->cfg;
   M2Args a{};
   a.Bt = c.batch; a.H = c.nheads; a.P = c.headdim; a.G = c.ngroups; a.L = c.window;
@@ -86,6 +88,7 @@ rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, c
 
 rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, const void *v, const float *alpha,
                     const float *beta, const unsigned char *mask, float *y, cudaStream_t stream) {
+  if (!x->loaded) return RSSM_ERR_UNSUPPORTED;
   const rssm_config &c = x->cfg;
   GArgs a{};
   a.Bt = c.batch; a.H = c.nheads; a.DV = c.headdim; a.L = c.window;
@@ -183,6 +186,7 @@ rssm_status rssm_load_checkpoint(rssm_ctx *x, const float *S, rssm_stream stream
   if (e == cudaSuccess) e = launch_meta_reset(reinterpret_cast<int4 *>(x->arena + x->lay.meta), c.batch, err_word(x), st);
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity = 0;
+  x->loaded = 1;
   return RSSM_OK;
 }
 
@@ -219,6 +223,7 @@ rssm_status rssm_verify(rssm_ctx *x, int T, const rssm_tokens *tok, float *y, rs
 
 rssm_status rssm_commit(rssm_ctx *x, const int *accepted, rssm_stream stream) {
   if (!x || !accepted) return RSSM_ERR_ARG;
+  if (!x->loaded) return RSSM_ERR_UNSUPPORTED;
   cudaError_t e = launch_commit(meta_cur(x), meta_next(x), accepted, x->cfg.batch, err_word(x),
                                 reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
@@ -235,6 +240,7 @@ rssm_status rssm_flush(rssm_ctx *x, const unsigned char *mask, rssm_stream strea
 
 rssm_status rssm_export(rssm_ctx *x, float *S_out, void *ring_out, int *meta_out, rssm_stream stream) {
   if (!x) return RSSM_ERR_ARG;
+  if (!x->loaded) return RSSM_ERR_UNSUPPORTED;
   const rssm_config &c = x->cfg;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t units = (size_t)c.batch * c.nheads;
@@ -283,7 +289,7 @@ rssm_status rssm_export_read_copy(rssm_ctx *x, unsigned char *codes, unsigned ch
                                   rssm_stream stream) {
   if (!x) return RSSM_ERR_ARG;
   const rssm_config &c = x->cfg;
-  if (c.read == RSSM_READ_SAME) return RSSM_ERR_UNSUPPORTED;
+  if (c.read == RSSM_READ_SAME || !x->loaded) return RSSM_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t elems = (size_t)c.batch * c.nheads * c.headdim * kCols;
   cudaError_t e = cudaSuccess;
@@ -298,6 +304,7 @@ rssm_status rssm_export_read_copy(rssm_ctx *x, unsigned char *codes, unsigned ch
 
 rssm_status rssm_get_error(rssm_ctx *x, int *code, int *seq, rssm_stream stream) {
   if (!x || !code || !seq) return RSSM_ERR_ARG;
+  if (!x->loaded) return RSSM_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int w = kErrClean;
   cudaError_t e = cudaStreamSynchronize(st);

@@ -38,7 +38,7 @@ __host__ __device__ inline int dt_stride(int L) { return (int)align_up((size_t)(
 // Byte offsets of the regions of a context's arena.
 struct ArenaLayout {
   size_t meta;     // int4 [2][Bt]: count, epoch, pending, 0  (ping-pong by call parity)
-  size_t err;      // int [1]
+  size_t err;      // int [4]: sticky error word, next unit to hand out, blocks finished, 0
   size_t hp;       // checkpoint: fp32 or fp16 [Bt][H][R][128]
   size_t rq;       // NVFP4 codes u8 [Bt][H][R][64]
   size_t rs;       // NVFP4 block scales u8 [Bt][H][R][8]
@@ -235,10 +235,44 @@ __device__ __forceinline__ void warp_transpose_reduce(float (&v)[V], int lane) {
   }
 }
 
+// ---- dynamic unit scheduling.  A launch hands its work units to its persistent blocks through a
+// counter next to the error word (one atomic per unit), so that blocks whose units cost more (a fold
+// reads and writes the state) do not hold up a launch whose other blocks drew cheaper ones.  The last
+// block to finish re-arms the counters for the next launch on the stream.
+__device__ __forceinline__ int sched_grab(int *err) { return atomicAdd(err + 1, 1); }
+__device__ __forceinline__ void sched_finish(int *err) {  // one thread per block, after the block's last grab
+  if (atomicAdd(err + 2, 1) == (int)gridDim.x - 1) {
+    atomicExch(err + 1, 0);
+    atomicExch(err + 2, 0);
+  }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return v;
+}
+
+// ---- register-operand tensor-core tile (warp-wide): d[16x8] += a[16x16] b[16x8], bf16 in, fp32 accumulate.
+// Lane 4g+t holds a = {A[g][2t..2t+1], A[g+8][2t..2t+1], A[g][2t+8..2t+9], A[g+8][2t+8..2t+9]},
+// b = {B[2t..2t+1][g], B[2t+8..2t+9][g]}, d = {D[g][2t..2t+1], D[g+8][2t..2t+1]}; the lower-indexed
+// element of a pair sits in the low half of its register.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// fp32 pair -> bf16 pairs hi + lo with hi = RN(v) and lo = RN(v - hi): |v - hi - lo| <= 2^-17 |v|, so two
+// bf16 products against an exact bf16 operand carry a fp32 operand to ~16 significant bits.
+__device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const uint32_t hb = *reinterpret_cast<const uint32_t *>(&h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x - __uint_as_float(hb << 16), y - __uint_as_float(hb & 0xffff0000u));
+  hi = hb;
+  lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
 }  // namespace rssm

@@ -47,7 +47,7 @@ namespace {
 constexpr int kGHdrBytes = 1024;
 enum {
   Q_ACTIVE = 0, Q_NREC, Q_M, Q_NRING, Q_NNEW, Q_TOUT, Q_SLOT0, Q_MC, Q_ME, Q_MP, Q_B, Q_H0, Q_NH, Q_BASE,
-  Q_WMETA,
+  Q_WMETA, Q_END,
   Q_F = 32,                // floats: alpha of new tokens [8][8] (token, head)
   Q_FB = Q_F + 64          // beta of new tokens [8][8]
 };
@@ -125,8 +125,6 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunks = (a.H + HG - 1) / HG;
   const int units = a.Bt * chunks;
-  const int u_begin = (int)(((long long)blockIdx.x * units) / gridDim.x);
-  const int u_end = (int)(((long long)(blockIdx.x + 1) * units) / gridDim.x);
   const bool fp4_read = a.read_mode != RSSM_READ_SAME;
   const bool shared_fp4 = a.read_mode == RSSM_READ_SHARED_NVFP4;
   const bool hp16 = a.hp_mode == RSSM_HP_F16_SR;
@@ -157,27 +155,26 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     const uint64_t pol_stream = policy_evict_first();
     const uint64_t pol_keep = policy_evict_last();
     const uint32_t krow = (uint32_t)kCols * esz, vrow = (uint32_t)R * esz;
-    const int b_first = u_begin / chunks;
-    int mw_base = -1, mk = 1;
-    int4 mw = make_int4(0, 0, 0, 0);
     struct Sched {
       int b, h0, nh, active, n_ring, n_new, m, t_out, slot0, base_e;
     };
+    // schedule of unit u from the sequence's bookkeeping word; u >= units writes the end marker
     auto schedule = [&](int u, Sched &S, int *hdr) {
+      if (u >= units) {
+        S = Sched{};
+        if (lane == 0) { hdr[Q_ACTIVE] = 0; hdr[Q_END] = 1; }
+        return;
+      }
       const int b = u / chunks, ch = u % chunks;
       S.b = b; S.h0 = ch * HG; S.nh = min(HG, a.H - S.h0);
-      const int base32 = b_first + ((b - b_first) & ~31);
-      if (base32 != mw_base) {
-        const int bq = base32 + lane;
-        if (bq < a.Bt) {
-          mw = a.meta_in[bq];
-          mk = (a.mask == nullptr) ? 1 : (int)a.mask[bq];
-        }
-        mw_base = base32;
+      int4 mw = make_int4(0, 0, 0, 0);
+      int mk = 1;
+      if (lane == 0) {
+        mw = a.meta_in[b];
+        mk = (a.mask == nullptr) ? 1 : (int)a.mask[b];
       }
-      const int src = b - base32;
-      const int c = __shfl_sync(0xffffffffu, mw.x, src), e = __shfl_sync(0xffffffffu, mw.y, src);
-      const int pend = __shfl_sync(0xffffffffu, mw.z, src), msk = __shfl_sync(0xffffffffu, mk, src);
+      const int c = __shfl_sync(0xffffffffu, mw.x, 0), e = __shfl_sync(0xffffffffu, mw.y, 0);
+      const int pend = __shfl_sync(0xffffffffu, mw.z, 0), msk = __shfl_sync(0xffffffffu, mk, 0);
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
       int mc = c, me = e, mp = pend;
       const int base_e = (e & 1) * L, base_n = ((e + 1) & 1) * L;
@@ -204,19 +201,18 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       S.active = active; S.n_ring = n_ring; S.n_new = n_new; S.m = m; S.t_out = t_out; S.slot0 = slot0;
       S.base_e = base_e;
-      if (hdr != nullptr && lane == 0) {
+      if (lane == 0) {
         hdr[Q_ACTIVE] = active; hdr[Q_NREC] = n_ring + n_new; hdr[Q_M] = m; hdr[Q_NRING] = n_ring;
         hdr[Q_NNEW] = n_new; hdr[Q_TOUT] = t_out; hdr[Q_SLOT0] = slot0; hdr[Q_MC] = mc; hdr[Q_ME] = me;
         hdr[Q_MP] = mp; hdr[Q_B] = b; hdr[Q_H0] = S.h0; hdr[Q_NH] = S.nh; hdr[Q_BASE] = base_e;
-        hdr[Q_WMETA] = (S.h0 == 0);
+        hdr[Q_WMETA] = (S.h0 == 0); hdr[Q_END] = 0;
       }
     };
     // group data of unit u: k records and q of every head, alpha / beta ring rows
-    auto issue_group = [&](int u, int gi) -> bool {
+    auto issue_group = [&](int u, int gi, Sched &S) -> bool {
       const int gs = gi % kGBG;
       if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGBG) & 1) ^ 1), abort_flag)) return false;
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
-      Sched S;
       schedule(u, S, reinterpret_cast<int *>(gb));
       __syncwarp();
       const int n_rec = S.n_ring + S.n_new, nh = S.nh;
@@ -258,65 +254,77 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       return true;
     };
-    bool ok = true;
-    if (u_begin < u_end) ok = issue_group(u_begin, 0);
+    // units come from the launch's counter: the group data of the next unit is issued before
+    // the current unit's tiles, and the unit after that is requested (atomic in flight) meanwhile
+    int u_cur = 0, u_nxt = 0;
+    if (lane == 0) u_cur = sched_grab(a.err);
+    u_cur = __shfl_sync(0xffffffffu, u_cur, 0);
+    if (lane == 0 && u_cur < units) u_nxt = sched_grab(a.err);
+    u_nxt = u_cur < units ? __shfl_sync(0xffffffffu, u_nxt, 0) : units;
+    Sched Sc, Sn;
+    bool ok = issue_group(u_cur, 0, Sc);
     int ti = 0;
-    for (int u = u_begin, gi = 0; ok && u < u_end; ++u, ++gi) {
-      if (u + 1 < u_end && !issue_group(u + 1, gi + 1)) {
+    for (int gi = 0; ok && u_cur < units; ++gi) {
+      if (!issue_group(u_nxt, gi + 1, Sn)) {
         ok = false;
         break;
       }
-      Sched S;
-      schedule(u, S, nullptr);
-      if (!S.active) continue;
-      const int n_rec = S.n_ring + S.n_new;
-      const bool fold = S.m > 0;
-      const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
-                              : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
-      for (int tt = 0; tt < S.nh * nrb; ++tt, ++ti) {
-        const int i = tt / nrb, t = tt % nrb;
-        const int rows = min(kFp4Rows, R - kFp4Rows * t);
-        const size_t unit = (size_t)S.b * a.H + S.h0 + i;
-        const size_t row_abs = unit * R + (size_t)kFp4Rows * t;  // first state row of the tile
-        const int s = ti % NS;
-        if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
-          ok = false;
-          break;
-        }
-        unsigned char *st = stages + (size_t)s * lay.stage_bytes;
-        uint32_t tb = (uint32_t)n_rec * vrow;
-        if (srcfmt == SRC_F32) tb += rows * kCols * 4;
-        else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
-        else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
-        if (lane == 0) {
-          armed[s] = ti / NS;
-          mbar_arrive_expect_tx(&full[s], tb);
-        }
-        __syncwarp();
-        if (lane == 0) {
-          if (srcfmt == SRC_F32)
-            bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
-          else if (srcfmt == SRC_F16)
-            bulk_g2s(st, reinterpret_cast<const __half *>(a.hp) + row_abs * kCols, rows * kCols * 2, &full[s], pol_stream);
-          else
-            bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
-        }
-        if (lane == 1 && srcfmt == SRC_FP4)
-          bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
-        if (lane == 2 && srcfmt == SRC_FP4) {
-          const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
-          bulk_g2s(st + lay.st_g, a.rg + gi4, 16, &full[s], pol_keep);
-        }
-        if (lane == 3 && S.n_ring)
-          bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + S.base_e) * vrow,
-                   S.n_ring * vrow, &full[s], pol_keep);
-        if (lane >= 4 && lane < 4 + S.n_new) {
-          const int tk = lane - 4;
-          bulk_g2s(st + lay.st_v + (S.n_ring + tk) * vrow,
-                   reinterpret_cast<const unsigned char *>(a.v) + (((size_t)S.b * a.T + tk) * a.H + S.h0 + i) * vrow,
-                   vrow, &full[s], pol_keep);
+      int u_after = units;  // read back (and so completed) at the end of the iteration on every path
+      if (lane == 0 && u_nxt < units) u_after = sched_grab(a.err);
+      const Sched S = Sc;
+      if (S.active) {
+        const int n_rec = S.n_ring + S.n_new;
+        const bool fold = S.m > 0;
+        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
+                                : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
+        for (int tt = 0; tt < S.nh * nrb; ++tt, ++ti) {
+          const int i = tt / nrb, t = tt % nrb;
+          const int rows = min(kFp4Rows, R - kFp4Rows * t);
+          const size_t unit = (size_t)S.b * a.H + S.h0 + i;
+          const size_t row_abs = unit * R + (size_t)kFp4Rows * t;  // first state row of the tile
+          const int s = ti % NS;
+          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          uint32_t tb = (uint32_t)n_rec * vrow;
+          if (srcfmt == SRC_F32) tb += rows * kCols * 4;
+          else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
+          else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
+          if (lane == 0) {
+            armed[s] = ti / NS;
+            mbar_arrive_expect_tx(&full[s], tb);
+          }
+          __syncwarp();
+          if (lane == 0) {
+            if (srcfmt == SRC_F32)
+              bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
+            else if (srcfmt == SRC_F16)
+              bulk_g2s(st, reinterpret_cast<const __half *>(a.hp) + row_abs * kCols, rows * kCols * 2, &full[s], pol_stream);
+            else
+              bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
+          }
+          if (lane == 1 && srcfmt == SRC_FP4)
+            bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
+          if (lane == 2 && srcfmt == SRC_FP4) {
+            const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
+            bulk_g2s(st + lay.st_g, a.rg + gi4, 16, &full[s], pol_keep);
+          }
+          if (lane == 3 && S.n_ring)
+            bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + S.base_e) * vrow,
+                     S.n_ring * vrow, &full[s], pol_keep);
+          if (lane >= 4 && lane < 4 + S.n_new) {
+            const int tk = lane - 4;
+            bulk_g2s(st + lay.st_v + (S.n_ring + tk) * vrow,
+                     reinterpret_cast<const unsigned char *>(a.v) + (((size_t)S.b * a.T + tk) * a.H + S.h0 + i) * vrow,
+                     vrow, &full[s], pol_keep);
+          }
         }
       }
+      Sc = Sn;
+      u_cur = u_nxt;
+      u_nxt = __shfl_sync(0xffffffffu, u_after, 0);
     }
     if (!ok && lane == 0) {
       record_error(a.err, 0, RSSM_DEV_TIMEOUT);
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       ++rdv;
       return ok;
     };
-    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+    for (int gi = 0;; ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
       if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGBG) & 1), abort_flag) ||
           !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
@@ -344,6 +352,11 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
+      if (gh[Q_END]) {  // no more units: let the consumers see the marker
+        __syncwarp();
+        if (pw == 0 && lane == 0) mbar_arrive(&tfull[tsl]);
+        break;
+      }
       float *gf = reinterpret_cast<float *>(gb);
       const int b = gh[Q_B], h0 = gh[Q_H0], nh = gh[Q_NH];
       if (pw == 0 && gh[Q_WMETA] && lane == 0) a.meta_out[b] = make_int4(gh[Q_MC], gh[Q_ME], gh[Q_MP], 0);
@@ -361,31 +374,6 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           const size_t unit = (size_t)b * a.H + h0 + i;
           a.ring_a[unit * dts + slot0 + t] = al;
           a.ring_b[unit * dts + slot0 + t] = be;
-        }
-        {  // v rows of the new tokens, straight from the inputs: eight 16-byte loads in flight per lane
-          const int vq = R * esz / 16, nq = n_new * nh * vq;
-          for (int q0 = 0; q0 < nq; q0 += 512) {
-            uint4 v[8];
-#pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
-              const int q = q0 + k2 * 64 + pw * 32 + lane;
-              if (q < nq) {
-                const int c16 = q % vq, ti2 = q / vq, t = ti2 / nh, i = ti2 % nh;
-                v[k2] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.v) +
-                                                         (((size_t)b * a.T + t) * a.H + h0 + i) * R * esz + c16 * 16);
-              }
-            }
-#pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
-              const int q = q0 + k2 * 64 + pw * 32 + lane;
-              if (q < nq) {
-                const int c16 = q % vq, ti2 = q / vq, t = ti2 / nh, i = ti2 % nh;
-                const size_t unit = (size_t)b * a.H + h0 + i;
-                *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_v) +
-                                           ((unit * 2 * L + slot0 + t) * R) * esz + c16 * 16) = v[k2];
-              }
-            }
-          }
         }
         const int kq = kCols * esz / 16;
         for (int q = pw * 32 + lane; q < n_new * nh * kq; q += 64) {
@@ -460,8 +448,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     // All eight take every tile; warp w owns rows 8w..8w+7 of the 64-row tile.
     const int row0 = warp * 8;
     const uint64_t pol_wr = policy_evict_first();
+    const uint64_t pol_ring = policy_evict_last();
     int ti = 0, rdv = 0;
-    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+    for (int gi = 0;; ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
       if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
@@ -469,10 +458,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
+      if (gh[Q_END]) break;
       const int b = gh[Q_B], h0 = gh[Q_H0], nh = gh[Q_NH];
       if (gh[Q_ACTIVE]) {
         const int n_rec = gh[Q_NREC], m = gh[Q_M], t_out = gh[Q_TOUT];
         const int me = gh[Q_ME];
+        const int n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], slot0 = gh[Q_SLOT0];
         const bool fold = m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
                                 : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
@@ -492,6 +483,15 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           }
           const unsigned char *st = stages + (size_t)s * lay.stage_bytes;
           const TI *vr = reinterpret_cast<const TI *>(st + lay.st_v);
+          // the new tokens' v rows, landed behind the buffered ones in the head's first tile
+          // stage, go to the head's ring row with one bulk store (warps take turns); every warp
+          // waits for its bulk stores to have read the stage before releasing it
+          if (t == 0 && n_new > 0 && (ti & (kConsumerWarps - 1)) == warp && lane == 0) {
+            const uint32_t vrow = (uint32_t)R * esz;
+            bulk_s2g(reinterpret_cast<unsigned char *>(a.ring_v) + (unit * 2 * a.L + slot0) * vrow,
+                     st + lay.st_v + (size_t)n_ring * vrow, (uint32_t)n_new * vrow, pol_ring);
+            bulk_commit();
+          }
           const float g_tile = reinterpret_cast<const float *>(st + lay.st_g)[(unit * nrb + t) & 3];
           const float *co_h = cot + (size_t)i * lay.no * lay.rmax;
           const float *u0_h = u0t + (size_t)i * lay.no * kCols;
@@ -733,6 +733,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     for (int s = 0; s < kGBG; ++s)
       if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
   }
+  if (threadIdx.x == 0) sched_finish(a.err);
 }
 
 }  // namespace

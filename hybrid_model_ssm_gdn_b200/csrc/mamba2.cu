@@ -42,7 +42,7 @@ constexpr int kGHdr = 1024;      // group header bytes
 // group header: ints then floats
 enum {
   G_ACTIVE = 0, G_NREC, G_M, G_NRING, G_NNEW, G_TOUT, G_SLOT0, G_MC, G_ME, G_MP, G_B, G_G, G_H0, G_NH,
-  G_BASE, G_WMETA, G_WB,
+  G_BASE, G_WMETA, G_WB, G_END,
   G_A = 32,                  // floats: A[16]
   G_D = G_A + kHG,           // D[16]
   G_DT = G_D + kHG           // dt of new tokens [8][16]
@@ -50,6 +50,8 @@ enum {
 
 struct M2Layout {
   int rmax, no;
+  bool mma;                  // output contraction on tensor cores (bf16 inputs, 8 outputs per row)
+  int nq;                    // 16-record steps of the buffered term on that path
   int tile_bytes;            // P*128*4
   int xr;                    // offset of the x records in a tile stage
   int stage_bytes;
@@ -61,7 +63,9 @@ struct M2Layout {
 __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
   M2Layout l;
   l.no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
+  l.mma = l.no == 8 && esz == 2;
   l.rmax = L + (tmax > 1 ? tmax : 1);
+  l.nq = (l.rmax + 15) / 16;
   l.tile_bytes = P * kCols * 4;
   l.xr = l.tile_bytes;
   l.stage_bytes = (int)align_up((size_t)l.xr + (size_t)l.rmax * P * esz, 128);
@@ -69,8 +73,10 @@ __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
   l.gb_C = (int)align_up((size_t)l.gb_B + (size_t)l.rmax * kCols * esz, 16);
   l.gb_dt = (int)align_up((size_t)l.gb_C + (size_t)l.no * kCols * esz, 16);
   l.gb_bytes = (int)align_up((size_t)l.gb_dt + (size_t)kHG * dt_stride(L) * 4, 128);
-  // tables: g[no][rmax], coef[kHG][no][rmax], ao[kHG][no], wf[kHG][rmax], af[kHG], flags[8]
-  const int floats = l.no * l.rmax + kHG * l.no * l.rmax + kHG * l.no + kHG * l.rmax + kHG + 8;
+  // tables: g[no][rmax], coef[kHG][no][rmax] (or, on the tensor-core path, its fragments
+  // [kHG][nq][32 lanes][4 words]), ao[kHG][no], wf[kHG][rmax], af[kHG], flags[8]
+  const int coef_floats = l.mma ? kHG * l.nq * 32 * 4 : kHG * l.no * l.rmax;
+  const int floats = l.no * l.rmax + coef_floats + kHG * l.no + kHG * l.rmax + kHG + 8;
   l.tab_bytes = (int)align_up((size_t)floats * 4, 128);
   l.cx_bytes = (int)align_up((size_t)kConsumerWarps * l.rmax * 8 * 4, 128);
   return l;
@@ -85,6 +91,9 @@ constexpr int kProducerWarp = kConsumerWarps, kPrepWarp = kConsumerWarps + 1;
 template <typename TI, int NO>
 __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // S'.C_j on tensor cores for 5..8 drafts (measured: at 4 the CUDA-core reduction is as fast): C_j is
+  // exact in bf16 and S' enters as a hi + lo bf16 pair
+  constexpr bool kMma = NO == 8 && sizeof(TI) == 2;
   const int esz = sizeof(TI);
   const M2Layout lay = m2_layout(a.P, a.L, a.tmax, esz);
   const int NS = a.nstage;
@@ -108,7 +117,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     Tables t;
     t.g = reinterpret_cast<float *>(tabs + (size_t)which * lay.tab_bytes);  // [NO][rmax]   B_r . C_j
     t.coef = t.g + NO * rmax;                                                // [kHG][NO][rmax]
-    t.ao = t.coef + kHG * NO * rmax;                                         // [kHG][NO]
+    t.ao = t.coef + (kMma ? kHG * lay.nq * 32 * 4 : kHG * NO * rmax);       // [kHG][NO]
     t.wf = t.ao + kHG * NO;                                                  // [kHG][rmax]
     t.af = t.wf + kHG * rmax;                                                // [kHG]
     return t;
@@ -118,8 +127,6 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   const int hpg = a.H / a.G;
   const int chunks = (hpg + kHG - 1) / kHG;
   const int units = a.Bt * a.G * chunks;
-  const int u_begin = (int)(((long long)blockIdx.x * units) / gridDim.x);
-  const int u_end = (int)(((long long)(blockIdx.x + 1) * units) / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s) {
@@ -146,32 +153,27 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     const uint64_t pol_keep = policy_evict_last();
     const uint32_t xrow = (uint32_t)a.P * esz, brow = (uint32_t)kCols * esz;
     const int L = a.L, dts = dt_stride(L);
-    // bookkeeping words: lane q holds sequence (first + q) of the block's range, loaded up front
-    // (and refreshed every 32 sequences) so the issue loop never waits on a global load
-    const int b_first = u_begin / (a.G * chunks);
-    int mw_base = -1;
-    int4 mw = make_int4(0, 0, 0, 0);
-    int mk = 1;
     struct Sched {
       int b, g, h0, nh, active, n_ring, n_new, m, t_out, slot0, base_e;
     };
-    // schedule of unit u (identical for every head of the sequence); loads nothing but the
-    // prefetched bookkeeping words
+    // schedule of unit u (identical for every head of the sequence) from the sequence's
+    // bookkeeping word; u >= units writes the end marker
     auto schedule = [&](int u, Sched &S, int *hdr) {
+      if (u >= units) {
+        S = Sched{};
+        if (lane == 0) { hdr[G_ACTIVE] = 0; hdr[G_END] = 1; }
+        return;
+      }
       const int b = u / (a.G * chunks), g = (u / chunks) % a.G, ch = u % chunks;
       S.b = b; S.g = g; S.h0 = g * hpg + ch * kHG; S.nh = min(kHG, hpg - ch * kHG);
-      const int base32 = b_first + ((b - b_first) & ~31);
-      if (base32 != mw_base) {
-        const int bq = base32 + lane;
-        if (bq < a.Bt) {
-          mw = a.meta_in[bq];
-          mk = (a.mask == nullptr) ? 1 : (int)a.mask[bq];
-        }
-        mw_base = base32;
+      int4 mw = make_int4(0, 0, 0, 0);
+      int mk = 1;
+      if (lane == 0) {
+        mw = a.meta_in[b];
+        mk = (a.mask == nullptr) ? 1 : (int)a.mask[b];
       }
-      const int src = b - base32;
-      const int c = __shfl_sync(0xffffffffu, mw.x, src), e = __shfl_sync(0xffffffffu, mw.y, src);
-      const int pend = __shfl_sync(0xffffffffu, mw.z, src), msk = __shfl_sync(0xffffffffu, mk, src);
+      const int c = __shfl_sync(0xffffffffu, mw.x, 0), e = __shfl_sync(0xffffffffu, mw.y, 0);
+      const int pend = __shfl_sync(0xffffffffu, mw.z, 0), msk = __shfl_sync(0xffffffffu, mk, 0);
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
       int mc = c, me = e, mp = pend;
       const int base_e = (e & 1) * L, base_n = ((e + 1) & 1) * L;
@@ -198,19 +200,18 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       S.active = active; S.n_ring = n_ring; S.n_new = n_new; S.m = m; S.t_out = t_out; S.slot0 = slot0;
       S.base_e = base_e;
-      if (hdr != nullptr && lane == 0) {
+      if (lane == 0) {
         hdr[G_ACTIVE] = active; hdr[G_NREC] = n_ring + n_new; hdr[G_M] = m; hdr[G_NRING] = n_ring;
         hdr[G_NNEW] = n_new; hdr[G_TOUT] = t_out; hdr[G_SLOT0] = slot0; hdr[G_MC] = mc; hdr[G_ME] = me;
         hdr[G_MP] = mp; hdr[G_B] = b; hdr[G_G] = g; hdr[G_H0] = S.h0; hdr[G_NH] = S.nh; hdr[G_BASE] = base_e;
-        hdr[G_WMETA] = (S.h0 == 0); hdr[G_WB] = (ch == 0);
+        hdr[G_WMETA] = (S.h0 == 0); hdr[G_WB] = (ch == 0); hdr[G_END] = 0;
       }
     };
-    // group data of unit u into buffer u % kGB (B records, B and C of the new tokens, dt rows)
-    auto issue_group = [&](int u, int gi) -> bool {
+    // group data of unit u into buffer gi % kGB (B records, B and C of the new tokens, dt rows)
+    auto issue_group = [&](int u, int gi, Sched &S) -> bool {
       const int gs = gi % kGB;
       if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGB) & 1) ^ 1), abort_flag)) return false;
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
-      Sched S;
       schedule(u, S, reinterpret_cast<int *>(gb));
       __syncwarp();
       const int n_rec = S.n_ring + S.n_new;
@@ -242,43 +243,55 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       return true;
     };
-    bool ok = true;
-    if (u_begin < u_end) ok = issue_group(u_begin, 0);
+    // units come from the launch's counter: the group data of the next unit is issued before
+    // the current unit's tiles, and the unit after that is requested (atomic in flight) meanwhile
+    int u_cur = 0, u_nxt = 0;
+    if (lane == 0) u_cur = sched_grab(a.err);
+    u_cur = __shfl_sync(0xffffffffu, u_cur, 0);
+    if (lane == 0 && u_cur < units) u_nxt = sched_grab(a.err);
+    u_nxt = u_cur < units ? __shfl_sync(0xffffffffu, u_nxt, 0) : units;
+    Sched Sc, Sn;
+    bool ok = issue_group(u_cur, 0, Sc);
     int ti = 0;
-    for (int u = u_begin, gi = 0; ok && u < u_end; ++u, ++gi) {
-      if (u + 1 < u_end && !issue_group(u + 1, gi + 1)) {
+    for (int gi = 0; ok && u_cur < units; ++gi) {
+      if (!issue_group(u_nxt, gi + 1, Sn)) {
         ok = false;
         break;
       }
-      Sched S;
-      schedule(u, S, nullptr);
-      if (!S.active) continue;
-      const int n_rec = S.n_ring + S.n_new;
-      const uint32_t tbytes = (uint32_t)lay.tile_bytes + n_rec * xrow;
-      for (int i = 0; i < S.nh; ++i, ++ti) {
-        const int s = ti % NS;
-        if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
-          ok = false;
-          break;
-        }
-        unsigned char *st = stages + (size_t)s * lay.stage_bytes;
-        const size_t unit = (size_t)S.b * a.H + S.h0 + i;
-        if (lane == 0) {
-          armed[s] = ti / NS;
-          mbar_arrive_expect_tx(&full[s], tbytes);
-        }
-        __syncwarp();
-        if (lane == 0) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
-        if (lane == 1 && S.n_ring)
-          bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + S.base_e) * xrow,
-                   S.n_ring * xrow, &full[s], pol_keep);
-        if (lane >= 4 && lane < 4 + S.n_new) {
-          const int t = lane - 4;
-          bulk_g2s(st + lay.xr + (S.n_ring + t) * xrow,
-                   reinterpret_cast<const unsigned char *>(a.x) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * xrow, xrow,
-                   &full[s], pol_keep);
+      int u_after = units;  // read back (and so completed) at the end of the iteration on every path
+      if (lane == 0 && u_nxt < units) u_after = sched_grab(a.err);
+      const Sched S = Sc;
+      if (S.active) {
+        const int n_rec = S.n_ring + S.n_new;
+        const uint32_t tbytes = (uint32_t)lay.tile_bytes + n_rec * xrow;
+        for (int i = 0; i < S.nh; ++i, ++ti) {
+          const int s = ti % NS;
+          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          const size_t unit = (size_t)S.b * a.H + S.h0 + i;
+          if (lane == 0) {
+            armed[s] = ti / NS;
+            mbar_arrive_expect_tx(&full[s], tbytes);
+          }
+          __syncwarp();
+          if (lane == 0) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
+          if (lane == 1 && S.n_ring)
+            bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + S.base_e) * xrow,
+                     S.n_ring * xrow, &full[s], pol_keep);
+          if (lane >= 4 && lane < 4 + S.n_new) {
+            const int t = lane - 4;
+            bulk_g2s(st + lay.xr + (S.n_ring + t) * xrow,
+                     reinterpret_cast<const unsigned char *>(a.x) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * xrow, xrow,
+                     &full[s], pol_keep);
+          }
         }
       }
+      Sc = Sn;
+      u_cur = u_nxt;
+      u_nxt = __shfl_sync(0xffffffffu, u_after, 0);
     }
     if (!ok && lane == 0) {
       record_error(a.err, 0, RSSM_DEV_TIMEOUT);
@@ -286,7 +299,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     }
   } else if (warp == kPrepWarp) {
     // ================================================================== prep warp
-    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+    for (int gi = 0;; ++gi) {
       const int gs = gi % kGB, tsl = gi & 1;
       if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGB) & 1), abort_flag) ||
           !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
@@ -295,6 +308,11 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
+      if (gh[G_END]) {  // no more units: let the consumers see the marker
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tfull[tsl]);
+        break;
+      }
       const float *gf = reinterpret_cast<const float *>(gb);
       const int b = gh[G_B], g = gh[G_G], nh = gh[G_NH], h0 = gh[G_H0];
       if (gh[G_WMETA] && lane == 0) a.meta_out[b] = make_int4(gh[G_MC], gh[G_ME], gh[G_MP], 0);
@@ -356,33 +374,6 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
                                        ((((size_t)b * a.G + g) * 2 * a.L + slot0 + t) * kCols) * esz + c16 * 16) = v;
           }
         }
-        // x rows of the new tokens go to each head's ring row, straight from the inputs: eight
-        // 16-byte loads in flight per lane before the stores
-        {
-          const int xq = a.P * esz / 16, nq = n_new * nh * xq;
-          for (int q0 = 0; q0 < nq; q0 += 256) {
-            uint4 v[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int q = q0 + k * 32 + lane;
-              if (q < nq) {
-                const int c16 = q % xq, ti2 = q / xq, t = ti2 / nh, i = ti2 % nh;
-                v[k] = *reinterpret_cast<const uint4 *>(reinterpret_cast<const unsigned char *>(a.x) +
-                                                        (((size_t)b * a.T + t) * a.H + h0 + i) * a.P * esz + c16 * 16);
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int q = q0 + k * 32 + lane;
-              if (q < nq) {
-                const int c16 = q % xq, ti2 = q / xq, t = ti2 / nh, i = ti2 % nh;
-                const size_t unit = (size_t)b * a.H + h0 + i;
-                *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_x) +
-                                           ((unit * 2 * a.L + slot0 + t) * a.P) * esz + c16 * 16) = v[k];
-              }
-            }
-          }
-        }
         // dt of the new tokens goes to each head's ring row
         for (int q = lane; q < n_new * nh; q += 32) {
           const int t = q / nh, i = q % nh;
@@ -396,16 +387,39 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
           const int i = pr / t_out, j = pr % t_out;
           const float A = gf[G_A + i];
           const int e_j = n_rec - t_out + j + 1;
-          float *co = T.coef + (i * NO + j) * rmax;
-          for (int r = e_j; r < n_rec; ++r) co[r] = 0.f;
           float sfx = 0.f;
-          for (int r = e_j - 1; r >= m; --r) {
-            const float d = dt_of(i, r);
-            co[r] = d * __expf(A * sfx) * T.g[j * rmax + r];
-            sfx += d;
+          if constexpr (kMma) {
+            // coefficient row j of head i as the A operand of nq 16-record tensor-core steps, split
+            // into bf16 hi + lo: record r = 16q + k sits with lane 4j + (k & 7) / 2, word (k >= 8),
+            // half (k & 1); words 2, 3 repeat words 0, 1 for the lo part.  Records outside
+            // [m, e_j), up to 16 nq, are zero.
+            unsigned short *cf = reinterpret_cast<unsigned short *>(T.coef) + (size_t)i * lay.nq * 32 * 8;
+            for (int r = 16 * lay.nq - 1; r >= 0; --r) {
+              float co = 0.f;
+              if (r >= m && r < e_j) {
+                const float d = dt_of(i, r);
+                co = d * __expf(A * sfx) * T.g[j * rmax + r];
+                sfx += d;
+              }
+              if (r == e_j - 1) co += gf[G_D + i];
+              const __nv_bfloat16 hi = __float2bfloat16_rn(co);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(co - __bfloat162float(hi));
+              const int q = r >> 4, k = r & 15;
+              unsigned short *w = cf + ((q * 32 + 4 * j + ((k & 7) >> 1)) * 4 + (k >> 3)) * 2 + (k & 1);
+              w[0] = __bfloat16_as_ushort(hi);
+              w[4] = __bfloat16_as_ushort(lo);
+            }
+          } else {
+            float *co = T.coef + (i * NO + j) * rmax;
+            for (int r = e_j; r < n_rec; ++r) co[r] = 0.f;
+            for (int r = e_j - 1; r >= m; --r) {
+              const float d = dt_of(i, r);
+              co[r] = d * __expf(A * sfx) * T.g[j * rmax + r];
+              sfx += d;
+            }
+            for (int r = 0; r < m; ++r) co[r] = 0.f;
+            co[e_j - 1] += gf[G_D + i];
           }
-          for (int r = 0; r < m; ++r) co[r] = 0.f;
-          co[e_j - 1] += gf[G_D + i];
           T.ao[i * NO + j] = __expf(A * sfx);
         }
         if (m > 0 && lane < nh) {
@@ -426,8 +440,9 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   } else {
     // ================================================================== consumer warps
     const int row0 = warp * 8;
+    const uint64_t pol_ring = policy_evict_last();
     int ti = 0;
-    for (int u = u_begin, gi = 0; u < u_end; ++u, ++gi) {
+    for (int gi = 0;; ++gi) {
       const int gs = gi % kGB, tsl = gi & 1;
       if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
@@ -435,17 +450,33 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       const unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       const int *gh = reinterpret_cast<const int *>(gb);
+      if (gh[G_END]) break;
       const int b = gh[G_B], h0 = gh[G_H0], nh = gh[G_NH];
       if (gh[G_ACTIVE]) {
         const Tables T = tables(tsl);
         const float *t_coef = T.coef, *t_ao = T.ao, *t_wf = T.wf, *t_af = T.af;
         const int n_rec = gh[G_NREC], m = gh[G_M], t_out = gh[G_TOUT];
+        const int n_ring = gh[G_NRING], n_new = gh[G_NNEW], slot0 = gh[G_SLOT0];
         const TI *Bg = reinterpret_cast<const TI *>(gb + lay.gb_B);
         const TI *Cg = reinterpret_cast<const TI *>(gb + lay.gb_C);
         // ---- stream the heads' tiles; each warp works and releases on its own
-        float4 cv[NO];
+        float4 cv[kMma ? 1 : NO];
+        // tensor-core path: C_j as the B operand of eight 16-column steps (column j = lane / 4;
+        // lane 4g + t holds columns 16c + 4t .. 16c + 4t + 3 of step c, the k order the S' loads use)
+        uint32_t ac[kMma ? 8 : 1][2];
+        if constexpr (kMma) {
+          const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-        for (int j = 0; j < NO; ++j) cv[j] = (j < t_out) ? load4(Cg + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
+          for (int c = 0; c < 8; ++c) {
+            uint2 v = make_uint2(0u, 0u);
+            if (g < t_out) v = *reinterpret_cast<const uint2 *>(Cg + g * kCols + 16 * c + 4 * t4);
+            ac[c][0] = v.x;
+            ac[c][1] = v.y;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NO; ++j) cv[j] = (j < t_out) ? load4(Cg + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
+        }
         constexpr int V = 8 * NO;
         constexpr int KEEP = V >= 32 ? V / 32 : 1;
         constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
@@ -460,10 +491,22 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
           const TI *xr = reinterpret_cast<const TI *>(st + lay.xr);
           const int h = h0 + i;
           const size_t unit = (size_t)b * a.H + h;
+          // the new tokens' x rows, landed in the stage behind the buffered ones, go to the head's
+          // ring row with one bulk store (warps take turns); the stage is released after it has
+          // been read
+          const bool appender = (ti & (kConsumerWarps - 1)) == warp && n_new > 0;
+          if (appender && lane == 0) {
+            const uint32_t xrow = (uint32_t)a.P * esz;
+            bulk_s2g(reinterpret_cast<unsigned char *>(a.ring_x) + (unit * 2 * a.L + slot0) * xrow,
+                     st + lay.xr + (size_t)n_ring * xrow, (uint32_t)n_new * xrow, pol_ring);
+            bulk_commit();
+          }
           if (row0 < a.P) {
             float4 sv[8];
+            if (!kMma || m > 0) {
 #pragma unroll
             for (int rr = 0; rr < 8; ++rr) sv[rr] = *reinterpret_cast<const float4 *>(tile + (row0 + rr) * kCols + 4 * lane);
+            }
             if (m > 0) {
               const float af = t_af[i];
 #pragma unroll
@@ -496,7 +539,55 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
 #pragma unroll
               for (int rr = 0; rr < 8; ++rr)
                 __stcs(reinterpret_cast<float4 *>(dst + (row0 + rr) * kCols + 4 * lane), sv[rr]);
+              if constexpr (kMma) {  // the folded rows replace this warp's rows of the stage
+                float *tw = const_cast<float *>(tile);
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) *reinterpret_cast<float4 *>(tw + (row0 + rr) * kCols + 4 * lane) = sv[rr];
+                fence_async_smem();  // ordered before the stage's next bulk fill
+                __syncwarp();
+              }
             }
+            if constexpr (kMma) {
+              if (t_out > 0) {
+                // D[16 x 8] = [S'_hi; S'_lo] (the warp's 8 state rows, split into bf16 hi and lo
+                // halves as rows 0-7 and 8-15) times [C_1 .. C_T] over 8 k-steps of 16 state
+                // columns, in two independent accumulators; lane 4g + t then holds rows
+                // p = row0 + g, outputs j = 2t, 2t + 1 of both halves.  The buffered term
+                // sum_r x_r[p] coef_{j,r} follows as [x_r (exact bf16); 0] times the coefficient
+                // split into hi + lo, over 16-record steps.
+                const int g = lane >> 2, t4 = lane & 3;
+                float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+                const float *srow = tile + (row0 + g) * kCols + 4 * t4;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const float4 v = *reinterpret_cast<const float4 *>(srow + 16 * c);
+                  uint32_t h0, l0, h1, l1;
+                  split_bf16x2(v.x, v.y, h0, l0);
+                  split_bf16x2(v.z, v.w, h1, l1);
+                  mma_16816((c & 1) ? d1 : d0, h0, l0, h1, l1, ac[c][0], ac[c][1]);
+                }
+                float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint4 *cf = reinterpret_cast<const uint4 *>(t_coef) + (size_t)i * lay.nq * 32;
+                const unsigned short *xs = reinterpret_cast<const unsigned short *>(xr) + row0 + g;
+                for (int q = 0; q * 16 < n_rec; ++q) {
+                  const uint4 w = cf[q * 32 + lane];
+                  const int r0 = 16 * q + 2 * t4;
+                  const uint32_t x0 = r0 < n_rec ? xs[r0 * a.P] : 0u, x1 = r0 + 1 < n_rec ? xs[(r0 + 1) * a.P] : 0u;
+                  const uint32_t x8 = r0 + 8 < n_rec ? xs[(r0 + 8) * a.P] : 0u;
+                  const uint32_t x9 = r0 + 9 < n_rec ? xs[(r0 + 9) * a.P] : 0u;
+                  const uint32_t xa = x0 | (x1 << 16), xb = x8 | (x9 << 16);
+                  mma_16816(e0, xa, 0u, xb, 0u, w.x, w.y);
+                  mma_16816(e1, xa, 0u, xb, 0u, w.z, w.w);
+                }
+                const int j0 = 2 * t4;
+                float *yo = a.y + (((size_t)b * a.T + j0) * a.H + h) * a.P + row0 + g;
+                const size_t jstride = (size_t)a.H * a.P;
+                if (j0 < t_out)
+                  yo[0] = t_ao[i * NO + j0] * ((d0[0] + d1[0]) + (d0[2] + d1[2])) + (e0[0] + e1[0]);
+                if (j0 + 1 < t_out)
+                  yo[jstride] = t_ao[i * NO + j0 + 1] * ((d0[1] + d1[1]) + (d0[3] + d1[3])) + (e0[1] + e1[1]);
+              }
+            } else {
             // S'[row] . (ao_j C_j) over this lane's 4 columns, plus the buffered part: lane r
             // (< n_rec) adds coef_{j,r} x_r[row] for the warp's 8 rows (one 16-byte load of x_r)
             float part[V];
@@ -526,7 +617,9 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
               if (j < t_out && (lane % SPREAD) == 0)
                 a.y[(((size_t)b * a.T + j) * a.H + h) * a.P + row0 + rr] = part[k2];
             }
+            }
           }
+          if (appender && lane == 0) bulk_wait_read();
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[s]);
         }
@@ -538,6 +631,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         mbar_arrive(&tempty[tsl]);
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
@@ -547,6 +641,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     for (int s = 0; s < kGB; ++s)
       if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
   }
+  if (threadIdx.x == 0) sched_finish(a.err);
 }
 
 }  // namespace

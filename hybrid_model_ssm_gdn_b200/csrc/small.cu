@@ -15,7 +15,11 @@ namespace {
 __global__ void meta_reset_kernel(int4 *meta, int Bt, int *err) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < 2 * Bt) meta[i] = make_int4(0, 0, 0, 0);
-  if (i == 0) *err = kErrClean;
+  if (i == 0) {
+    err[0] = kErrClean;
+    err[1] = 0;  // unit scheduler: next unit, blocks finished
+    err[2] = 0;
+  }
 }
 
 __global__ void commit_kernel(const int4 *meta_in, int4 *meta_out, const int *accepted, int Bt, int *err) {

@@ -115,7 +115,8 @@ rssm_status rssm_arena_bytes(const rssm_config *cfg, size_t *bytes);
 
 /* Create a context over a caller-owned device arena (256-byte aligned, >= rssm_arena_bytes).
  * Only the small host handle is allocated (malloc).  The arena contents are undefined
- * until rssm_load_checkpoint. */
+ * until rssm_load_checkpoint: until its first success, every other call on the context
+ * (decode, commit, flush, export, rssm_get_error) returns RSSM_ERR_UNSUPPORTED. */
 rssm_status rssm_create(const rssm_config *cfg, void *arena, size_t arena_bytes, rssm_ctx **out);
 
 /* Free the host handle.  The arena stays the caller's. */

@@ -7,8 +7,8 @@ import torch
 from gpu_harness import TOL_F32, dev, head_rel_err
 from hybrid_model_ssm_gdn_b200 import conv_gdn_step, conv_mamba2_step, make_config, snap_commit, snap_verify
 from oracle import recurrence as rc
-from synth import (GDN_B256, MAMBA2_TINY, accepted_lengths, gdn_initial_state, gdn_step_inputs, mamba2_draft_inputs,
-                   mamba2_initial_state, mamba2_params, mamba2_step_inputs)
+from synth import (GDN_B256, MAMBA2_TINY, accepted_lengths, gdn_draft_inputs, gdn_initial_state, gdn_step_inputs,
+                   mamba2_draft_inputs, mamba2_initial_state, mamba2_params, mamba2_step_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +71,35 @@ def test_snapshot_per_draft_mamba2(cuda_ok, T):
         for j in range(T):
             Sj, yj = rc.mamba2_step(states[-1], dr["x"][:, j], dr["B"][:, j], dr["C"][:, j], dr["dt"][:, j],
                                     p["A"], p["D"], hg)
+            states.append(Sj)
+            assert head_rel_err(y[:, j].cpu().numpy(), yj).max() <= TOL_F32
+        snap_commit(cfg, cur, torch.from_numpy(acc).cuda())
+        S_ref = np.stack([states[a][b] for b, a in enumerate(acc)])
+        live = snaps[torch.arange(wl.batch), cur.long()].cpu().numpy()
+        err = head_rel_err(live.reshape(wl.batch, wl.nheads, -1), S_ref.reshape(wl.batch, wl.nheads, -1))
+        assert err.max() <= 1e-5
+
+
+@pytest.mark.parametrize("T", [4, 8])
+def test_snapshot_per_draft_gdn(cuda_ok, T):
+    """GDN snapshot-per-draft verify and its commit against the float64 recurrence."""
+    wl = GDN_B256.replace(batch=3, nheads=4, dv=96)
+    cfg = make_config("gdn", wl.batch, wl.nheads, wl.dv, 128, 1, wl.window, T, torch.bfloat16)
+    S0 = gdn_initial_state(wl)
+    snaps = torch.zeros(wl.batch, T + 1, wl.nheads, wl.dv, 128, device="cuda")
+    snaps[:, 0].copy_(torch.from_numpy(S0))
+    cur = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
+    S_ref = S0.astype(np.float64)
+    y = torch.empty(wl.batch, T, wl.nheads, wl.dv, device="cuda")
+    for rnd in range(5):
+        dr = gdn_draft_inputs(wl, rnd, T)
+        d = {k: dev(v, torch.float32 if k in ("alpha", "beta") else torch.bfloat16) for k, v in dr.items()}
+        snap_verify(cfg, snaps, cur, T, y, **d)
+        acc = accepted_lengths(wl, rnd, T)
+        states = [S_ref]
+        for j in range(T):
+            Sj, yj = rc.gdn_step(states[-1], dr["q"][:, j], dr["k"][:, j], dr["v"][:, j], dr["alpha"][:, j],
+                                 dr["beta"][:, j])
             states.append(Sj)
             assert head_rel_err(y[:, j].cpu().numpy(), yj).max() <= TOL_F32
         snap_commit(cfg, cur, torch.from_numpy(acc).cuda())

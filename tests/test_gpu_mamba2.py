@@ -52,9 +52,11 @@ def test_fewer_units_than_sms(cuda_ok):
     run_steps(p, 20)
 
 
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("T", [1, 4, 8])
-def test_verify_commit_random(cuda_ok, T):
-    wl = SPEC_MAMBA2_B512.replace(batch=6, nheads=16, ngroups=2)
+def test_verify_commit_random(cuda_ok, T, in_dtype):
+    """bf16 inputs with T > 4 take the tensor-core output path; fp32 inputs and T <= 4 the CUDA-core one."""
+    wl = SPEC_MAMBA2_B512.replace(batch=6, nheads=16, ngroups=2, in_dtype=in_dtype)
     p = Pair(wl, max_draft=T)
     step = 0
     for rnd in range(12):
@@ -69,6 +71,20 @@ def test_verify_commit_random(cuda_ok, T):
                 step += 1
                 assert head_rel_err(y, y_true).max() <= TOL_F32
         p.check_bookkeeping()
+    assert p.gpu.get_error() == (0, -1)
+
+
+@pytest.mark.parametrize("T", [3, 8])
+def test_verify_long_window_ragged_rows(cuda_ok, T):
+    """L = 32 (up to 40 records per verify: three 16-record steps), P = 40 (five active row groups)."""
+    wl = SPEC_MAMBA2_B512.replace(batch=5, nheads=20, headdim=40, ngroups=2, window=32)
+    p = Pair(wl, max_draft=T)
+    for rnd in range(14):
+        y, _, y_true = p.verify(T, mamba2_draft_inputs(wl, rnd, T))
+        assert head_rel_err(y, y_true).max() <= TOL_F32
+        p.commit(accepted_lengths(wl, rnd, T))
+        p.check_bookkeeping()
+    p.check_checkpoint()
     assert p.gpu.get_error() == (0, -1)
 
 
@@ -118,6 +134,28 @@ def test_device_errors_leave_state_untouched(cuda_ok):
     assert p2.gpu.get_error() == (abi.DEV_PENDING, 1)    # lowest (sequence, code), sticky
     assert p2.orc.err == (1, abi.DEV_PENDING)
     p2.check_bookkeeping()
+
+
+def test_calls_before_load_are_refused(cuda_ok):
+    """Until the first checkpoint load the arena is undefined: decode, commit and error reads are refused."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM, abi
+    wl = MAMBA2_TINY.replace(batch=2, nheads=4, in_dtype="bf16")
+    from synth import mamba2_params
+    p = mamba2_params(wl)
+    layer = ReplaySSM("mamba2", wl.batch, wl.nheads, wl.headdim, 128, wl.ngroups, wl.window, 2, torch.bfloat16,
+                      A=torch.from_numpy(p["A"]), D=torch.from_numpy(p["D"]))
+    d = {k: torch.from_numpy(v).cuda().to(torch.bfloat16) for k, v in mamba2_step_inputs(wl, 0).items()}
+    for call in (lambda: layer.mamba2_step(d["x"], d["B"], d["C"], d["dt"]),
+                 lambda: layer.commit(torch.zeros(wl.batch, dtype=torch.int32, device="cuda")),
+                 lambda: layer.flush(), lambda: layer.get_error()):
+        with pytest.raises(abi.RSSMError) as ei:
+            call()
+        assert ei.value.status == 3
+    layer.load_checkpoint(torch.zeros(wl.batch, wl.nheads, wl.headdim, 128, device="cuda"))
+    layer.mamba2_step(d["x"], d["B"], d["C"], d["dt"])
+    assert layer.get_error() == (0, -1)
 
 
 @pytest.mark.slow
