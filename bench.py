@@ -492,7 +492,7 @@ def gdn_section(steps: int) -> dict:
             "steps": K, "device_error": layer.get_error()}
 
 
-def verify_section(rounds: int) -> dict:
+def verify_section(rounds: int, kinds=("mamba2", "gdn")) -> dict:
     """Speculative verify + commit (T = 4, 8) vs snapshot-per-draft: the Mamba-2 shape at batch 512 and the
     Gated DeltaNet layer at batch 256."""
     import torch
@@ -503,6 +503,8 @@ def verify_section(rounds: int) -> dict:
     out = {"workload": "mamba2 speculative verify + commit, batch 512, 128 heads, P 64, N 128, 8 groups, L 16",
            "gdn": {"workload": "gdn speculative verify + commit, batch 256, 32 heads, d_k = d_v = 128, L 16"}}
     for kind, wl in (("mamba2", SPEC_MAMBA2_B512), ("gdn", GDN_B256)):
+        if kind not in kinds:
+            continue
         if kind == "mamba2":
             p = mamba2_params(wl)
             A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
@@ -600,7 +602,7 @@ def main():
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN and speculative-verify sections")
-    ap.add_argument("--only", choices=["gdn", "verify", "window"], default=None,
+    ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -617,7 +619,9 @@ def main():
     if args.only is not None:
         if rank == 0:
             out = (gdn_section(args.steps) if args.only == "gdn" else
-                   verify_section(args.steps) if args.only == "verify" else window_section())
+                   verify_section(args.steps) if args.only == "verify" else
+                   verify_section(args.steps, (args.only.split("-")[1],)) if args.only.startswith("verify-") else
+                   window_section())
             print(json.dumps(out))
         return
 
