@@ -76,6 +76,22 @@ def test_verify_commit_random(cuda_ok, T):
     assert p.gpu.get_error() == (0, -1)
 
 
+@pytest.mark.parametrize("T,in_dtype,L,dv", [(8, "f32", 16, 128), (8, "bf16", 32, 96), (3, "bf16", 32, 96),
+                                              (5, "bf16", 8, 128)])
+def test_verify_paths(cuda_ok, T, in_dtype, L, dv):
+    """bf16 and fp32 inputs, 3 to 8 outputs per row; L = 32 gives up to 40 records per verify, d_v = 96 leaves a
+    32-row tile."""
+    wl = SMALL.replace(batch=3, nheads=3, window=L, dv=dv, in_dtype=in_dtype)
+    p = Pair(wl, max_draft=T)
+    for rnd in range(12):
+        y, _, y_true = p.verify(T, gdn_draft_inputs(wl, rnd, T))
+        assert head_rel_err(y, y_true).max() <= TOL_F32
+        p.commit(accepted_lengths(wl, rnd, T))
+        p.check_bookkeeping()
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
 def test_flush_mask(cuda_ok):
     p = Pair(SMALL)
     run_steps(p, 5)
@@ -165,6 +181,26 @@ def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
         assert errs.mean() <= 2 * spread.mean() + TOL_F32
     else:
         assert frac <= FLIP_FRACTION
+
+
+@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "same")])
+def test_verify_lowprec_modes(cuda_ok, hp, read):
+    """8-draft verify reading an NVFP4 copy or an fp16 checkpoint against the method-mirroring oracle, with the
+    flip-aware bound of the step test."""
+    wl = GDN_LOWPREC.replace(batch=3, nheads=4, window=8)
+    p = Pair(wl, hp=hp, read=read, seed=7, max_draft=8)
+    errs = []
+    for rnd in range(10):
+        y, y_ref, _ = p.verify(8, gdn_draft_inputs(wl, rnd, 8))
+        err = head_rel_err(y, y_ref)
+        assert err.max() <= TOL_FLIP, f"round {rnd}: {err.max():.3e}"
+        errs.append(err.ravel())
+        p.commit(accepted_lengths(wl, rnd, 8))
+        p.check_bookkeeping(ring=False)
+    errs = np.concatenate(errs)
+    if hp == "f32":
+        assert float(np.mean(errs > TOL_F32)) <= FLIP_FRACTION
+    assert p.gpu.get_error() == (0, -1)
 
 
 @pytest.mark.slow
