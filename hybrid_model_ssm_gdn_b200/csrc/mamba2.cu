@@ -349,20 +349,44 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         auto dt_of = [&](int i, int r) -> float {
           return r < n_ring ? dtg[i * dts + base_e + r] : gf[G_DT + (r - n_ring) * kHG + i];
         };
-        // g[j][r] = B_r . C_j, eight records per task
-        const int rblocks = (n_rec + 7) / 8;
-        for (int task = 0; task < t_out * rblocks; ++task) {
-          const int j = task / rblocks, r0 = (task % rblocks) * 8;
-          const float4 cv = load4(Cg + j * kCols + 4 * lane);
-          float pd[8];
+        if constexpr (kMma) {
+          // g[j][r] = B_r . C_j on tensor cores (both exact in bf16): rows = outputs (8 of 16), columns =
+          // 8 records per tile, 8 k-steps of 16 state columns
+          const int gq = lane >> 2, tq = lane & 3;
+          uint32_t ca[8][2];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int r = r0 + q < n_rec ? r0 + q : n_rec - 1;
-            const float4 bv = load4(Bg + r * kCols + 4 * lane);
-            pd[q] = bv.x * cv.x + bv.y * cv.y + bv.z * cv.z + bv.w * cv.w;
+          for (int c = 0; c < 8; ++c) {
+            const TI *cr = Cg + gq * kCols + 16 * c + 2 * tq;
+            ca[c][0] = gq < t_out ? *reinterpret_cast<const uint32_t *>(cr) : 0u;
+            ca[c][1] = gq < t_out ? *reinterpret_cast<const uint32_t *>(cr + 8) : 0u;
           }
-          warp_transpose_reduce<8>(pd, lane);
-          if ((lane & 3) == 0 && r0 + (lane >> 2) < n_rec) T.g[j * rmax + r0 + (lane >> 2)] = pd[0];
+          for (int r0 = 0; r0 < n_rec; r0 += 8) {
+            const TI *br = Bg + (size_t)min(r0 + gq, n_rec - 1) * kCols + 2 * tq;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              mma_16816(d, ca[c][0], 0u, ca[c][1], 0u, *reinterpret_cast<const uint32_t *>(br + 16 * c),
+                        *reinterpret_cast<const uint32_t *>(br + 16 * c + 8));
+            const int r = r0 + 2 * tq;
+            if (r < n_rec) T.g[gq * rmax + r] = d[0];
+            if (r + 1 < n_rec) T.g[gq * rmax + r + 1] = d[1];
+          }
+        } else {
+          // g[j][r] = B_r . C_j, eight records per task
+          const int rblocks = (n_rec + 7) / 8;
+          for (int task = 0; task < t_out * rblocks; ++task) {
+            const int j = task / rblocks, r0 = (task % rblocks) * 8;
+            const float4 cv = load4(Cg + j * kCols + 4 * lane);
+            float pd[8];
+  #pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int r = r0 + q < n_rec ? r0 + q : n_rec - 1;
+              const float4 bv = load4(Bg + r * kCols + 4 * lane);
+              pd[q] = bv.x * cv.x + bv.y * cv.y + bv.z * cv.z + bv.w * cv.w;
+            }
+            warp_transpose_reduce<8>(pd, lane);
+            if ((lane & 3) == 0 && r0 + (lane >> 2) < n_rec) T.g[j * rmax + r0 + (lane >> 2)] = pd[0];
+          }
         }
         // B records of the new tokens go to the group's ring row (first chunk only)
         if (gh[G_WB]) {
@@ -383,33 +407,60 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         // per-head weights of every record in every output (log-space suffix sums of dt):
         // coef[r] = dt_r exp(A s(r+1, e_j)) (B_r . C_j) for m <= r < e_j, plus D on the output's
         // own token r = e_j - 1, and 0 elsewhere; ao = exp(A s(m, e_j)) scales S' C_j
-        for (int pr = lane; pr < nh * t_out; pr += 32) {
-          const int i = pr / t_out, j = pr % t_out;
-          const float A = gf[G_A + i];
-          const int e_j = n_rec - t_out + j + 1;
-          float sfx = 0.f;
-          if constexpr (kMma) {
-            // coefficient row j of head i as the A operand of nq 16-record tensor-core steps, split
-            // into bf16 hi + lo: record r = 16q + k sits with lane 4j + (k & 7) / 2, word (k >= 8),
-            // half (k & 1); words 2, 3 repeat words 0, 1 for the lo part.  Records outside
-            // [m, e_j), up to 16 nq, are zero.
-            unsigned short *cf = reinterpret_cast<unsigned short *>(T.coef) + (size_t)i * lay.nq * 32 * 8;
-            for (int r = 16 * lay.nq - 1; r >= 0; --r) {
-              float co = 0.f;
-              if (r >= m && r < e_j) {
-                const float d = dt_of(i, r);
-                co = d * __expf(A * sfx) * T.g[j * rmax + r];
-                sfx += d;
+        if constexpr (kMma) {
+          // per head, T[x] = sum of dt over records x .. n_rec - 1 (records below m left out), by a reverse
+          // warp scan over lanes x and x + 32.  Record r weighs dt_r exp(A (T[r+1] - T[e_j])) (B_r . C_j) in
+          // output j for m <= r < e_j, plus D on r = e_j - 1, and ao_j = exp(A (T[m] - T[e_j])).  Lane 4j + t
+          // writes its fragment slot of every 16-record step (records 16q + 2t + {0, 1, 8, 9}) as bf16 hi
+          // and lo words.
+          const int jl = lane >> 2, tl = lane & 3;
+          const int e_l = n_rec - t_out + jl + 1;
+          const bool jv = jl < t_out;
+          for (int i = 0; i < nh; ++i) {
+            const float A = gf[G_A + i];
+            const float dlo = (lane >= m && lane < n_rec) ? dt_of(i, lane) : 0.f;
+            const float dhi = (lane + 32 >= m && lane + 32 < n_rec) ? dt_of(i, lane + 32) : 0.f;
+            float tlo = dlo, thi = dhi;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+              const float vlo = __shfl_down_sync(0xffffffffu, tlo, off);
+              const float vhi = __shfl_down_sync(0xffffffffu, thi, off);
+              if (lane + off < 32) {
+                tlo += vlo;
+                thi += vhi;
               }
-              if (r == e_j - 1) co += gf[G_D + i];
-              const __nv_bfloat16 hi = __float2bfloat16_rn(co);
-              const __nv_bfloat16 lo = __float2bfloat16_rn(co - __bfloat162float(hi));
-              const int q = r >> 4, k = r & 15;
-              unsigned short *w = cf + ((q * 32 + 4 * j + ((k & 7) >> 1)) * 4 + (k >> 3)) * 2 + (k & 1);
-              w[0] = __bfloat16_as_ushort(hi);
-              w[4] = __bfloat16_as_ushort(lo);
             }
-          } else {
+            tlo += __shfl_sync(0xffffffffu, thi, 0);
+            auto at = [&](float lo, float hi, int x) -> float {  // value of lane x of the 64-lane pair
+              const float a0 = __shfl_sync(0xffffffffu, lo, x & 31), a1 = __shfl_sync(0xffffffffu, hi, x & 31);
+              return x < 32 ? a0 : a1;
+            };
+            const float Te = at(tlo, thi, e_l), Tm = at(tlo, thi, m);
+            if (jv && tl == 0) T.ao[i * NO + jl] = __expf(A * (Tm - Te));
+            uint4 *cf = reinterpret_cast<uint4 *>(T.coef) + (size_t)i * lay.nq * 32;
+            for (int q = 0; q < lay.nq; ++q) {
+              float co[4];
+#pragma unroll
+              for (int z = 0; z < 4; ++z) {
+                const int r = 16 * q + 2 * tl + (z & 1) + 8 * (z >> 1);
+                const float Tn = at(tlo, thi, r + 1), dr = at(dlo, dhi, r);
+                float v = 0.f;
+                if (jv && r >= m && r < e_l) v = dr * __expf(A * (Tn - Te)) * T.g[jl * rmax + r];
+                if (jv && r == e_l - 1) v += gf[G_D + i];
+                co[z] = v;
+              }
+              uint4 w;
+              split_bf16x2(co[0], co[1], w.x, w.z);
+              split_bf16x2(co[2], co[3], w.y, w.w);
+              cf[q * 32 + lane] = w;
+            }
+          }
+        } else {
+          for (int pr = lane; pr < nh * t_out; pr += 32) {
+            const int i = pr / t_out, j = pr % t_out;
+            const float A = gf[G_A + i];
+            const int e_j = n_rec - t_out + j + 1;
+            float sfx = 0.f;
             float *co = T.coef + (i * NO + j) * rmax;
             for (int r = e_j; r < n_rec; ++r) co[r] = 0.f;
             for (int r = e_j - 1; r >= m; --r) {
@@ -419,8 +470,8 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
             }
             for (int r = 0; r < m; ++r) co[r] = 0.f;
             co[e_j - 1] += gf[G_D + i];
+            T.ao[i * NO + j] = __expf(A * sfx);
           }
-          T.ao[i * NO + j] = __expf(A * sfx);
         }
         if (m > 0 && lane < nh) {
           const int i = lane;
