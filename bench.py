@@ -109,20 +109,29 @@ def weak_scaling_value(tokens_per_rank_step: int, world: int, steps: int, max_ms
     return tokens_per_rank_step * world * steps / (max_ms * 1e-3)
 
 
+def source_hash(sources) -> str:
+    """sha1 of the kernel sources with comments and blank lines left out (a change of code, not of prose)."""
+    import hashlib
+    import re
+    m = hashlib.sha1()
+    for f in sources:
+        for line in open(os.path.join(ROOT, "hybrid_model_ssm_gdn_b200", "csrc", f)).read().splitlines():
+            code = re.sub(r"//.*$", "", line).strip()
+            if code:
+                m.update(code.encode() + b"\n")
+    return m.hexdigest()
+
+
 def profiled_traffic(summary: str, sources) -> "float | None":
     """DRAM bytes per launch from the committed ncu summary, or None if the kernel changed since it was taken."""
-    import hashlib
     import re
     path = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m = hashlib.sha1()
-    for f in sources:
-        m.update(open(os.path.join(ROOT, "hybrid_model_ssm_gdn_b200", "csrc", f), "rb").read())
     h = re.search(r"Kernel source hash[^`]*`([0-9a-f]+)`", text)
     t = re.search(r"traffic_bytes_per_launch_window_avg:\s*([0-9.]+)", text)
-    if not h or not t or h.group(1) != m.hexdigest():
+    if not h or not t or h.group(1) != source_hash(sources):
         return None
     return float(t.group(1))
 

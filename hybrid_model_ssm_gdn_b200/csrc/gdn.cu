@@ -20,11 +20,12 @@
 // that is also the state the recurrence continues from.  Outputs of a call that folds
 // come from the fp32 fold result.
 //
-// Block roles (one block per SM, persistent):
+// Block roles (one block per SM, persistent; units drawn from a per-launch counter):
 //  * producer warp: TMA bulk copies (cp.async.bulk) of each unit's k records, q and
 //    alpha/beta rows into one of three group buffers, one unit ahead of the unit whose
 //    tiles it is issuing, and of each 64-row tile of a head's state (in its stored
-//    format) plus the head's v records into a ring of stages;
+//    format) plus the head's v records into a ring of stages (the head's first tile
+//    stage also feeds the bulk store that appends its new v rows);
 //  * two prep warps: 8-lane subgroups walk q back for every (head, draft) pair of the
 //    unit, writing u_0 and the coefficients beta_r c_r into double-buffered tables;
 //    they also append k, alpha, beta of the new tokens and write the bookkeeping word;

@@ -17,18 +17,23 @@
 // (products of exp(dt A) taken in log space).  Only a fold writes the state; a plain
 // step reads the checkpoint once and writes its output and its input record.
 //
-// Work unit: (sequence, group of <= 16 heads sharing B and C).  Warp roles in a block:
-//  * producer warp: issues TMA bulk copies (cp.async.bulk; evict-first for the
-//    checkpoint stream) into a double-buffered group buffer (B, C and dt rows of the
-//    unit) and into a ring of tile stages (one head's checkpoint tile + its x records);
+// Work unit: (sequence, group of <= 16 heads sharing B and C).  The persistent blocks draw
+// units from a per-launch counter.  Warp roles in a block:
+//  * producer warp: takes the next unit, writes its schedule into one of three group
+//    buffers and issues TMA bulk copies (cp.async.bulk; evict-first for the checkpoint
+//    stream) of the unit's B, C and dt rows into it, one unit ahead, then of each head's
+//    checkpoint tile and x records into a ring of tile stages;
 //  * prep warp: one unit ahead of the consumers, computes from the group buffer the
 //    dot products B_r . C_j and every head's decay weights into double-buffered tables,
-//    appends the group's B records and writes the sequence's bookkeeping word;
+//    appends the group's B and dt records and writes the sequence's bookkeeping word;
 //  * eight consumer warps: warp w owns rows 8w..8w+7 of every tile, lane l columns
 //    4l..4l+3; a warp waits on the stage's full barrier, computes its rows (fold, dot
-//    products, transpose reduction, buffered part of y) and releases the stage on its
-//    own.  No block-wide barrier sits on the streaming path, so one block per SM keeps
-//    the checkpoint stream in flight while the next unit is being prepared.
+//    products, transpose reduction, buffered part of y), appends the head's new x rows
+//    with one bulk store when it is its turn, and releases the stage on its own.  With
+//    bf16 inputs and 5..8 outputs, S'.C and the buffered term run on tensor cores
+//    (mma.sync, register operands).  No block-wide barrier sits on the streaming path,
+//    so one block per SM keeps the checkpoint stream in flight while the next unit is
+//    being prepared.
 #include "common.cuh"
 #include "kernels.h"
 

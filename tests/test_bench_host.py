@@ -1,0 +1,56 @@
+"""Host-side pieces of bench.py: the traffic models and the link to the committed ncu summaries (CPU only)."""
+
+import os
+import sys
+
+import numpy as np
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+from synth import GDN_B256, MAMBA2_120B, SPEC_MAMBA2_B512  # noqa: E402
+
+
+def test_step_traffic_model_window():
+    """Over a window, the checkpoint is read every step and written once; records are read count times."""
+    wl = MAMBA2_120B
+    L, state = wl.window, wl.batch * wl.nheads * wl.headdim * wl.dstate * 4
+    parts = [bench.traffic_model(wl, c) for c in range(L)]
+    assert sum(p["state_read"] for p in parts) == L * state
+    assert sum(p["state_write"] for p in parts) == state
+    rec = parts[1]["ring_read"]
+    assert sum(p["ring_read"] for p in parts) == rec * L * (L - 1) // 2
+
+
+def test_verify_traffic_no_fold_and_fold():
+    """With T + count <= L nothing folds: every round reads the checkpoint once.  Accepting T every round
+    with L = 2T makes every second round pre-fold (one extra state write per sequence)."""
+    wl = SPEC_MAMBA2_B512.replace(batch=4, nheads=2, ngroups=1, window=8)
+    state = wl.nheads * wl.headdim * wl.dstate * 4
+    zero = [np.zeros(wl.batch, np.int32)] * 3
+    base = bench.verify_traffic(wl, 4, zero)
+    full = [np.full(wl.batch, 4, np.int32)] * 4
+    folded = bench.verify_traffic(wl, 4, full)
+    esz = 2
+    rec = wl.nheads * wl.headdim * esz + wl.ngroups * wl.dstate * esz + wl.nheads * 4
+    per_round_fixed = wl.batch * state + wl.batch * 4 * (
+        (wl.nheads * wl.headdim * esz + 2 * wl.ngroups * wl.dstate * esz + wl.nheads * esz) + rec + wl.nheads * wl.headdim * 4)
+    assert base == 3 * per_round_fixed
+    # counts before the rounds: 0, 4, 8 (pre-fold: 8 + 4 > 8), 4 -> one fold; buffered reads 0 + 4 + 8 + 4
+    assert folded == 4 * per_round_fixed + wl.batch * state + wl.batch * rec * (0 + 4 + 8 + 4)
+
+
+def test_gdn_traffic_model_window():
+    wl = GDN_B256
+    state = wl.batch * wl.nheads * wl.dv * wl.dk * 4
+    tot = sum(bench.gdn_traffic(wl, c) for c in range(wl.window))
+    assert tot > (wl.window + 1) * state
+    assert tot < (wl.window + 1) * state * 1.2
+
+
+def test_committed_profile_matches_kernel_source():
+    """The committed ncu summary of the headline kernel was taken on the present kernel code, so the bench
+    line reports its measured DRAM traffic (a kernel change without a new capture fails here)."""
+    t = bench.profiled_traffic("m2_replay_kernel__mamba2_b256_L16.md", ("mamba2.cu", "common.cuh", "kernels.h"))
+    assert t is not None
+    model = sum(sum(bench.traffic_model(MAMBA2_120B, c).values()) for c in range(MAMBA2_120B.window)) / 16
+    assert 0.9 * model < t < 1.1 * model
