@@ -19,7 +19,7 @@ import torch
 from . import abi
 from .abi import RSSMError
 
-__all__ = ["ReplaySSM", "RSSMError", "conv_mamba2_step", "conv_gdn_step", "snap_verify", "snap_commit",
+__all__ = ["ReplaySSM", "RSSMError", "conv_mamba2_step", "conv_gdn_step", "snap_verify", "snap_commit", "sched_probe",
            "make_config", "abi"]
 
 _DT = {torch.float32: abi.F32, torch.bfloat16: abi.BF16}
@@ -196,6 +196,17 @@ def snap_verify(cfg, snaps, cur, T, y, **tok):
     abi.check(lib.rssm_snap_verify(C.byref(cfg), _ptr(snaps), _ptr(cur), T, C.byref(toks), _ptr(y), _stream()),
               "rssm_snap_verify")
     return y
+
+
+def sched_probe(units, blocks):
+    """Run the unit-scheduler self-test (no caller device memory): -> (units drawn per block, units not drawn
+    exactly once)."""
+    lib = abi.load()
+    per_block = (C.c_int * blocks)()
+    bad = C.c_int(-1)
+    abi.check(lib.rssm_sched_probe(units, blocks, C.cast(per_block, C.c_void_p), C.cast(C.pointer(bad), C.c_void_p),
+                                   _stream()), "rssm_sched_probe")
+    return list(per_block), bad.value
 
 
 def snap_commit(cfg, cur, accepted):

@@ -60,6 +60,7 @@ _SIGS = {
     "rssm_conv_gdn_step": [C.POINTER(Config), _P, _P, _P, _P, _P, _P, _P, _P],
     "rssm_snap_verify": [C.POINTER(Config), _P, _P, C.c_int, C.POINTER(Tokens), _P, _P],
     "rssm_snap_commit": [C.POINTER(Config), _P, _P, _P],
+    "rssm_sched_probe": [C.c_int, C.c_int, _P, _P, _P],
 }
 
 _lib = None

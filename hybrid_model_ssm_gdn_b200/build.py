@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "lib", "librssm.so")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
-SOURCES = ["api.cu", "mamba2.cu", "gdn.cu", "lowprec.cu", "conv.cu", "small.cu"]
+SOURCES = ["api.cu", "mamba2.cu", "gdn.cu", "lowprec.cu", "conv.cu", "small.cu", "sched.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE]
 

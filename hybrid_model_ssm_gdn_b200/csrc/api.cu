@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include "kernels.h"
+#include "sched.h"
 
 using namespace rssm;
 
@@ -386,6 +387,13 @@ rssm_status rssm_snap_commit(const rssm_config *cfg, int *cur, const int *accept
   if (!cfg || !cur || !accepted) return RSSM_ERR_ARG;
   if (cfg->batch < 1 || cfg->max_draft < 1) return RSSM_ERR_SHAPE;
   cudaError_t e = launch_snap_commit(cur, accepted, cfg->batch, cfg->max_draft + 1, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RSSM_OK : cuda_fail(e);
+}
+
+rssm_status rssm_sched_probe(int units, int blocks, int *per_block, int *bad_units, rssm_stream stream) {
+  if (units < 1 || units > kProbeMaxUnits || blocks < 1 || blocks > kProbeMaxBlocks || !per_block || !bad_units)
+    return RSSM_ERR_ARG;
+  const cudaError_t e = launch_sched_probe(units, blocks, per_block, bad_units, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RSSM_OK : cuda_fail(e);
 }
 

@@ -218,6 +218,19 @@ rssm_status rssm_snap_verify(const rssm_config *cfg, float *snaps, const int *cu
                              float *y, rssm_stream stream);
 rssm_status rssm_snap_commit(const rssm_config *cfg, int *cur, const int *accepted, rssm_stream stream);
 
+/* ---------------------------------------------------------------- scheduler self-test */
+
+/* Run the unit scheduler of the replay kernels on its own: `blocks` blocks draw `units` work
+ * units from a counter with one atomic per unit, and the last block to finish re-arms the
+ * counter (the mechanism the replay kernels use on the counter in the context's arena).  Needs
+ * no caller device memory: the counter, per-unit claim marks and per-block tallies live in
+ * file-scope device arrays of the library, so calls must not overlap in time.
+ *   units 1 .. 65536, blocks 1 .. 1024;
+ *   per_block host int [blocks]: units each block drew (they sum to `units`);
+ *   bad_units host int [1]: number of units not drawn exactly once (0 when correct).
+ * Synchronises `stream`.  RSSM_ERR_ARG on a count out of range or a null pointer. */
+rssm_status rssm_sched_probe(int units, int blocks, int *per_block, int *bad_units, rssm_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
