@@ -613,6 +613,52 @@ def window_section(windows=(4, 8, 16, 32), windows_timed: int = 8) -> dict:
     return out
 
 
+def batch_section(batches=(1, 2, 4, 8, 16, 32, 64, 128, 256, 512), windows_timed: int = 4) -> dict:
+    """Mamba-2 layer (128 heads, P 64, N 128, 8 groups, L 16) at batch 1 .. 512: replay vs the conventional
+    step-by-step kernel, window-averaged step time.  At small batches both are bound by launch and per-unit
+    latency rather than by the state bytes, so the replay's gain should grow with the batch."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM, conv_mamba2_step, make_config
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    stream = torch.cuda.current_stream()
+    out = {"workload": "mamba2 decode, 128 heads, P 64, N 128, 8 groups, L 16, bf16 inputs, fp32 state; batch sweep"}
+    for Bt in batches:
+        wl = WL.replace(batch=Bt)
+        p = mamba2_params(wl)
+        A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
+        S0 = torch.from_numpy(mamba2_initial_state(wl)).to(dev)
+        pool = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in mamba2_step_inputs(wl, t).items()} for t in range(4)]
+        y = torch.empty(Bt, wl.nheads, wl.headdim, device=dev)
+        layer = ReplaySSM("mamba2", Bt, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window, 0, bf, A=A, D=D)
+        layer.load_checkpoint(S0)
+
+        def step(i):
+            t = pool[i % 4]
+            layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], y)
+
+        for i in range(2 * wl.window):
+            step(i)
+        K = wl.window * windows_timed
+        ms = timed(step, K, stream)
+        err = layer.get_error()
+        del layer
+        cfg = make_config("mamba2", Bt, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.window, 0, bf, A=A, D=D)
+        S = S0.clone()
+
+        def conv(i):
+            t = pool[i % 4]
+            conv_mamba2_step(cfg, S, t["x"], t["B"], t["C"], t["dt"], y)
+
+        for i in range(8):
+            conv(i)
+        ms_conv = timed(conv, K, stream)
+        del S, S0
+        out[f"B{Bt}"] = {"replay_ms_per_step": ms, "conventional_ms_per_step": ms_conv, "speedup": ms_conv / ms,
+                         "replay_tokens_per_s": Bt / (ms * 1e-3), "device_error": err}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -621,7 +667,7 @@ def main():
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN and speculative-verify sections")
-    ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window"], default=None,
+    ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -640,7 +686,7 @@ def main():
             out = (gdn_section(args.steps) if args.only == "gdn" else
                    verify_section(args.steps) if args.only == "verify" else
                    verify_section(args.steps, (args.only.split("-")[1],)) if args.only.startswith("verify-") else
-                   window_section())
+                   batch_section() if args.only == "batch" else window_section())
             print(json.dumps(out))
         return
 
