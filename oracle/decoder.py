@@ -42,9 +42,10 @@ Readings taken where the pages are silent (per sequence; L = window):
   precision; the stored checkpoint is read for folding, the read copy for
   outputs of calls that do not fold.
 
-Precision modes: hp = "f32" (fp32 checkpoint) or "f16sr" (fp16 with stochastic
+Precision modes: hp = "f32" (fp32 checkpoint), "f16sr" (fp16 with stochastic
 rounding, random words from Philox4x32-10 with counter (sequence*H + head,
-new epoch, element/4, 0) and the 64-bit seed as key); read = "same" (outputs
+new epoch, element/4, 0) and the 64-bit seed as key) or "f8sr" (E4M3 with a
+per-64-row-tile scale and the same stochastic rounding); read = "same" (outputs
 read the checkpoint), "nvfp4" (separate NVFP4 read copy, re-quantised from the
 fp32 fold result at every fold) or "shared_nvfp4" (the NVFP4 copy is also the
 checkpoint the recurrence continues from; contrast mode).  The NVFP4 copy is
@@ -83,7 +84,7 @@ class ReplayOracle:
     def __init__(self, kind, S0, window, *, nheads, ngroups=1, params=None, seq_ids=None, head_ids=None,
                  hp="f32", read="same", seed=0, q_scale=1.0):
         assert kind in ("mamba2", "gdn")
-        assert hp in ("f32", "f16sr") and read in ("same", "nvfp4", "shared_nvfp4")
+        assert hp in ("f32", "f16sr", "f8sr") and read in ("same", "nvfp4", "shared_nvfp4")
         self.kind, self.L, self.H, self.G = kind, int(window), int(nheads), int(ngroups)
         S0 = np.asarray(S0, np.float64)
         self.nb = S0.shape[0]
@@ -160,7 +161,10 @@ class ReplayOracle:
             units = int(self.seq_ids[b]) * self.H + self.head_ids.astype(np.int64)
             n = S32.shape[-1] * S32.shape[-2]
             words = sr_words(self.seed, units, int(self.epoch[b]), n).reshape(S32.shape)
-            self.hp[b] = lowprec.fp16_stochastic_round(S32, words).astype(np.float64)
+            if self.hp_mode == "f16sr":
+                self.hp[b] = lowprec.fp16_stochastic_round(S32, words).astype(np.float64)
+            else:
+                self.hp[b] = lowprec.fp8_quantize_state(S32, words)["values"].astype(np.float64)
         self.rd[b] = self.hp[b] if self.read_mode == "same" else self._read_copy(S32)
 
     def _error(self, b, code):

@@ -24,6 +24,16 @@ E2M1 (OCP FP4): magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}; round to nearest,
     ties to the even code; saturate at 6.  Code = sign << 3 | magnitude index,
     with the sign bit set iff x < 0.
 
+FP8 recurrence checkpoint (the pages evaluate NVFP4 reads with an FP16 or an FP8
+recurrence, "Hybrid-model decoding has a new bottleneck", Interpretation, fourth
+paragraph; the format and rounding are this reading, chosen like the FP16 mode).
+Per tile of 64 consecutive rows of one head's state:
+    s   = amax(tile) / 448 in fp32, or 1 if amax = 0
+    y   = x / s (fp32 divide), stochastically rounded to the E4M3 grid with the
+          FP16 rule above and E4M3 spacings (2^(floor(log2|y|) - 3), 2^-9 below
+          2^-6), saturating at 448; the random words are those of FP16 SR
+    value = E4M3(y) * s (fp32)
+
 NVFP4 read copy.  A tile is 64 consecutive rows (fewer for the last rows) of
 one sequence's and head's state matrix, all 128 columns; blocks are 16
 consecutive elements along the contracted (contiguous) axis:
@@ -71,6 +81,50 @@ def fp16_stochastic_round(x, r) -> np.ndarray:
     mag = np.where(finite, mag, np.where(mant == 0, FP16_MAX, np.nan))
     out = np.where(sign == 1, -mag, mag)
     return out.astype(np.float16)      # exact: every value is on the fp16 grid
+
+
+def e4m3_stochastic_round(y, r) -> np.ndarray:
+    """Stochastically round fp32 ``y`` to the E4M3FN grid with uint32 words ``r`` (the FP16 rule with E4M3
+    spacings), saturating at 448; returns float64 values on the grid."""
+    y = np.ascontiguousarray(y, np.float32)
+    r = np.asarray(r, np.uint32).astype(np.uint64)
+    bits = y.view(np.uint32).astype(np.uint64)
+    sign = (bits >> np.uint64(31)) & np.uint64(1)
+    E = ((bits >> np.uint64(23)) & np.uint64(0xFF)).astype(np.int64)
+    mant = bits & np.uint64(0x7FFFFF)
+    M = np.where(E > 0, mant | np.uint64(0x800000), mant)        # |y| = M * 2^(Eeff - 150)
+    Eeff = np.maximum(E, 1)
+    s = np.maximum(20, 141 - Eeff).astype(np.uint64)             # fp32 bits below the E4M3 spacing
+    q = np.where(s >= np.uint64(24), np.uint64(0), M >> np.minimum(s, np.uint64(63)))
+    F = np.where(s >= np.uint64(24), M, M & ((np.uint64(1) << np.minimum(s, np.uint64(63))) - np.uint64(1)))
+    thr = np.where(s <= np.uint64(32), F << (np.uint64(32) - np.minimum(s, np.uint64(32))),
+                   F >> (np.maximum(s, np.uint64(32)) - np.uint64(32)))
+    up = (r < thr).astype(np.uint64)
+    ulp_exp = np.maximum(Eeff - 127, -6) - 3
+    mag = np.minimum(np.ldexp((q + up).astype(np.float64), ulp_exp), E4M3_MAX)
+    return np.where(sign == 1, -mag, mag)
+
+
+def fp8_quantize_state(S, words) -> dict:
+    """FP8 checkpoint of states [..., rows, 128] by 64-row tiles with uint32 ``words`` [..., rows, 128].
+
+    Returns {"codes": uint8 [..., rows, 128] (E4M3 bit patterns), "s": float32 [..., ceil(rows/64)],
+    "values": float32 [..., rows, 128]}."""
+    x = np.ascontiguousarray(S, np.float32)
+    words = np.asarray(words, np.uint32).reshape(x.shape)
+    rows = x.shape[-2]
+    codes, scales, values = [], [], []
+    for r0 in range(0, rows, NVFP4_TILE_ROWS):
+        t = x[..., r0:r0 + NVFP4_TILE_ROWS, :]
+        amax = np.abs(t).reshape(*t.shape[:-2], -1).max(axis=-1)
+        s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        y = (t / s[..., None, None]).astype(np.float32)
+        q = e4m3_stochastic_round(y, words[..., r0:r0 + NVFP4_TILE_ROWS, :])
+        codes.append(e4m3_code(q))
+        scales.append(s)
+        values.append((q.astype(np.float32) * s[..., None, None]).astype(np.float32))
+    return {"codes": np.concatenate(codes, axis=-2), "s": np.stack(scales, axis=-1),
+            "values": np.concatenate(values, axis=-2)}
 
 
 # --------------------------------------------------------------------------- E4M3 / E2M1

@@ -169,3 +169,25 @@ def test_fp16_checkpoint_is_on_the_fp16_grid():
         o3.step(gdn_step_inputs(G_WL, t))
     np.testing.assert_array_equal(o.hp, o2.hp)
     assert np.any(o.hp != o3.hp)
+
+
+def test_fp8_checkpoint_tiles_and_separate_read_copy():
+    """FP8 checkpoint: each 64-row tile of the stored state is E4M3 grid values times one scale (its largest
+    magnitude / 448), and an NVFP4 read copy beside it leaves that checkpoint unchanged."""
+    import torch
+    grid = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    o = _gdn(4, hp="f8sr", seed=5)
+    sep = _gdn(4, hp="f8sr", read="nvfp4", seed=5)
+    for t in range(8):
+        o.step(gdn_step_inputs(G_WL, t))
+        sep.step(gdn_step_inputs(G_WL, t))
+        np.testing.assert_array_equal(sep.hp, o.hp)
+    rows = o.hp.shape[-2]
+    for r0 in range(0, rows, 64):
+        tile = o.hp[..., r0:r0 + 64, :]
+        s = np.abs(tile).max(axis=(-1, -2)) / 448.0
+        y = np.abs(tile) / s[..., None, None]
+        nearest = grid[np.clip(np.searchsorted(grid, y), 0, len(grid) - 1)]
+        below = grid[np.clip(np.searchsorted(grid, y) - 1, 0, len(grid) - 1)]
+        dist = np.minimum(np.abs(nearest - y), np.abs(below - y))
+        assert np.all(dist <= 1e-5 * np.maximum(y, 2.0 ** -9))

@@ -200,3 +200,80 @@ def test_nvfp4_state_tiles_are_64_rows():
     np.testing.assert_array_equal(lp.nvfp4_roundtrip_state(S)[..., :64, :], lp.nvfp4_roundtrip(S[..., :64, :]))
     S40 = S[..., :40, :]
     assert lp.nvfp4_quantize_state(S40)["g"].shape == (2, 3, 1)
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3) stochastic rounding
+
+def _e4m3_grid():
+    """All finite non-negative E4M3FN values, from torch's own conversion of the bit patterns."""
+    codes = torch.arange(0, 0x7F, dtype=torch.uint8)
+    return codes.view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+
+
+def test_fp8_sr_grid_points_unchanged():
+    g = _e4m3_grid()
+    v = np.concatenate([g, -g[1:]]).astype(np.float32)
+    for r in (0, 1, 0x80000000, 0xFFFFFFFF):
+        np.testing.assert_array_equal(lp.e4m3_stochastic_round(v, np.full(v.shape, r, np.uint32)), v.astype(np.float64))
+
+
+def test_fp8_sr_extreme_words_floor_or_ceil_to_the_grid():
+    """The largest word never rounds away from zero and the zero word always does (unless exact): the two
+    results are the E4M3 neighbours of |y| found by search in torch's grid."""
+    g = _e4m3_grid()
+    rng = np.random.default_rng(7)
+    y = (rng.standard_normal(20000) * 10.0 ** rng.uniform(-4, 2.6, 20000)).astype(np.float32)
+    y = y[np.abs(y) < 448]
+    a = np.abs(y).astype(np.float64)
+    idx = np.searchsorted(g, a, side="right") - 1
+    lo = g[idx]
+    hi = np.where(lo == a, lo, g[np.minimum(idx + 1, len(g) - 1)])
+    down = lp.e4m3_stochastic_round(y, np.full(y.shape, 0xFFFFFFFF, np.uint32))
+    up = lp.e4m3_stochastic_round(y, np.zeros(y.shape, np.uint32))
+    np.testing.assert_array_equal(np.abs(down), lo)
+    np.testing.assert_array_equal(np.abs(up), hi)
+    assert np.all(np.signbit(up) == np.signbit(y))
+
+
+def test_fp8_sr_threshold_is_exact_fraction():
+    # y = (q + k/8) u rounds up exactly for r < k * 2^29, normal (u = 2^-3 at 1) and subnormal (u = 2^-9)
+    for base, u in ((1.0, 2.0 ** -3), (3 * 2.0 ** -9, 2.0 ** -9), (256.0, 32.0)):
+        for k in range(1, 8):
+            y = np.float32(base + k / 8 * u)
+            thr = k << 29
+            out = lp.e4m3_stochastic_round(np.full(4, y), np.array([thr - 1, thr, 0, 0xFFFFFFFF], np.uint32))
+            assert out[0] == base + u and out[2] == base + u
+            assert out[1] == base and out[3] == base
+
+
+def test_fp8_sr_unbiased_and_saturating():
+    rng = np.random.default_rng(8)
+    y = (rng.standard_normal(32) * 10.0 ** rng.uniform(-3, 2, 32)).astype(np.float32)
+    r = (np.arange(65536, dtype=np.uint64) << np.uint64(16)).astype(np.uint32)
+    g = _e4m3_grid()
+    for yi in y:
+        a = abs(float(yi))
+        i = np.searchsorted(g, a, side="right") - 1
+        u = (g[min(i + 1, len(g) - 1)] - g[i]) if g[i] != a else 0.0
+        out = lp.e4m3_stochastic_round(np.full(r.shape, yi), r)
+        assert abs(out.mean() - float(yi)) <= u * 2.0 ** -16 * 1.0001
+    sat = lp.e4m3_stochastic_round(np.array([449.0, 1e6, -500.0], np.float32), np.zeros(3, np.uint32))
+    np.testing.assert_array_equal(sat, [448.0, 448.0, -448.0])
+
+
+def test_fp8_state_tiles_scale_and_bound():
+    """Tiles of 64 rows, s = amax / 448, values = E4M3(x / s) * s with each element within one grid step
+    of x; a zero tile keeps scale 1 and zero codes; codes decode to the values."""
+    rng = np.random.default_rng(9)
+    S = rng.standard_normal((2, 3, 96, 128)).astype(np.float32)
+    S[1, 2, 64:] = 0.0                                              # a zero tile (the second of that head)
+    words = rng.integers(0, 2 ** 32, S.shape, dtype=np.uint64).astype(np.uint32)
+    q = lp.fp8_quantize_state(S, words)
+    assert q["s"].shape == (2, 3, 2)
+    np.testing.assert_array_equal(q["s"][..., 0], (np.abs(S[..., :64, :]).max(axis=(-1, -2)) / np.float32(448)))
+    assert q["s"][1, 2, 1] == 1.0 and not q["codes"][1, 2, 64:].any()
+    s_rows = np.repeat(q["s"], 64, axis=-1)[..., :96, None]
+    y = (S / s_rows).astype(np.float32)
+    step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6))) - 3), 2.0 ** -9)
+    assert np.all(np.abs(q["values"] / s_rows - y) <= step * (1 + 1e-6))
+    np.testing.assert_array_equal((lp.e4m3_value(q["codes"]).astype(np.float32) * s_rows).astype(np.float32), q["values"])
