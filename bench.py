@@ -430,15 +430,27 @@ def run_gpu(args, rank, world):
     return res
 
 
-def gdn_traffic(wl, count_before: int) -> int:
-    """Algorithmic bytes of one GDN replay step (same terms as the Mamba-2 model)."""
+# bytes per state element of each stored format: fp32, fp16, E4M3 with one fp32 scale per 64 x 128 tile,
+# and NVFP4 (E2M1 codes, an E4M3 scale per 16 elements, one fp32 scale per tile)
+HP_BYTES = {"f32": 4.0, "f16sr": 2.0, "f8sr": 1.0 + 4.0 / (64 * 128)}
+NVFP4_BYTES = 0.5 + 1.0 / 16 + 4.0 / (64 * 128)
+
+
+def gdn_traffic(wl, count_before: int, hp: str = "f32", read: str = "same") -> float:
+    """Algorithmic bytes of one GDN replay step (same terms as the Mamba-2 model) with the checkpoint stored
+    as ``hp``.  Steps that do not fold read the checkpoint (``read="same"``) or the NVFP4 copy beside it
+    (``"nvfp4"``); a fold reads the checkpoint and writes it and the copy.  ``"shared_nvfp4"``: the NVFP4
+    copy is the checkpoint."""
     Bt, H, dk, dv, L = wl.batch, wl.nheads, wl.dk, wl.dv, wl.window
     esz = 2 if wl.in_dtype == "bf16" else 4
-    state = Bt * H * dv * dk * 4
+    elems = Bt * H * dv * dk
+    ckpt = elems * (NVFP4_BYTES if read == "shared_nvfp4" else HP_BYTES[hp])
+    copy = elems * NVFP4_BYTES if read == "nvfp4" else 0.0
     rec = Bt * H * (dk * esz + dv * esz + 8)
     tok = Bt * H * (2 * dk * esz + dv * esz + 8)
     fold = count_before + 1 == L
-    return state + (state if fold else 0) + count_before * rec + tok + rec + Bt * H * dv * 4
+    state = ckpt + ckpt + copy if fold else (copy if read == "nvfp4" else ckpt)
+    return state + count_before * rec + tok + rec + Bt * H * dv * 4
 
 
 def timed(fn, n, stream):
@@ -509,6 +521,59 @@ def gdn_section(steps: int) -> dict:
             "conventional_tokens_per_s": wl.batch / (ms_conv * 1e-3), "conventional_ms_per_step": ms_conv,
             "conventional_GBps": conv_bytes / (ms_conv * 1e-3) / 1e9, "replay_speedup": ms_conv / ms,
             "steps": K, "device_error": layer.get_error()}
+
+
+PRECISION_MODES = (("f32", "same"), ("f16sr", "same"), ("f8sr", "same"), ("f32", "nvfp4"), ("f16sr", "nvfp4"),
+                   ("f8sr", "nvfp4"), ("f32", "shared_nvfp4"))
+
+
+def precision_section(windows_timed: int = 4) -> dict:
+    """GDN layer (batch 256, 32 heads, d 128, L 16) with each checkpoint format and read mode: window-averaged
+    step time, plain and fold launches, and the rate of the mode's algorithmic bytes."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM
+    wl, dev, bf = GDN_B256, torch.device("cuda"), torch.bfloat16
+    S0 = torch.from_numpy(gdn_initial_state(wl)).to(dev)
+    pool = []
+    for t in range(16):
+        inp = gdn_step_inputs(wl, t)
+        pool.append({k: torch.from_numpy(v).to(dev).to(torch.float32 if k in ("alpha", "beta") else bf)
+                     for k, v in inp.items()})
+    y = torch.empty(wl.batch, wl.nheads, wl.dv, device=dev)
+    stream = torch.cuda.current_stream()
+    hbm, _ = load_peaks()
+    out = {"workload": "gdn replay decode, batch 256, 32 heads, d_k = d_v = 128, L 16, bf16 inputs; checkpoint "
+                       "format x read mode"}
+    for hp, read in PRECISION_MODES:
+        layer = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, wl.dk, 1, wl.window, 0, bf, hp, read, seed=3)
+        layer.load_checkpoint(S0)
+
+        def step(i):
+            t = pool[i % 16]
+            layer.gdn_step(t["q"], t["k"], t["v"], t["alpha"], t["beta"], y)
+
+        for i in range(2 * wl.window):
+            step(i)
+        K = wl.window * windows_timed
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(K):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+        ms = ev[0].elapsed_time(ev[K]) / K
+        nbytes = sum(gdn_traffic(wl, i % wl.window, hp, read) for i in range(K)) / K
+        out[f"{hp}/{read}"] = {
+            "ms_per_step": ms, "tokens_per_s": wl.batch / (ms * 1e-3), "bytes_per_step": nbytes,
+            "GBps": nbytes / (ms * 1e-3) / 1e9, "frac_of_measured_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+            "plain_launch_ms": statistics.median([d for i, d in enumerate(per) if (i + 1) % wl.window != 0]),
+            "fold_launch_ms": statistics.mean([d for i, d in enumerate(per) if (i + 1) % wl.window == 0]),
+            "device_error": layer.get_error()}
+        del layer
+    return out
 
 
 def verify_section(rounds: int, kinds=("mamba2", "gdn")) -> dict:
@@ -666,8 +731,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-extra", action="store_true", help="skip the GDN and speculative-verify sections")
-    ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch"], default=None,
+    ap.add_argument("--no-extra", action="store_true", help="skip the GDN, speculative-verify and precision sections")
+    ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch",
+                                                  "precision"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -686,7 +752,8 @@ def main():
             out = (gdn_section(args.steps) if args.only == "gdn" else
                    verify_section(args.steps) if args.only == "verify" else
                    verify_section(args.steps, (args.only.split("-")[1],)) if args.only.startswith("verify-") else
-                   batch_section() if args.only == "batch" else window_section())
+                   batch_section() if args.only == "batch" else
+                   precision_section() if args.only == "precision" else window_section())
             print(json.dumps(out))
         return
 
@@ -699,6 +766,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_extra:
         res["gdn"] = gdn_section(min(args.steps, 1024))
         res["verify"] = verify_section(512)
+        res["precision"] = precision_section()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -23,7 +23,7 @@ __all__ = ["ReplaySSM", "RSSMError", "conv_mamba2_step", "conv_gdn_step", "snap_
            "make_config", "abi"]
 
 _DT = {torch.float32: abi.F32, torch.bfloat16: abi.BF16}
-_HP = {"f32": abi.HP_F32, "f16sr": abi.HP_F16_SR}
+_HP = {"f32": abi.HP_F32, "f16sr": abi.HP_F16_SR, "f8sr": abi.HP_F8_SR}
 _READ = {"same": abi.READ_SAME, "nvfp4": abi.READ_NVFP4, "shared_nvfp4": abi.READ_SHARED_NVFP4}
 
 

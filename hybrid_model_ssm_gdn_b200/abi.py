@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libr
 # enums (values as in include/rssm.h)
 MAMBA2, GDN = 0, 1
 F32, BF16 = 0, 1
-HP_F32, HP_F16_SR = 0, 1
+HP_F32, HP_F16_SR, HP_F8_SR = 0, 1, 2
 READ_SAME, READ_NVFP4, READ_SHARED_NVFP4 = 0, 1, 2
 STATUS = {0: "RSSM_OK", 1: "RSSM_ERR_ARG", 2: "RSSM_ERR_SHAPE", 3: "RSSM_ERR_UNSUPPORTED",
           4: "RSSM_ERR_ARENA_TOO_SMALL", 5: "RSSM_ERR_CUDA", 6: "RSSM_ERR_DEVICE"}

@@ -39,7 +39,7 @@ rssm_status validate(const rssm_config *c) {
   if (!c) return RSSM_ERR_ARG;
   if (c->kind != RSSM_MAMBA2 && c->kind != RSSM_GDN) return RSSM_ERR_ARG;
   if (c->in_dtype != RSSM_F32 && c->in_dtype != RSSM_BF16) return RSSM_ERR_ARG;
-  if (c->hp != RSSM_HP_F32 && c->hp != RSSM_HP_F16_SR) return RSSM_ERR_ARG;
+  if (c->hp != RSSM_HP_F32 && c->hp != RSSM_HP_F16_SR && c->hp != RSSM_HP_F8_SR) return RSSM_ERR_ARG;
   if (c->read < RSSM_READ_SAME || c->read > RSSM_READ_SHARED_NVFP4) return RSSM_ERR_ARG;
   if (c->batch < 1 || c->nheads < 1) return RSSM_ERR_SHAPE;
   if ((long long)c->batch * c->nheads > (1LL << 26)) return RSSM_ERR_SHAPE;
@@ -102,6 +102,7 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   if (a.nstage < 2 || a.nstage > 8 || g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) > x->smem_optin) return RSSM_ERR_SHAPE;
   a.meta_in = meta_cur(x); a.meta_out = meta_next(x); a.err = err_word(x);
   a.hp = x->arena + x->lay.hp;
+  a.hs = reinterpret_cast<float *>(x->arena + x->lay.hs);
   a.rq = x->arena + x->lay.rq; a.rs = x->arena + x->lay.rs; a.rg = reinterpret_cast<float *>(x->arena + x->lay.rg);
   a.ring_k = x->arena + x->lay.ring_a; a.ring_v = x->arena + x->lay.ring_b;
   a.ring_a = reinterpret_cast<float *>(x->arena + x->lay.ring_c);
@@ -179,7 +180,8 @@ rssm_status rssm_load_checkpoint(rssm_ctx *x, const float *S, rssm_stream stream
   if (c.hp == RSSM_HP_F32 && c.read == RSSM_READ_SAME)
     e = cudaMemcpyAsync(x->arena + x->lay.hp, S, units * c.headdim * kCols * 4, cudaMemcpyDeviceToDevice, st);
   else
-    e = launch_store_state(S, x->arena + x->lay.hp, c.hp, x->arena + x->lay.rq, x->arena + x->lay.rs,
+    e = launch_store_state(S, x->arena + x->lay.hp, reinterpret_cast<float *>(x->arena + x->lay.hs), c.hp,
+                           x->arena + x->lay.rq, x->arena + x->lay.rs,
                            reinterpret_cast<float *>(x->arena + x->lay.rg), c.read, (int)units, c.headdim, c.seed,
                            c.nheads, st);
   if (e == cudaSuccess)  // empty ring: count = 0 everywhere; zeroed so exports are deterministic
@@ -251,7 +253,8 @@ rssm_status rssm_export(rssm_ctx *x, float *S_out, void *ring_out, int *meta_out
     if (c.hp == RSSM_HP_F32 && c.read != RSSM_READ_SHARED_NVFP4)
       e = cudaMemcpyAsync(S_out, x->arena + x->lay.hp, units * R * kCols * 4, cudaMemcpyDeviceToDevice, st);
     else
-      e = launch_widen_state(x->arena + x->lay.hp, c.hp, x->arena + x->lay.rq, x->arena + x->lay.rs,
+      e = launch_widen_state(x->arena + x->lay.hp, reinterpret_cast<const float *>(x->arena + x->lay.hs), c.hp,
+                             x->arena + x->lay.rq, x->arena + x->lay.rs,
                              reinterpret_cast<const float *>(x->arena + x->lay.rg), c.read, S_out, (int)units, R, st);
   }
   if (e == cudaSuccess && meta_out) e = launch_export_meta(meta_cur(x), meta_out, c.batch, L, st);

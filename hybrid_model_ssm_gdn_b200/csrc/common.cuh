@@ -39,7 +39,8 @@ __host__ __device__ inline int dt_stride(int L) { return (int)align_up((size_t)(
 struct ArenaLayout {
   size_t meta;     // int4 [2][Bt]: count, epoch, pending, 0  (ping-pong by call parity)
   size_t err;      // int [4]: sticky error word, next unit to hand out, blocks finished, 0
-  size_t hp;       // checkpoint: fp32 or fp16 [Bt][H][R][128]
+  size_t hp;       // checkpoint: fp32, fp16 or E4M3 [Bt][H][R][128]
+  size_t hs;       // E4M3 checkpoint tile scales fp32 [Bt][H][ceil(R/64)] (padded to 16 bytes)
   size_t rq;       // NVFP4 codes u8 [Bt][H][R][64]
   size_t rs;       // NVFP4 block scales u8 [Bt][H][R][8]
   size_t rg;       // NVFP4 tile scale fp32 [Bt][H][ceil(R/64)] (padded to 16 bytes)
@@ -60,7 +61,9 @@ inline ArenaLayout make_layout(const rssm_config &c) {
   a.meta = take(2 * Bt * 16);
   a.err = take(16);
   const bool shared_fp4 = c.read == RSSM_READ_SHARED_NVFP4;
-  a.hp = take(shared_fp4 ? 0 : units * R * kCols * (c.hp == RSSM_HP_F16_SR ? 2 : 4));
+  const size_t hp_esz = c.hp == RSSM_HP_F16_SR ? 2 : c.hp == RSSM_HP_F8_SR ? 1 : 4;
+  a.hp = take(shared_fp4 ? 0 : units * R * kCols * hp_esz);
+  a.hs = take(!shared_fp4 && c.hp == RSSM_HP_F8_SR ? align_up(units * ((R + 63) / 64), 4) * 4 : 0);
   const bool fp4 = c.read != RSSM_READ_SAME;
   a.rq = take(fp4 ? units * R * kCols / 2 : 0);
   a.rs = take(fp4 ? units * R * kCols / 16 : 0);

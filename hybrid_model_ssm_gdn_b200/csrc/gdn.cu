@@ -92,7 +92,7 @@ constexpr int kBarBytesG = 512;  // mbarriers (29 x 8 B) + armed phases + abort 
 constexpr int kGBG = 3;  // group buffers: the producer loads a unit's group data one unit ahead
 
 // tile source formats
-enum { SRC_F32 = 0, SRC_F16 = 1, SRC_FP4 = 2 };
+enum { SRC_F32 = 0, SRC_F16 = 1, SRC_FP4 = 2, SRC_F8 = 3 };
 
 template <typename TI>
 __device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 consecutive elements
@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   const bool fp4_read = a.read_mode != RSSM_READ_SAME;
   const bool shared_fp4 = a.read_mode == RSSM_READ_SHARED_NVFP4;
   const bool hp16 = a.hp_mode == RSSM_HP_F16_SR;
+  const bool hp8 = a.hp_mode == RSSM_HP_F8_SR;
+  const int hp_fmt = hp16 ? SRC_F16 : hp8 ? SRC_F8 : SRC_F32;  // format of the stored checkpoint
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s) {
@@ -276,8 +278,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       if (S.active) {
         const int n_rec = S.n_ring + S.n_new;
         const bool fold = S.m > 0;
-        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
-                                : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
+        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : hp_fmt)
+                                : (fp4_read ? SRC_FP4 : hp_fmt);
         for (int tt = 0; tt < S.nh * nrb; ++tt, ++ti) {
           const int i = tt / nrb, t = tt % nrb;
           const int rows = min(kFp4Rows, R - kFp4Rows * t);
@@ -292,6 +294,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           uint32_t tb = (uint32_t)n_rec * vrow;
           if (srcfmt == SRC_F32) tb += rows * kCols * 4;
           else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
+          else if (srcfmt == SRC_F8) tb += rows * kCols + 16;
           else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
           if (lane == 0) {
             armed[s] = ti / NS;
@@ -303,14 +306,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
             else if (srcfmt == SRC_F16)
               bulk_g2s(st, reinterpret_cast<const __half *>(a.hp) + row_abs * kCols, rows * kCols * 2, &full[s], pol_stream);
+            else if (srcfmt == SRC_F8)
+              bulk_g2s(st, static_cast<const unsigned char *>(a.hp) + row_abs * kCols, rows * kCols, &full[s], pol_stream);
             else
               bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
           }
           if (lane == 1 && srcfmt == SRC_FP4)
             bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
-          if (lane == 2 && srcfmt == SRC_FP4) {
+          if (lane == 2 && (srcfmt == SRC_FP4 || srcfmt == SRC_F8)) {
             const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
-            bulk_g2s(st + lay.st_g, a.rg + gi4, 16, &full[s], pol_keep);
+            bulk_g2s(st + lay.st_g, (srcfmt == SRC_FP4 ? a.rg : a.hs) + gi4, 16, &full[s], pol_keep);
           }
           if (lane == 3 && S.n_ring)
             bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + S.base_e) * vrow,
@@ -466,8 +471,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         const int me = gh[Q_ME];
         const int n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], slot0 = gh[Q_SLOT0];
         const bool fold = m > 0;
-        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32))
-                                : (fp4_read ? SRC_FP4 : (hp16 ? SRC_F16 : SRC_F32));
+        const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : hp_fmt)
+                                : (fp4_read ? SRC_FP4 : hp_fmt);
         const float *u0t = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_u0);
         const float *cot = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_coef);
         float *amx = reinterpret_cast<float *>(tabs + lay.tb_amax);  // [2 slots][8 warps], table buffer 0
@@ -504,6 +509,13 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.x));
               const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&hv.y));
               return make_float4(f0.x, f0.y, f1.x, f1.y);
+            }
+            if (srcfmt == SRC_F8) {  // E4M3 codes times the tile scale
+              const uint32_t cw = *reinterpret_cast<const uint32_t *>(st + row * kCols + col);
+              return make_float4(__fmul_rn(e4m3_signed_value(cw & 0xFFu), g_tile),
+                                 __fmul_rn(e4m3_signed_value((cw >> 8) & 0xFFu), g_tile),
+                                 __fmul_rn(e4m3_signed_value((cw >> 16) & 0xFFu), g_tile),
+                                 __fmul_rn(e4m3_signed_value(cw >> 24), g_tile));
             }
             const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + col / 2);
             const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + col / 16];
@@ -631,43 +643,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               z += __shfl_xor_sync(0xffffffffu, z, 2);
               if (live && qtr == 0) a.y[(((size_t)b * a.T + j) * a.H + h) * R + rowg] = z;
             }
-            // write the new state in the checkpoint format: each lane puts its values back where it
-            // read them in the stage, then one bulk store per warp moves the warp's rows (contiguous
-            // in shared and in global memory) with full-line writes
-            if (!shared_fp4) {
-              unsigned char *stw = stages + (size_t)s * lay.stage_bytes;
-              if (live) {
-                if (!hp16) {
-#pragma unroll
-                  for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<float4 *>(stw + (row * kCols + qtr * 32 + ((c + lane) & 7) * 4) * 4) = sv[c];
-                } else {
-                  const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
-#pragma unroll
-                  for (int c = 0; c < 8; ++c) {
-                    const int ch = (c + lane) & 7;
-                    const uint32_t elem = (uint32_t)(rowg * kCols + qtr * 32 + ch * 4);
-                    const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
-                    const __half h0v = fp16_sr(sv[c].x, rw.x), h1v = fp16_sr(sv[c].y, rw.y);
-                    const __half h2v = fp16_sr(sv[c].z, rw.z), h3v = fp16_sr(sv[c].w, rw.w);
-                    uint2 pk;
-                    pk.x = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
-                    pk.y = (uint32_t)__half_as_ushort(h2v) | ((uint32_t)__half_as_ushort(h3v) << 16);
-                    *reinterpret_cast<uint2 *>(stw + (row * kCols + qtr * 32 + ch * 4) * 2) = pk;
-                  }
-                }
-              }
-              fence_async_smem();
-              __syncwarp();
-              const int wrows = min(8, rows - row0);
-              if (lane == 0 && wrows > 0) {
-                const int esz_hp = hp16 ? 2 : 4;
-                bulk_s2g(static_cast<unsigned char *>(a.hp) + (unit * R + kFp4Rows * t + row0) * kCols * esz_hp,
-                         stw + row0 * kCols * esz_hp, (uint32_t)(wrows * kCols * esz_hp), pol_wr);
-                bulk_commit();
-              }
-            }
-            if (fp4_read) {
+            // the E4M3 checkpoint and the NVFP4 read copy both scale by the maximum over the
+            // 64-row tile, which spans the eight warps: each posts its rows' maximum, then all read them
+            float tmax = 0.f;
+            if (fp4_read || hp8) {
               float am = 0.f;
 #pragma unroll
               for (int c = 0; c < 8; ++c)
@@ -683,9 +662,60 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                 break;
               }
               ++rdv;
-              float tmax = 0.f;
 #pragma unroll
               for (int w = 0; w < kConsumerWarps; ++w) tmax = fmaxf(tmax, amx[slot * 8 + w]);
+            }
+            // write the new state in the checkpoint format: each lane puts its values back where it
+            // read them in the stage, then one bulk store per warp moves the warp's rows (contiguous
+            // in shared and in global memory) with full-line writes
+            if (!shared_fp4) {
+              unsigned char *stw = stages + (size_t)s * lay.stage_bytes;
+              const uint32_t k0 = (uint32_t)a.seed, k1 = (uint32_t)(a.seed >> 32);
+              const float s8 = fp8_tile_scale(tmax);
+              if (live) {
+                if (hp_fmt == SRC_F32) {
+#pragma unroll
+                  for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4 *>(stw + (row * kCols + qtr * 32 + ((c + lane) & 7) * 4) * 4) = sv[c];
+                } else if (hp16) {
+#pragma unroll
+                  for (int c = 0; c < 8; ++c) {
+                    const int ch = (c + lane) & 7;
+                    const uint32_t elem = (uint32_t)(rowg * kCols + qtr * 32 + ch * 4);
+                    const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
+                    const __half h0v = fp16_sr(sv[c].x, rw.x), h1v = fp16_sr(sv[c].y, rw.y);
+                    const __half h2v = fp16_sr(sv[c].z, rw.z), h3v = fp16_sr(sv[c].w, rw.w);
+                    uint2 pk;
+                    pk.x = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
+                    pk.y = (uint32_t)__half_as_ushort(h2v) | ((uint32_t)__half_as_ushort(h3v) << 16);
+                    *reinterpret_cast<uint2 *>(stw + (row * kCols + qtr * 32 + ch * 4) * 2) = pk;
+                  }
+                } else {
+#pragma unroll
+                  for (int c = 0; c < 8; ++c) {
+                    const int ch = (c + lane) & 7;
+                    const uint32_t elem = (uint32_t)(rowg * kCols + qtr * 32 + ch * 4);
+                    const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, (uint32_t)me, elem >> 2, 0u), k0, k1);
+                    const uint32_t pk = fp8_sr_code(__fdiv_rn(sv[c].x, s8), rw.x) |
+                                        (fp8_sr_code(__fdiv_rn(sv[c].y, s8), rw.y) << 8) |
+                                        (fp8_sr_code(__fdiv_rn(sv[c].z, s8), rw.z) << 16) |
+                                        (fp8_sr_code(__fdiv_rn(sv[c].w, s8), rw.w) << 24);
+                    *reinterpret_cast<uint32_t *>(stw + row * kCols + qtr * 32 + ch * 4) = pk;
+                  }
+                }
+              }
+              if (hp8 && warp == 0 && lane == 0) a.hs[unit * nrb + t] = s8;
+              fence_async_smem();
+              __syncwarp();
+              const int wrows = min(8, rows - row0);
+              if (lane == 0 && wrows > 0) {
+                const int esz_hp = hp16 ? 2 : hp8 ? 1 : 4;
+                bulk_s2g(static_cast<unsigned char *>(a.hp) + (unit * R + kFp4Rows * t + row0) * kCols * esz_hp,
+                         stw + row0 * kCols * esz_hp, (uint32_t)(wrows * kCols * esz_hp), pol_wr);
+                bulk_commit();
+              }
+            }
+            if (fp4_read) {
               const float g = nvfp4_tile_scale(tmax);
               if (warp == 0 && lane == 0) a.rg[unit * nrb + t] = g;
               if (live) {

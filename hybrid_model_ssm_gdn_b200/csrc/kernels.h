@@ -41,7 +41,8 @@ struct GArgs {
   const int4 *meta_in;
   int4 *meta_out;
   int *err;
-  void *hp;                       // fp32 or fp16 [Bt][H][DV][128]
+  void *hp;                       // fp32, fp16 or E4M3 [Bt][H][DV][128]
+  float *hs;                      // E4M3 checkpoint tile scales [Bt][H][ceil(DV/64)]
   unsigned char *rq, *rs;         // NVFP4 codes [Bt][H][DV][64], scales [Bt][H][DV][8]
   float *rg;                      // tile scales [Bt][H][ceil(DV/64)]
   void *ring_k, *ring_v;          // input dtype [Bt][H][2L][128], [Bt][H][2L][DV]
@@ -63,11 +64,12 @@ cudaError_t launch_commit(const int4 *meta_in, int4 *meta_out, const int *accept
 cudaError_t launch_export_meta(const int4 *meta, int *out, int Bt, int L, cudaStream_t stream);
 cudaError_t launch_gather_window(const unsigned char *in, unsigned char *out, const int4 *meta, int Bt, int X,
                                  size_t in_group_bytes, int slot_bytes, int L, cudaStream_t stream);
-cudaError_t launch_store_state(const float *S, void *hp, int hp_mode, unsigned char *rq, unsigned char *rs, float *rg,
-                               int read_mode, int units, int rows, unsigned long long seed, int H,
+cudaError_t launch_store_state(const float *S, void *hp, float *hs, int hp_mode, unsigned char *rq, unsigned char *rs,
+                               float *rg, int read_mode, int units, int rows, unsigned long long seed, int H,
                                cudaStream_t stream);
-cudaError_t launch_widen_state(const void *hp, int hp_mode, const unsigned char *rq, const unsigned char *rs,
-                               const float *rg, int read_mode, float *out, int units, int rows, cudaStream_t stream);
+cudaError_t launch_widen_state(const void *hp, const float *hs, int hp_mode, const unsigned char *rq,
+                               const unsigned char *rs, const float *rg, int read_mode, float *out, int units, int rows,
+                               cudaStream_t stream);
 
 // comparison kernels (conventional step, snapshot-per-draft)
 struct ConvArgs {

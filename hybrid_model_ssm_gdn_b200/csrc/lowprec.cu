@@ -1,6 +1,6 @@
 // lowprec.cu -- stand-alone precision converters: write a loaded fp32 checkpoint in the
-// stored formats (fp32 or fp16 with stochastic rounding at epoch 0, plus the NVFP4 read
-// copy) and widen the stored checkpoint back to fp32 for export.  The rounding rules are
+// stored formats (fp32, fp16 or FP8 E4M3 with stochastic rounding at epoch 0, plus the
+// NVFP4 read copy) and widen the stored checkpoint back to fp32 for export.  The rounding rules are
 // those of lowprec.cuh.  One block of 64 threads per 64-row tile of a head's state;
 // thread r owns row r (128 columns).
 #include "kernels.h"
@@ -10,8 +10,9 @@ namespace rssm {
 
 namespace {
 
-__global__ void store_state_kernel(const float *S, void *hp, int hp_mode, unsigned char *rq, unsigned char *rs,
-                                   float *rg, int read_mode, int rows_per_head, unsigned long long seed) {
+__global__ void store_state_kernel(const float *S, void *hp, float *hs, int hp_mode, unsigned char *rq,
+                                   unsigned char *rs, float *rg, int read_mode, int rows_per_head,
+                                   unsigned long long seed) {
   const int nrb = (rows_per_head + kFp4Rows - 1) / kFp4Rows;
   const size_t unit = blockIdx.x / nrb;
   const int t = blockIdx.x % nrb;
@@ -24,8 +25,27 @@ __global__ void store_state_kernel(const float *S, void *hp, int hp_mode, unsign
   float am = 0.f;
   if (live)
     for (int c = 0; c < kCols; ++c) am = fmaxf(am, fabsf(src[c]));
+  // tile maximum (FP8 checkpoint scale, NVFP4 tile scale)
+  red[row] = am;
+  __syncthreads();
+  float tmax = 0.f;
+  for (int r = 0; r < kFp4Rows; ++r) tmax = fmaxf(tmax, red[r]);
+  const bool fp8 = hp_mode == RSSM_HP_F8_SR && read_mode != RSSM_READ_SHARED_NVFP4;
+  const float s8 = fp8_tile_scale(tmax);
+  if (fp8 && row == 0) hs[unit * nrb + t] = s8;
   if (read_mode != RSSM_READ_SHARED_NVFP4 && live) {
-    if (hp_mode == RSSM_HP_F32) {
+    if (hp_mode == RSSM_HP_F8_SR) {
+      unsigned char *dst = reinterpret_cast<unsigned char *>(hp) + (unit * rows_per_head + rowg) * kCols;
+      for (int c = 0; c < kCols; c += 4) {
+        const uint32_t elem = (uint32_t)(rowg * kCols + c);
+        const uint4 rw = philox4x32_10(make_uint4((uint32_t)unit, 0u, elem >> 2, 0u), (uint32_t)seed,
+                                       (uint32_t)(seed >> 32));
+        dst[c] = (unsigned char)fp8_sr_code(__fdiv_rn(src[c], s8), rw.x);
+        dst[c + 1] = (unsigned char)fp8_sr_code(__fdiv_rn(src[c + 1], s8), rw.y);
+        dst[c + 2] = (unsigned char)fp8_sr_code(__fdiv_rn(src[c + 2], s8), rw.z);
+        dst[c + 3] = (unsigned char)fp8_sr_code(__fdiv_rn(src[c + 3], s8), rw.w);
+      }
+    } else if (hp_mode == RSSM_HP_F32) {
       float *dst = reinterpret_cast<float *>(hp) + (unit * rows_per_head + rowg) * kCols;
       for (int c = 0; c < kCols; ++c) dst[c] = src[c];
     } else {
@@ -42,10 +62,6 @@ __global__ void store_state_kernel(const float *S, void *hp, int hp_mode, unsign
     }
   }
   if (read_mode == RSSM_READ_SAME) return;
-  red[row] = am;
-  __syncthreads();
-  float tmax = 0.f;
-  for (int r = 0; r < kFp4Rows; ++r) tmax = fmaxf(tmax, red[r]);
   const float g = nvfp4_tile_scale(tmax);
   if (row == 0) rg[unit * nrb + t] = g;
   if (!live) return;
@@ -61,8 +77,9 @@ __global__ void store_state_kernel(const float *S, void *hp, int hp_mode, unsign
   }
 }
 
-__global__ void widen_state_kernel(const void *hp, int hp_mode, const unsigned char *rq, const unsigned char *rs,
-                                   const float *rg, int read_mode, float *out, int rows_per_head) {
+__global__ void widen_state_kernel(const void *hp, const float *hs, int hp_mode, const unsigned char *rq,
+                                   const unsigned char *rs, const float *rg, int read_mode, float *out,
+                                   int rows_per_head) {
   const int nrb = (rows_per_head + kFp4Rows - 1) / kFp4Rows;
   const size_t unit = blockIdx.x / nrb;
   const int t = blockIdx.x % nrb;
@@ -83,6 +100,10 @@ __global__ void widen_state_kernel(const void *hp, int hp_mode, const unsigned c
   } else if (hp_mode == RSSM_HP_F16_SR) {
     const __half *src = reinterpret_cast<const __half *>(hp) + r * kCols;
     for (int c = 0; c < kCols; ++c) dst[c] = __half2float(src[c]);
+  } else if (hp_mode == RSSM_HP_F8_SR) {
+    const unsigned char *src = reinterpret_cast<const unsigned char *>(hp) + r * kCols;
+    const float s8 = hs[unit * nrb + t];
+    for (int c = 0; c < kCols; ++c) dst[c] = __fmul_rn(e4m3_signed_value(src[c]), s8);
   } else {
     const float *src = reinterpret_cast<const float *>(hp) + r * kCols;
     for (int c = 0; c < kCols; ++c) dst[c] = src[c];
@@ -91,20 +112,21 @@ __global__ void widen_state_kernel(const void *hp, int hp_mode, const unsigned c
 
 }  // namespace
 
-cudaError_t launch_store_state(const float *S, void *hp, int hp_mode, unsigned char *rq, unsigned char *rs, float *rg,
-                               int read_mode, int units, int rows, unsigned long long seed, int /*H*/,
+cudaError_t launch_store_state(const float *S, void *hp, float *hs, int hp_mode, unsigned char *rq, unsigned char *rs,
+                               float *rg, int read_mode, int units, int rows, unsigned long long seed, int /*H*/,
                                cudaStream_t stream) {
   const int nrb = (rows + kFp4Rows - 1) / kFp4Rows;
-  store_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(S, hp, hp_mode, rq, rs, rg, read_mode,
-                                                                                 rows, seed);
+  store_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(S, hp, hs, hp_mode, rq, rs, rg,
+                                                                                 read_mode, rows, seed);
   return cudaGetLastError();
 }
 
-cudaError_t launch_widen_state(const void *hp, int hp_mode, const unsigned char *rq, const unsigned char *rs,
-                               const float *rg, int read_mode, float *out, int units, int rows, cudaStream_t stream) {
+cudaError_t launch_widen_state(const void *hp, const float *hs, int hp_mode, const unsigned char *rq,
+                               const unsigned char *rs, const float *rg, int read_mode, float *out, int units, int rows,
+                               cudaStream_t stream) {
   const int nrb = (rows + kFp4Rows - 1) / kFp4Rows;
-  widen_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(hp, hp_mode, rq, rs, rg, read_mode, out,
-                                                                                 rows);
+  widen_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(hp, hs, hp_mode, rq, rs, rg, read_mode,
+                                                                                 out, rows);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,9 @@
 //   up to (q+1) u iff r < floor(f * 2^32); keep the sign; saturate at 65504.
 // * E4M3 (OCP FP8 E4M3FN) and E2M1 (OCP FP4): round to nearest, ties to even,
 //   saturating at 448 and 6.
+// * FP8 checkpoint tile (64 rows x 128 columns): s = amax(tile)/448 (1 if amax = 0);
+//   y = x / s rounded stochastically to the E4M3 grid with the FP16 rule and E4M3
+//   spacings (2^(floor(log2|y|)-3), 2^-9 below 2^-6), saturating at 448; value = E4M3 * s.
 // * NVFP4 tile (64 consecutive rows x 128 columns of one head's state), blocks of 16
 //   columns: g = amax(tile)/2688 (1 if amax = 0); s_b = E4M3(amax_b / (6 g));
 //   d_b = s_b g; code = sign | E2M1(|x| / d_b) (all zero if s_b = 0); value = E2M1 * d_b.
@@ -63,6 +66,49 @@ __device__ __forceinline__ __half fp16_sr(float x, uint32_t r) {
   mag = fminf(mag, 65504.f);
   return __float2half_rn(sign ? -mag : mag);          // exact: the value lies on the fp16 grid
 }
+
+// Stochastic rounding of fp32 y to E4M3 with the uniform word r; returns the E4M3 bit pattern
+// (sign bit set only for a non-zero negative result).
+__device__ __forceinline__ uint32_t fp8_sr_code(float y, uint32_t r) {
+  const uint32_t bits = __float_as_uint(y);
+  const uint32_t sign = bits >> 31;
+  const int E = (int)((bits >> 23) & 0xFFu);
+  const uint32_t mant = bits & 0x7FFFFFu;
+  const uint32_t M = E ? (mant | 0x800000u) : mant;  // |y| = M * 2^(Eeff - 150)
+  const int Eeff = E ? E : 1;
+  const int s = max(20, 141 - Eeff);                  // fp32 bits below the E4M3 spacing
+  uint32_t q, F;
+  if (s >= 24) { q = 0; F = M; } else { q = M >> s; F = M & ((1u << s) - 1u); }
+  uint64_t thr;
+  if (s <= 32) thr = (uint64_t)F << (32 - s);
+  else if (s - 32 < 24) thr = (uint64_t)(F >> (s - 32));
+  else thr = 0;
+  const uint32_t up = ((uint64_t)r < thr) ? 1u : 0u;
+  const int ulp_exp = max(Eeff - 127, -6) - 3;
+  const uint32_t n = q + up;                          // magnitude = n * 2^ulp_exp
+  if (n == 0u) return 0u;
+  uint32_t code;
+  if (ulp_exp == -9 && n < 8u) {
+    code = n;                                         // subnormal: mantissa n, exponent field 0
+  } else {
+    // normalise n * 2^ulp_exp (n <= 16) to (8 + m) * 2^(ef - 10)
+    int ef = ulp_exp + 10;
+    uint32_t mm = n;
+    if (mm >= 16u) { mm >>= 1; ++ef; }                 // n = 16: carried into the next binade
+    code = ((uint32_t)ef << 3) | (mm - 8u);
+    if (code > 0x7Eu) code = 0x7Eu;                   // saturate at 448
+  }
+  return code | (sign << 7);
+}
+
+__device__ __forceinline__ float e4m3_signed_value(uint32_t code) {
+  const uint32_t ef = (code >> 3) & 0xFu, m = code & 7u;
+  const float mag = ef == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8u + m), (int)ef - 10);
+  return (code & 0x80u) ? -mag : mag;
+}
+
+// FP8 checkpoint tile scale from the tile's largest magnitude.
+__device__ __forceinline__ float fp8_tile_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f; }
 
 // E4M3FN round-to-nearest-even of v >= 0, saturating at 448 (value, not code).
 __device__ __forceinline__ float e4m3_round(float v) {

@@ -75,8 +75,11 @@ enum {
 
 typedef enum { RSSM_MAMBA2 = 0, RSSM_GDN = 1 } rssm_kind;
 typedef enum { RSSM_F32 = 0, RSSM_BF16 = 1 } rssm_dtype;
-/* precision of the recurrence checkpoint ([HMD] Interpretation 4th paragraph, Perspective 2nd) */
-typedef enum { RSSM_HP_F32 = 0, RSSM_HP_F16_SR = 1 } rssm_hp;
+/* precision of the recurrence checkpoint ([HMD] Interpretation 4th paragraph, Perspective 2nd;
+ * FP8: [SSD] Interpretation 3rd paragraph): fp32; fp16 with stochastic rounding; or E4M3 (FP8)
+ * times one fp32 scale amax/448 per 64-row tile of a head's state, rounded stochastically with
+ * the same random words (GDN only) */
+typedef enum { RSSM_HP_F32 = 0, RSSM_HP_F16_SR = 1, RSSM_HP_F8_SR = 2 } rssm_hp;
 /* copy read for outputs: the checkpoint itself, a separate NVFP4 copy, or (contrast
  * only) one NVFP4 copy that is also the checkpoint the recurrence continues from */
 typedef enum { RSSM_READ_SAME = 0, RSSM_READ_NVFP4 = 1, RSSM_READ_SHARED_NVFP4 = 2 } rssm_read;

@@ -47,6 +47,22 @@ def test_gdn_traffic_model_window():
     assert tot < (wl.window + 1) * state * 1.2
 
 
+def test_gdn_traffic_by_format():
+    """Plain steps read the checkpoint in its own format, or the NVFP4 copy; a fold reads the checkpoint and
+    writes it and the copy.  E4M3 is a quarter of fp32 plus one fp32 scale per 64 x 128 tile."""
+    wl = GDN_B256
+    elems = wl.batch * wl.nheads * wl.dv * wl.dk
+    rest = bench.gdn_traffic(wl, 3) - elems * 4
+    assert bench.gdn_traffic(wl, 3, "f8sr", "same") == rest + elems + elems // (64 * 128) * 4
+    assert bench.gdn_traffic(wl, 3, "f16sr", "nvfp4") == rest + elems * (0.5 + 1 / 16) + elems // (64 * 128) * 4
+    fold = wl.window - 1
+    rest_f = bench.gdn_traffic(wl, fold) - 2 * elems * 4
+    f8 = elems + elems // (64 * 128) * 4
+    fp4 = elems * (0.5 + 1 / 16) + elems // (64 * 128) * 4
+    assert bench.gdn_traffic(wl, fold, "f8sr", "nvfp4") == rest_f + 2 * f8 + fp4
+    assert bench.gdn_traffic(wl, fold, "f32", "shared_nvfp4") == rest_f + 2 * fp4
+
+
 def test_committed_profile_matches_kernel_source():
     """The committed ncu summary of the headline kernel was taken on the present kernel code, so the bench
     line reports its measured DRAM traffic (a kernel change without a new capture fails here)."""

@@ -62,6 +62,8 @@ def test_drift_modes_and_window_sweep(cuda_ok):
         "fp32_hp+nvfp4_read": ("f32", "nvfp4", 16),
         "fp16sr_hp+nvfp4_read": ("f16sr", "nvfp4", 16),
         "fp16sr_hp": ("f16sr", "same", 16),
+        "fp8sr_hp": ("f8sr", "same", 16),
+        "fp8sr_hp+nvfp4_read": ("f8sr", "nvfp4", 16),
         "shared_nvfp4": ("f32", "shared_nvfp4", 16),
         "fp32_hp+nvfp4_read_L4": ("f32", "nvfp4", 4),
         "fp32_hp+nvfp4_read_L8": ("f32", "nvfp4", 8),

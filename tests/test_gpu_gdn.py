@@ -113,10 +113,12 @@ def _edge_state(shape, seed):
     S[0, 0, 5, :16] = 0.0                                        # a zero block
     S[0, 1, 7, :4] = [65504.0, -70000.0, 3e-6, -1e-8]            # saturation, fp16 subnormals
     S[0, 1, 9] = np.float16(0.125).astype(np.float32)            # on the fp16 grid
+    S[1, 2, 64:] = 0.0                                           # an all-zero 64-row tile (scale 1)
     return S
 
 
-@pytest.mark.parametrize("hp,read", [("f16sr", "nvfp4"), ("f32", "shared_nvfp4"), ("f16sr", "same")])
+@pytest.mark.parametrize("hp,read", [("f16sr", "nvfp4"), ("f32", "shared_nvfp4"), ("f16sr", "same"),
+                                     ("f8sr", "same"), ("f8sr", "nvfp4")])
 def test_load_converters_bit_exact(cuda_ok, hp, read):
     wl = SMALL.replace(batch=2, nheads=3, dv=128)
     S = _edge_state((2, 3, 128, 128), 1)
@@ -124,10 +126,12 @@ def test_load_converters_bit_exact(cuda_ok, hp, read):
     ex = p.gpu.export(state=True, ring=False)["S"].cpu().numpy()
     if read == "shared_nvfp4":
         np.testing.assert_array_equal(ex, lp.nvfp4_roundtrip_state(S))
-    elif hp == "f16sr":
+    elif hp in ("f16sr", "f8sr"):
         units = (np.arange(2)[:, None] * 3 + np.arange(3)[None, :])
         words = sr_words(0xABCDEF0123456789, units, 0, 128 * 128).reshape(2, 3, 128, 128)
-        np.testing.assert_array_equal(ex, lp.fp16_stochastic_round(S, words).astype(np.float32))
+        want = (lp.fp16_stochastic_round(S, words).astype(np.float32) if hp == "f16sr"
+                else lp.fp8_quantize_state(S, words)["values"])
+        np.testing.assert_array_equal(ex, want)
     if read != "same":
         rc = p.gpu.export_read_copy()
         q = lp.nvfp4_quantize_state(S)
@@ -149,7 +153,8 @@ TOL_FLIP = 2e-2
 FLIP_FRACTION = 0.02
 
 
-@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f16sr", "same"), ("f32", "shared_nvfp4")])
+@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f16sr", "same"), ("f32", "shared_nvfp4"),
+                                     ("f8sr", "same"), ("f8sr", "nvfp4")])
 def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
     """With stochastic rounding the oracle's trajectory is one sample among many, so the GPU is held to
     the spread between two oracle seeds (mean error at most twice the seed-to-seed mean, plus the fp32
@@ -158,7 +163,7 @@ def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
     wl = GDN_LOWPREC.replace(batch=4, nheads=4, window=8)
     p = Pair(wl, hp=hp, read=read, seed=7)
     other = None
-    if hp == "f16sr":
+    if hp in ("f16sr", "f8sr"):
         from synth import gdn_initial_state
         other = ReplayOracle("gdn", gdn_initial_state(wl), wl.window, nheads=wl.nheads, hp=hp, read=read, seed=8)
     errs, spread = [], []
@@ -183,9 +188,9 @@ def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
         assert frac <= FLIP_FRACTION
 
 
-@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "same")])
+@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "same"), ("f8sr", "nvfp4")])
 def test_verify_lowprec_modes(cuda_ok, hp, read):
-    """8-draft verify reading an NVFP4 copy or an fp16 checkpoint against the method-mirroring oracle, with the
+    """8-draft verify reading an NVFP4 copy, an fp16 or an E4M3 checkpoint against the method-mirroring oracle, with the
     flip-aware bound of the step test."""
     wl = GDN_LOWPREC.replace(batch=3, nheads=4, window=8)
     p = Pair(wl, hp=hp, read=read, seed=7, max_draft=8)
