@@ -51,6 +51,20 @@ fp32 fold result at every fold) or "shared_nvfp4" (the NVFP4 copy is also the
 checkpoint the recurrence continues from; contrast mode).  The NVFP4 copy is
 quantised tile by tile, a tile being 64 consecutive rows of one head's state.
 
+Decay-aware read skipping (GDN, ``skip_tau`` > 0): a head whose gates over
+the buffered inputs have multiplied down below a threshold may skip reading
+the checkpoint, which then counts as zero; a fold of such a head writes the
+new checkpoint from the buffer alone ("SSM decoding stops writing state every
+step", Perspective, first paragraph, names this as the next step and fixes
+no rule).  Reading taken: after each step, verify or flush, a head's flag is
+set iff the product of alpha over the committed records of the current
+window, taken in fp32 in record order, is below ``skip_tau``; the next call
+reads that flag.  The product only falls as records are added, so the
+skipped term S0 u0 of any later output has norm at most
+skip_tau * ||S0|| * q_scale * ||q|| (each (I - beta k k^T) has norm <= 1 for
+||k|| = 1, 0 <= beta <= 2).  Commit leaves the flags alone; a fold that empties
+the window clears them.
+
 Two outputs are produced per call: ``y`` mirrors the method (folds at the
 points above, state rounded to its stored formats, replay in float64) and
 ``y_true`` is conventional step-by-step decoding in float64 with no rounding
@@ -82,8 +96,9 @@ class ReplayOracle:
     """
 
     def __init__(self, kind, S0, window, *, nheads, ngroups=1, params=None, seq_ids=None, head_ids=None,
-                 hp="f32", read="same", seed=0, q_scale=1.0):
+                 hp="f32", read="same", seed=0, q_scale=1.0, skip_tau=0.0):
         assert kind in ("mamba2", "gdn")
+        assert skip_tau >= 0 and (skip_tau == 0 or kind == "gdn")
         assert hp in ("f32", "f16sr", "f8sr") and read in ("same", "nvfp4", "shared_nvfp4")
         self.kind, self.L, self.H, self.G = kind, int(window), int(nheads), int(ngroups)
         S0 = np.asarray(S0, np.float64)
@@ -99,6 +114,7 @@ class ReplayOracle:
             self.D = np.asarray(self.params["D"], np.float64)[self.head_ids]
         self.q_scale = float(q_scale)
         self.hp_mode, self.read_mode, self.seed = hp, read, int(seed)
+        self.skip_tau = np.float32(skip_tau)
 
         self.S_true = S0.copy()
         self.count = np.zeros(self.nb, np.int64)
@@ -109,6 +125,7 @@ class ReplayOracle:
         for b in range(self.nb):
             self._store(b, S0[b])
         self.pending = np.zeros(self.nb, np.int64)
+        self.skip = np.zeros((self.nb, self.nh), bool)       # decay-aware skip flags, read by the next call
         self.err = None                      # (seq, code) of the lowest failing sequence
         self.ring = [[None] * self.L for _ in range(self.nb)]   # per sequence, per slot: record dict
         self._drafts_true = [None] * self.nb                    # truth-side draft records awaiting commit
@@ -145,6 +162,21 @@ class ReplayOracle:
         if self.kind == "mamba2":
             return rc.mamba2_step(S, rec["x"], rec["B"], rec["C"], rec["dt"], self.A, self.D, self.head_group)
         return rc.gdn_step(S, rec["q"], rec["k"], rec["v"], rec["alpha"], rec["beta"], self.q_scale)
+
+    def _ckpt(self, S, b):
+        """The checkpoint as a call reads it: heads flagged for skipping contribute zero."""
+        if not self.skip[b].any():
+            return S
+        return np.where(self.skip[b][:, None, None], 0.0, S)
+
+    def _update_skip(self, b):
+        """Flags for the next call: fp32 product of alpha over the committed records, in order, < skip_tau."""
+        if self.skip_tau <= 0:
+            return
+        prod = np.ones(self.nh, np.float32)
+        for rec in self.ring[b][: self.count[b]]:
+            prod = (prod * np.asarray(rec["alpha"], np.float32)).astype(np.float32)
+        self.skip[b] = prod < self.skip_tau
 
     def _read_copy(self, S32):
         return lowprec.nvfp4_roundtrip_state(S32).astype(np.float64)
@@ -185,14 +217,14 @@ class ReplayOracle:
             rec = self._select(inp, b)
             self.S_true[b], y_true[b] = self._true_step(self.S_true[b], rec)
             folded = False
-            S = self.rd[b]
+            S = self._ckpt(self.rd[b], b)
             if self.count[b] == self.L:                               # pre-fold (after a commit)
-                S = self._fold(self.hp[b], self.ring[b][: self.L])
+                S = self._fold(self._ckpt(self.hp[b], b), self.ring[b][: self.L])
                 self.count[b] = 0
                 self.epoch[b] += 1
                 folded = True
             elif self.count[b] + 1 == self.L:
-                S = self.hp[b]
+                S = self._ckpt(self.hp[b], b)
             self.ring[b][self.count[b]] = rec
             self.count[b] += 1
             if self.count[b] == self.L:                               # eager fold
@@ -205,6 +237,7 @@ class ReplayOracle:
                 y[b] = self._replay(S, self.ring[b][: self.count[b]], rec)
             if folded:
                 self._store(b, S)
+            self._update_skip(b)
         return y, y_true
 
     def verify(self, T, inp):
@@ -217,9 +250,9 @@ class ReplayOracle:
             if self.pending[b]:
                 self._error(b, ERR_PENDING)
                 continue
-            S = self.rd[b]
+            S = self._ckpt(self.rd[b], b)
             if self.count[b] + T > self.L:                            # make room: fold committed records
-                S = self._fold(self.hp[b], self.ring[b][: self.count[b]])
+                S = self._fold(self._ckpt(self.hp[b], b), self.ring[b][: self.count[b]])
                 self.count[b] = 0
                 self.epoch[b] += 1
                 self._store(b, S)
@@ -233,6 +266,7 @@ class ReplayOracle:
                 St, y_true[b, j] = self._true_step(St, recs[j])
             self._drafts_true[b] = recs
             self.pending[b] = T
+            self._update_skip(b)
         return y, y_true
 
     def commit(self, accepted):
@@ -259,10 +293,11 @@ class ReplayOracle:
                 self._error(b, ERR_PENDING)
                 continue
             if self.count[b]:
-                S = self._fold(self.hp[b], self.ring[b][: self.count[b]])
+                S = self._fold(self._ckpt(self.hp[b], b), self.ring[b][: self.count[b]])
                 self.count[b] = 0
                 self.epoch[b] += 1
                 self._store(b, S)
+                self._update_skip(b)
 
     # ------------------------------------------------------------------ inspection
     def live_slots(self, b):

@@ -191,3 +191,77 @@ def test_fp8_checkpoint_tiles_and_separate_read_copy():
         below = grid[np.clip(np.searchsorted(grid, y) - 1, 0, len(grid) - 1)]
         dist = np.minimum(np.abs(nearest - y), np.abs(below - y))
         assert np.all(dist <= 1e-5 * np.maximum(y, 2.0 ** -9))
+
+
+# ------------------------------------------------------------------------------------ decay-aware skipping
+
+def _halving_inputs(t, zero_alpha_at=None):
+    """GDN step inputs with alpha = 1/2 for every head (products exact in fp32); optionally alpha = 0 once."""
+    inp = gdn_step_inputs(G_WL, t)
+    inp["alpha"] = np.full_like(inp["alpha"], 0.5 if t != zero_alpha_at else 0.0)
+    return inp
+
+
+def test_skip_flags_follow_the_gate_product_and_bound_the_dropped_term():
+    """alpha = 1/2 makes the product over n committed records exactly 2^-n, so with tau = 1.5 * 2^-5 a head is
+    flagged exactly when 5 or more records are committed, and a fold clears it.  Within the first window the
+    skipping oracle differs from the non-skipping one only on calls that read a set flag, and there by at most
+    tau * ||S0|| * q_scale * ||q|| per head (the whole dropped term S0 u0)."""
+    L, tau = 8, 1.5 * 2.0 ** -5
+    sk, ref = _gdn(L, skip_tau=tau), _gdn(L)
+    S0 = gdn_initial_state(G_WL)
+    for t in range(2 * L + 3):
+        inp = _halving_inputs(t)
+        before = sk.skip.copy()
+        y, _ = sk.step(inp)
+        y0, _ = ref.step(inp)
+        n = (t + 1) % L
+        np.testing.assert_array_equal(sk.skip, np.full((G_WL.batch, G_WL.nheads), n >= 5))
+        if t < L - 1:                                   # same checkpoint on both sides until the first fold
+            d = np.linalg.norm(y - y0, axis=-1)
+            bound = tau * np.linalg.norm(S0, axis=(-2, -1)) * np.linalg.norm(inp["q"], axis=-1)
+            assert np.all(d[~before] == 0)
+            assert np.all(d[before] <= bound[before] * (1 + 1e-9))
+            assert np.all(d[before] > 0)
+
+
+def test_skip_with_a_zero_gate_changes_nothing():
+    """With alpha = 0 at some token the checkpoint's true contribution after it is exactly zero, so skipping
+    it (and writing the next checkpoint from the buffer alone) gives the non-skipping oracle's results
+    exactly: the skip removes the checkpoint term and nothing else, head by head."""
+    L = 8
+    sk, ref = _gdn(L, skip_tau=1e-3), _gdn(L)
+    for t in range(3 * L):
+        inp = gdn_step_inputs(G_WL, t)
+        if t % L == 2:
+            inp["alpha"][:, 1] = 0.0                    # head 1 only
+        y, _ = sk.step(inp)
+        y0, _ = ref.step(inp)
+        np.testing.assert_array_equal(y, y0)
+        assert not sk.skip[:, 0].any()
+        np.testing.assert_array_equal(sk.skip[:, 1], (t % L) >= 2 and (t % L) != L - 1)
+    np.testing.assert_array_equal(sk.hp, ref.hp)
+
+
+def test_skip_flags_under_verify_commit_and_flush():
+    """Verify reads the flags but sets them from the committed records only (drafts excluded); commit leaves
+    them; a pre-fold or a flush clears them."""
+    L, tau = 8, 1.5 * 2.0 ** -5
+    o = _gdn(L, skip_tau=tau)
+    for t in range(6):
+        o.step(_halving_inputs(t))
+    assert o.skip.all()                                 # 6 records: 2^-6 < tau
+    drafts = gdn_draft_inputs(G_WL, 0, 2)
+    drafts["alpha"] = np.full_like(drafts["alpha"], 0.5)
+    o.verify(2, drafts)                                 # 6 + 2 <= 8: no pre-fold
+    assert o.skip.all()
+    o.commit(np.full(G_WL.batch, 2))
+    assert o.skip.all() and (o.count == 8).all()
+    o.verify(2, drafts)                                 # 8 + 2 > 8: pre-fold, nothing committed after it
+    assert not o.skip.any()
+    o.commit(np.zeros(G_WL.batch, np.int64))
+    for t in range(5):
+        o.step(_halving_inputs(10 + t))
+    assert o.skip.all()
+    o.flush()
+    assert not o.skip.any() and (o.count == 0).all()
