@@ -576,6 +576,52 @@ def precision_section(windows_timed: int = 4) -> dict:
     return out
 
 
+def skip_section(windows_timed: int = 8, tau: float = 1e-2) -> dict:
+    """GDN layer (batch 256, 32 heads, d 128, L 16) with fast-decaying gates (alpha = exp(-0.6 softplus(z)),
+    about 0.6 on average): decay-aware read skipping off and on.  The skip pattern repeats every window (the
+    inputs cycle with period L), so one untimed window of flag exports gives the skipped fraction of the
+    timed steps; the byte count leaves out the skipped heads' checkpoint reads."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM
+    wl, dev, bf = GDN_B256.replace(decay_scale=0.6), torch.device("cuda"), torch.bfloat16
+    L = wl.window
+    S0 = torch.from_numpy(gdn_initial_state(wl)).to(dev)
+    pool = []
+    for t in range(L):
+        inp = gdn_step_inputs(wl, t)
+        pool.append({k: torch.from_numpy(v).to(dev).to(torch.float32 if k in ("alpha", "beta") else bf)
+                     for k, v in inp.items()})
+    y = torch.empty(wl.batch, wl.nheads, wl.dv, device=dev)
+    stream = torch.cuda.current_stream()
+    head_bytes = wl.dv * wl.dk * 4
+    out = {"workload": "gdn replay decode, batch 256, 32 heads, d 128, L 16, bf16 inputs, fp32 checkpoint, "
+                       "gates alpha = exp(-0.6 softplus(z))", "tau": tau}
+    for name, t in (("off", 0.0), ("on", tau)):
+        layer = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, wl.dk, 1, L, 0, bf, skip_tau=t)
+        layer.load_checkpoint(S0)
+
+        def step(i):
+            p = pool[i % L]
+            layer.gdn_step(p["q"], p["k"], p["v"], p["alpha"], p["beta"], y)
+
+        for i in range(2 * L):
+            step(i)
+        skipped = []  # heads skipping their read at each position of the window
+        for i in range(L):
+            skipped.append(int(layer.export_skip().sum().item()) if t > 0 else 0)
+            step(i)
+        K = L * windows_timed
+        ms = timed(step, K, stream)
+        nbytes = sum(gdn_traffic(wl, i) - skipped[i] * head_bytes for i in range(L)) / L
+        out[name] = {"ms_per_step": ms, "tokens_per_s": wl.batch / (ms * 1e-3), "bytes_per_step": nbytes,
+                     "GBps": nbytes / (ms * 1e-3) / 1e9,
+                     "skipped_fraction": sum(skipped) / (L * wl.batch * wl.nheads), "device_error": layer.get_error()}
+        del layer
+    out["speedup"] = out["off"]["ms_per_step"] / out["on"]["ms_per_step"]
+    return out
+
+
 def verify_section(rounds: int, kinds=("mamba2", "gdn")) -> dict:
     """Speculative verify + commit (T = 4, 8) vs snapshot-per-draft: the Mamba-2 shape at batch 512 and the
     Gated DeltaNet layer at batch 256."""
@@ -731,9 +777,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-extra", action="store_true", help="skip the GDN, speculative-verify and precision sections")
+    ap.add_argument("--no-extra", action="store_true", help="skip the GDN, speculative-verify, precision and read-skipping sections")
     ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch",
-                                                  "precision"], default=None,
+                                                  "precision", "skip"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -753,7 +799,8 @@ def main():
                    verify_section(args.steps) if args.only == "verify" else
                    verify_section(args.steps, (args.only.split("-")[1],)) if args.only.startswith("verify-") else
                    batch_section() if args.only == "batch" else
-                   precision_section() if args.only == "precision" else window_section())
+                   precision_section() if args.only == "precision" else
+                   skip_section() if args.only == "skip" else window_section())
             print(json.dumps(out))
         return
 
@@ -767,6 +814,7 @@ def main():
         res["gdn"] = gdn_section(min(args.steps, 1024))
         res["verify"] = verify_section(512)
         res["precision"] = precision_section()
+        res["skip"] = skip_section()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:

@@ -44,11 +44,13 @@ def _dev(t, dtype, name):
 
 
 def make_config(kind, batch, nheads, headdim, dstate=128, ngroups=1, window=16, max_draft=0,
-                in_dtype=torch.bfloat16, hp="f32", read="same", seed=0, q_scale=1.0, A=None, D=None) -> abi.Config:
+                in_dtype=torch.bfloat16, hp="f32", read="same", seed=0, q_scale=1.0, A=None, D=None,
+                skip_tau=0.0) -> abi.Config:
     return abi.Config(kind={"mamba2": abi.MAMBA2, "gdn": abi.GDN}[kind], batch=batch, nheads=nheads,
                       headdim=headdim, dstate=dstate, ngroups=ngroups, window=window, max_draft=max_draft,
                       in_dtype=_DT[in_dtype], hp=_HP[hp], read=_READ[read], seed=seed, q_scale=q_scale,
-                      A=None if A is None else A.data_ptr(), D=None if D is None else D.data_ptr())
+                      A=None if A is None else A.data_ptr(), D=None if D is None else D.data_ptr(),
+                      skip_tau=skip_tau)
 
 
 class ReplaySSM:
@@ -56,7 +58,7 @@ class ReplaySSM:
 
     def __init__(self, kind, batch, nheads, headdim, dstate=128, ngroups=1, window=16, max_draft=0,
                  in_dtype=torch.bfloat16, hp="f32", read="same", seed=0, q_scale=1.0, A=None, D=None,
-                 device=None):
+                 device=None, skip_tau=0.0):
         self.lib = abi.load()
         self.kind, self.batch, self.nheads, self.headdim = kind, batch, nheads, headdim
         self.ngroups, self.window, self.max_draft, self.in_dtype = ngroups, window, max_draft, in_dtype
@@ -67,7 +69,7 @@ class ReplaySSM:
         else:
             self.A = self.D = None
         self.cfg = make_config(kind, batch, nheads, headdim, dstate, ngroups, window, max_draft, in_dtype, hp, read,
-                               seed, q_scale, self.A, self.D)
+                               seed, q_scale, self.A, self.D, skip_tau)
         nbytes = C.c_size_t()
         abi.check(self.lib.rssm_arena_bytes(C.byref(self.cfg), C.byref(nbytes)), "rssm_arena_bytes")
         self.arena_bytes = nbytes.value
@@ -164,6 +166,12 @@ class ReplaySSM:
         abi.check(self.lib.rssm_export_read_copy(self.handle, _ptr(codes), _ptr(scales), _ptr(g), _stream()),
                   "rssm_export_read_copy")
         return {"packed": codes, "scales": scales, "g": g}
+
+    def export_skip(self):
+        """Decay-aware skip flags uint8 [Bt][H] (1 = the next call skips that head's checkpoint read)."""
+        flags = torch.empty(self.batch, self.nheads, dtype=torch.uint8, device=self.device)
+        abi.check(self.lib.rssm_export_skip(self.handle, _ptr(flags), _stream()), "rssm_export_skip")
+        return flags
 
     def get_error(self):
         """(code, seq) of the sticky device error word; synchronises the current stream."""

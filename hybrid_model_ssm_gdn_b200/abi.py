@@ -26,7 +26,7 @@ class Config(C.Structure):
     _fields_ = [("kind", C.c_int), ("batch", C.c_int), ("nheads", C.c_int), ("headdim", C.c_int),
                 ("dstate", C.c_int), ("ngroups", C.c_int), ("window", C.c_int), ("max_draft", C.c_int),
                 ("in_dtype", C.c_int), ("hp", C.c_int), ("read", C.c_int), ("seed", C.c_ulonglong),
-                ("q_scale", C.c_float), ("A", C.c_void_p), ("D", C.c_void_p)]
+                ("q_scale", C.c_float), ("A", C.c_void_p), ("D", C.c_void_p), ("skip_tau", C.c_float)]
 
 
 class Tokens(C.Structure):
@@ -55,6 +55,7 @@ _SIGS = {
     "rssm_flush": [_P, _P, _P],
     "rssm_export": [_P, _P, _P, _P, _P],
     "rssm_export_read_copy": [_P, _P, _P, _P, _P],
+    "rssm_export_skip": [_P, _P, _P],
     "rssm_get_error": [_P, C.POINTER(C.c_int), C.POINTER(C.c_int), _P],
     "rssm_conv_mamba2_step": [C.POINTER(Config), _P, _P, _P, _P, _P, _P, _P],
     "rssm_conv_gdn_step": [C.POINTER(Config), _P, _P, _P, _P, _P, _P, _P, _P],

@@ -41,6 +41,7 @@ rssm_status validate(const rssm_config *c) {
   if (c->in_dtype != RSSM_F32 && c->in_dtype != RSSM_BF16) return RSSM_ERR_ARG;
   if (c->hp != RSSM_HP_F32 && c->hp != RSSM_HP_F16_SR && c->hp != RSSM_HP_F8_SR) return RSSM_ERR_ARG;
   if (c->read < RSSM_READ_SAME || c->read > RSSM_READ_SHARED_NVFP4) return RSSM_ERR_ARG;
+  if (!(c->skip_tau >= 0.f) || c->skip_tau > 3.0e38f) return RSSM_ERR_ARG;  // NaN, negative or infinite
   if (c->batch < 1 || c->nheads < 1) return RSSM_ERR_SHAPE;
   if ((long long)c->batch * c->nheads > (1LL << 26)) return RSSM_ERR_SHAPE;
   if (c->dstate != kCols) return RSSM_ERR_SHAPE;
@@ -52,7 +53,7 @@ rssm_status validate(const rssm_config *c) {
     if (c->headdim > 64) return RSSM_ERR_SHAPE;
     if (c->ngroups < 1 || c->nheads % c->ngroups != 0) return RSSM_ERR_SHAPE;
     if (!c->A || !c->D) return RSSM_ERR_ARG;
-    if (c->hp != RSSM_HP_F32 || c->read != RSSM_READ_SAME) return RSSM_ERR_UNSUPPORTED;
+    if (c->hp != RSSM_HP_F32 || c->read != RSSM_READ_SAME || c->skip_tau != 0.f) return RSSM_ERR_UNSUPPORTED;
   } else {
     if (c->headdim > 128) return RSSM_ERR_SHAPE;
     if (c->ngroups != 1) return RSSM_ERR_SHAPE;
@@ -107,6 +108,8 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   a.ring_k = x->arena + x->lay.ring_a; a.ring_v = x->arena + x->lay.ring_b;
   a.ring_a = reinterpret_cast<float *>(x->arena + x->lay.ring_c);
   a.ring_b = reinterpret_cast<float *>(x->arena + x->lay.ring_d);
+  a.skip = c.skip_tau > 0.f ? x->arena + x->lay.skip : nullptr;
+  a.skip_tau = c.skip_tau;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.mask = mask; a.y = y;
   cudaError_t e = launch_gdn_replay(a, esz, stream);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -304,6 +307,15 @@ rssm_status rssm_export_read_copy(rssm_ctx *x, unsigned char *codes, unsigned ch
                         cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return RSSM_OK;
+}
+
+rssm_status rssm_export_skip(rssm_ctx *x, unsigned char *flags, rssm_stream stream) {
+  if (!x || !flags) return RSSM_ERR_ARG;
+  if (!x->loaded || x->cfg.skip_tau == 0.f) return RSSM_ERR_UNSUPPORTED;
+  const size_t units = (size_t)x->cfg.batch * x->cfg.nheads;
+  cudaError_t e = cudaMemcpyAsync(flags, x->arena + x->lay.skip, units, cudaMemcpyDeviceToDevice,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RSSM_OK : cuda_fail(e);
 }
 
 rssm_status rssm_get_error(rssm_ctx *x, int *code, int *seq, rssm_stream stream) {

@@ -48,6 +48,7 @@ struct ArenaLayout {
   size_t ring_b;   // Mamba-2 B [Bt][G][2L][128] / GDN v [Bt][H][2L][d_v] (input dtype)
   size_t ring_c;   // Mamba-2 dt / GDN alpha: fp32 [Bt][H][dt_stride(L)]
   size_t ring_d;   // GDN beta: fp32 [Bt][H][dt_stride(L)]
+  size_t skip;     // GDN decay-aware skip flags u8 [Bt][H] (only with skip_tau > 0)
   size_t total;
 };
 
@@ -80,6 +81,7 @@ inline ArenaLayout make_layout(const rssm_config &c) {
     a.ring_c = take(units * dt_stride(c.window) * 4);
     a.ring_d = take(units * dt_stride(c.window) * 4);
   }
+  a.skip = take(c.kind == RSSM_GDN && c.skip_tau > 0.f ? units : 0);
   a.total = off;
   return a;
 }

@@ -14,11 +14,18 @@
 //     s <- alpha_r s + beta_r (v_r[row] - alpha_r (s . k_r)) k_r.
 //
 // Precision modes ("Hybrid-model decoding has a new bottleneck", Interpretation, fourth
-// paragraph, Perspective, second paragraph): the checkpoint is fp32 or fp16 written with
-// stochastic rounding; the copy read by non-fold outputs is the checkpoint itself, a
-// separate NVFP4 copy re-quantised from the fp32 fold result, or (contrast) an NVFP4 copy
-// that is also the state the recurrence continues from.  Outputs of a call that folds
-// come from the fp32 fold result.
+// paragraph, Perspective, second paragraph; FP8: "SSM decoding stops writing state every
+// step", Interpretation, third paragraph): the checkpoint is fp32, fp16 written with
+// stochastic rounding, or E4M3 times a per-tile fp32 scale written the same way; the copy
+// read by non-fold outputs is the checkpoint itself, a separate NVFP4 copy re-quantised
+// from the fp32 fold result, or (contrast) an NVFP4 copy that is also the state the
+// recurrence continues from.  Outputs of a call that folds come from the fp32 fold result.
+//
+// Decay-aware read skipping ("SSM decoding stops writing state every step", Perspective,
+// first paragraph): with a threshold tau > 0, a head whose alpha product over the
+// committed records of its window is below tau (fp32, record order; decided by the prep
+// warps at the end of a call) skips the next call's checkpoint read: no tile copy, a zero
+// term, and a fold from zero.
 //
 // Block roles (one block per SM, persistent; units drawn from a per-launch counter):
 //  * producer warp: TMA bulk copies (cp.async.bulk) of each unit's k records, q and
@@ -33,9 +40,9 @@
 //    owns columns 4l..4l+3, the row dot products with u_0 and the buffered term finish in
 //    one warp transpose reduction.  Fold tiles: four lanes own one row (32 columns each,
 //    in registers) and run the sequential row update with two shuffles per record; then
-//    the new state is written in the checkpoint format and, in NVFP4 modes, quantised
-//    (tile maximum over the eight warps through an mbarrier rendezvous with bounded
-//    waits).
+//    the new state is written in the checkpoint format and, in E4M3 and NVFP4 modes,
+//    quantised (tile maximum over the eight warps through an mbarrier rendezvous with
+//    bounded waits).
 // Work unit: (sequence, chunk of HG heads), HG = 4, 4, 2, 1 for 1, 2, 4, 8 outputs.
 #include "common.cuh"
 #include "kernels.h"
@@ -48,7 +55,7 @@ namespace {
 constexpr int kGHdrBytes = 1024;
 enum {
   Q_ACTIVE = 0, Q_NREC, Q_M, Q_NRING, Q_NNEW, Q_TOUT, Q_SLOT0, Q_MC, Q_ME, Q_MP, Q_B, Q_H0, Q_NH, Q_BASE,
-  Q_WMETA, Q_END,
+  Q_WMETA, Q_SKIP, Q_END,  // Q_SKIP: bit i set = head h0 + i skips its checkpoint read in this call
   Q_F = 32,                // floats: alpha of new tokens [8][8] (token, head)
   Q_FB = Q_F + 64          // beta of new tokens [8][8]
 };
@@ -103,7 +110,9 @@ __device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 c
   }
 }
 
-template <typename TI, int NO>
+// LP: the context stores a low-precision checkpoint or keeps an NVFP4 read copy.  LP = false
+// compiles the fp32-checkpoint path alone, with every format branch folded away.
+template <typename TI, int NO, bool LP>
 __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int esz = sizeof(TI);
@@ -126,10 +135,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunks = (a.H + HG - 1) / HG;
   const int units = a.Bt * chunks;
-  const bool fp4_read = a.read_mode != RSSM_READ_SAME;
-  const bool shared_fp4 = a.read_mode == RSSM_READ_SHARED_NVFP4;
-  const bool hp16 = a.hp_mode == RSSM_HP_F16_SR;
-  const bool hp8 = a.hp_mode == RSSM_HP_F8_SR;
+  const bool fp4_read = LP && a.read_mode != RSSM_READ_SAME;
+  const bool shared_fp4 = LP && a.read_mode == RSSM_READ_SHARED_NVFP4;
+  const bool hp16 = LP && a.hp_mode == RSSM_HP_F16_SR;
+  const bool hp8 = LP && a.hp_mode == RSSM_HP_F8_SR;
   const int hp_fmt = hp16 ? SRC_F16 : hp8 ? SRC_F8 : SRC_F32;  // format of the stored checkpoint
 
   if (threadIdx.x == 0) {
@@ -160,6 +169,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     const uint32_t krow = (uint32_t)kCols * esz, vrow = (uint32_t)R * esz;
     struct Sched {
       int b, h0, nh, active, n_ring, n_new, m, t_out, slot0, base_e;
+      unsigned skip;
     };
     // schedule of unit u from the sequence's bookkeeping word; u >= units writes the end marker
     auto schedule = [&](int u, Sched &S, int *hdr) {
@@ -171,11 +181,14 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       const int b = u / chunks, ch = u % chunks;
       S.b = b; S.h0 = ch * HG; S.nh = min(HG, a.H - S.h0);
       int4 mw = make_int4(0, 0, 0, 0);
-      int mk = 1;
+      int mk = 1, fl = 0;
       if (lane == 0) {
         mw = a.meta_in[b];
         mk = (a.mask == nullptr) ? 1 : (int)a.mask[b];
       }
+      // skip flags left by the previous call, loaded beside the bookkeeping word
+      if (a.skip != nullptr && lane < S.nh) fl = a.skip[(size_t)b * a.H + S.h0 + lane];
+      const unsigned skm = __ballot_sync(0xffffffffu, fl != 0);
       const int c = __shfl_sync(0xffffffffu, mw.x, 0), e = __shfl_sync(0xffffffffu, mw.y, 0);
       const int pend = __shfl_sync(0xffffffffu, mw.z, 0), msk = __shfl_sync(0xffffffffu, mk, 0);
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
@@ -204,11 +217,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       S.active = active; S.n_ring = n_ring; S.n_new = n_new; S.m = m; S.t_out = t_out; S.slot0 = slot0;
       S.base_e = base_e;
+      S.skip = active ? skm : 0u;
       if (lane == 0) {
         hdr[Q_ACTIVE] = active; hdr[Q_NREC] = n_ring + n_new; hdr[Q_M] = m; hdr[Q_NRING] = n_ring;
         hdr[Q_NNEW] = n_new; hdr[Q_TOUT] = t_out; hdr[Q_SLOT0] = slot0; hdr[Q_MC] = mc; hdr[Q_ME] = me;
         hdr[Q_MP] = mp; hdr[Q_B] = b; hdr[Q_H0] = S.h0; hdr[Q_NH] = S.nh; hdr[Q_BASE] = base_e;
-        hdr[Q_WMETA] = (S.h0 == 0); hdr[Q_END] = 0;
+        hdr[Q_WMETA] = (S.h0 == 0); hdr[Q_SKIP] = (int)S.skip; hdr[Q_END] = 0;
       }
     };
     // group data of unit u: k records and q of every head, alpha / beta ring rows
@@ -291,8 +305,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             break;
           }
           unsigned char *st = stages + (size_t)s * lay.stage_bytes;
+          const bool skp = (S.skip >> i) & 1u;  // decay-aware skip: no checkpoint tile for this head
           uint32_t tb = (uint32_t)n_rec * vrow;
-          if (srcfmt == SRC_F32) tb += rows * kCols * 4;
+          if (skp) {
+          } else if (srcfmt == SRC_F32) tb += rows * kCols * 4;
           else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
           else if (srcfmt == SRC_F8) tb += rows * kCols + 16;
           else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
@@ -301,7 +317,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             mbar_arrive_expect_tx(&full[s], tb);
           }
           __syncwarp();
-          if (lane == 0) {
+          if (lane == 0 && !skp) {
             if (srcfmt == SRC_F32)
               bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
             else if (srcfmt == SRC_F16)
@@ -311,9 +327,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             else
               bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
           }
-          if (lane == 1 && srcfmt == SRC_FP4)
+          if (lane == 1 && srcfmt == SRC_FP4 && !skp)
             bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
-          if (lane == 2 && (srcfmt == SRC_FP4 || srcfmt == SRC_F8)) {
+          if (lane == 2 && (srcfmt == SRC_FP4 || srcfmt == SRC_F8) && !skp) {
             const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
             bulk_g2s(st + lay.st_g, (srcfmt == SRC_FP4 ? a.rg : a.hs) + gi4, 16, &full[s], pol_keep);
           }
@@ -394,6 +410,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
+      if (active && a.skip != nullptr && pw == 1 && lane < nh) {
+        // skip flag for the next call: fp32 product of alpha, in record order, over the records
+        // committed after this call (records m.. ; a verify's drafts are not committed)
+        const int n_comm = a.op == OP_VERIFY ? n_ring : n_rec;
+        const float *agf = reinterpret_cast<const float *>(gb + lay.gb_a);
+        float prod = 1.f;
+        for (int r = m; r < n_comm; ++r)
+          prod = __fmul_rn(prod, r < n_ring ? agf[lane * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + lane]);
+        a.skip[(size_t)b * a.H + h0 + lane] = prod < a.skip_tau ? 1 : 0;
+      }
       if (active) {
         float *u0t = reinterpret_cast<float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_u0);
         float *cot = reinterpret_cast<float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_coef);
@@ -470,6 +496,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         const int n_rec = gh[Q_NREC], m = gh[Q_M], t_out = gh[Q_TOUT];
         const int me = gh[Q_ME];
         const int n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], slot0 = gh[Q_SLOT0];
+        const unsigned skm = (unsigned)gh[Q_SKIP];
         const bool fold = m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : hp_fmt)
                                 : (fp4_read ? SRC_FP4 : hp_fmt);
@@ -534,7 +561,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               for (int j = 0; j < NO; ++j)
                 uv[j] = (j < t_out) ? *reinterpret_cast<const float4 *>(u0_h + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
               float4 sv[8];
-              if (srcfmt == SRC_F32) {
+              if ((skm >> i) & 1u) {  // skipped head: the checkpoint term is zero
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) sv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
+              } else if (srcfmt == SRC_F32) {
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr)
                   sv[rr] = *reinterpret_cast<const float4 *>(st + ((row0 + rr) * kCols + 4 * lane) * 4);
@@ -574,11 +604,12 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             const int row = row0 + (lane >> 2);
             const bool live = row < rows;
             const int rowg = kFp4Rows * t + row;  // row within the head's state
+            const bool from_ckpt = live && !((skm >> i) & 1u);  // a skipped head folds from zero
             float4 sv[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               const int ch = (c + lane) & 7;
-              sv[c] = live ? load_row4(row, qtr * 32 + ch * 4) : make_float4(0, 0, 0, 0);
+              sv[c] = from_ckpt ? load_row4(row, qtr * 32 + ch * 4) : make_float4(0, 0, 0, 0);
             }
             // s <- alpha s + beta (v[row] - alpha (s . k)) k, record by record.  The row is kept as
             // s = sig * s~ so that each record costs one FMA per element: s~ += (coef / sig') k with
@@ -790,8 +821,9 @@ cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream) {
   const int no = a.tmax <= 1 ? 1 : a.tmax <= 2 ? 2 : a.tmax <= 4 ? 4 : 8;
   const size_t smem = g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage);
   void (*kern)(GArgs) = nullptr;
+  const bool lp = a.hp_mode != RSSM_HP_F32 || a.read_mode != RSSM_READ_SAME;
 #define RSSM_PICK(TI, NOV) \
-  if (no == NOV) kern = gdn_replay_kernel<TI, NOV>;
+  if (no == NOV) kern = lp ? gdn_replay_kernel<TI, NOV, true> : gdn_replay_kernel<TI, NOV, false>;
   if (esz == 2) {
     RSSM_PICK(__nv_bfloat16, 1) RSSM_PICK(__nv_bfloat16, 2) RSSM_PICK(__nv_bfloat16, 4) RSSM_PICK(__nv_bfloat16, 8)
   } else {

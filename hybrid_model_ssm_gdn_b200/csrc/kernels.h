@@ -45,6 +45,8 @@ struct GArgs {
   float *hs;                      // E4M3 checkpoint tile scales [Bt][H][ceil(DV/64)]
   unsigned char *rq, *rs;         // NVFP4 codes [Bt][H][DV][64], scales [Bt][H][DV][8]
   float *rg;                      // tile scales [Bt][H][ceil(DV/64)]
+  unsigned char *skip;            // decay-aware skip flags [Bt][H], or null when skipping is off
+  float skip_tau;                 // flag threshold on the product of alpha over the committed records
   void *ring_k, *ring_v;          // input dtype [Bt][H][2L][128], [Bt][H][2L][DV]
   float *ring_a, *ring_b;         // alpha, beta [Bt][H][dt_stride(L)]
   const void *q, *k, *v;          // [Bt][T][H][128], [Bt][T][H][128], [Bt][T][H][DV]

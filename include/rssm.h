@@ -100,6 +100,13 @@ typedef struct {
   float q_scale;   /* GDN output scale (y = q_scale * S q) */
   const float *A;  /* Mamba-2: device [H], A_h < 0; must stay valid while the context is used */
   const float *D;  /* Mamba-2: device [H] */
+  float skip_tau;  /* GDN decay-aware read skipping ([SSD] Perspective 1st paragraph); 0 = off.  After
+                    * each step, verify or flush, a head is flagged iff the fp32 product of alpha over the
+                    * committed records of its window (in record order) is below skip_tau; the next call
+                    * then neither reads that head's checkpoint nor its read copy (the term counts as
+                    * zero, at most skip_tau * |S0| * q_scale * |q| in norm), and a fold writes the new
+                    * checkpoint from the buffer alone.  A fold that empties the window clears the flag.
+                    * Must be finite and >= 0; Mamba-2 requires 0. */
 } rssm_config;
 
 typedef struct rssm_ctx rssm_ctx;
@@ -196,6 +203,10 @@ rssm_status rssm_export(rssm_ctx *ctx, float *S_out, void *ring_out, int *meta_o
  * RSSM_ERR_UNSUPPORTED if the context has no read copy. */
 rssm_status rssm_export_read_copy(rssm_ctx *ctx, unsigned char *codes, unsigned char *scales, float *g,
                                   rssm_stream stream);
+
+/* Copy the decay-aware skip flags out: flags uint8 [Bt][H] (device), 1 = the next call skips
+ * that head's checkpoint read.  RSSM_ERR_UNSUPPORTED if the context has skip_tau == 0. */
+rssm_status rssm_export_skip(rssm_ctx *ctx, unsigned char *flags, rssm_stream stream);
 
 /* Synchronise the stream and read the sticky device error word: *code (RSSM_DEV_*) and
  * *seq (lowest failing sequence, -1 if none).  Returns RSSM_ERR_DEVICE if one is set. */

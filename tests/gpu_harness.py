@@ -41,7 +41,7 @@ class Pair:
     """A GPU ReplaySSM context and a ReplayOracle over (seq_ids x head_ids)."""
 
     def __init__(self, wl, seq_ids=None, head_ids=None, max_draft=0, hp="f32", read="same", seed=0,
-                 S0=None):
+                 S0=None, skip_tau=0.0):
         self.wl = wl
         self.kind = wl.kind
         self.seq_ids = np.arange(wl.batch) if seq_ids is None else np.asarray(seq_ids)
@@ -60,10 +60,11 @@ class Pair:
         else:
             S_full = gdn_initial_state(wl) if S0 is None else S0
             self.gpu = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, 128, 1, wl.window, max_draft, self.dt, hp, read,
-                                 seed, wl.q_scale)
+                                 seed, wl.q_scale, skip_tau=skip_tau)
             S_sel = S_full[self.seq_ids][:, self.head_ids]
             self.orc = ReplayOracle("gdn", S_sel, wl.window, nheads=wl.nheads, seq_ids=self.seq_ids,
-                                    head_ids=self.head_ids, hp=hp, read=read, seed=seed, q_scale=wl.q_scale)
+                                    head_ids=self.head_ids, hp=hp, read=read, seed=seed, q_scale=wl.q_scale,
+                                    skip_tau=skip_tau)
         self.gpu.load_checkpoint(torch.from_numpy(np.ascontiguousarray(S_full, np.float32)).cuda())
 
     # ------------------------------------------------------------------ inputs
@@ -114,6 +115,9 @@ class Pair:
         np.testing.assert_array_equal(meta[:, 0], self.orc.count)
         np.testing.assert_array_equal(meta[:, 1], self.orc.epoch)
         np.testing.assert_array_equal(meta[:, 2], self.orc.pending)
+        if self.orc.skip_tau > 0:
+            flags = self.gpu.export_skip().cpu().numpy()[self.seq_ids][:, self.head_ids]
+            np.testing.assert_array_equal(flags.astype(bool), self.orc.skip, err_msg="skip flags")
         if not ring:
             return
         fields = (("x", "x", True), ("dt", "dt", True), ("B", "B", False)) if self.kind == "mamba2" else \

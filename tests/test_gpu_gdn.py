@@ -208,6 +208,54 @@ def test_verify_lowprec_modes(cuda_ok, hp, read):
     assert p.gpu.get_error() == (0, -1)
 
 
+# ------------------------------------------------------------------------------------ decay-aware skipping
+
+FAST_DECAY = SMALL.replace(batch=5, nheads=8, decay_scale=0.6)   # alpha spread over (0.2, 1)
+
+
+@pytest.mark.parametrize("hp,read", [("f32", "same"), ("f32", "nvfp4"), ("f8sr", "same")])
+def test_skip_steps_match_oracle(cuda_ok, hp, read):
+    """Steps over three windows with tau = 1e-2 on fast-decaying gates: flags bit-exact after every call, outputs
+    and checkpoints against the oracle that skips the same reads, and some heads really skipped."""
+    wl = FAST_DECAY
+    p = Pair(wl, hp=hp, read=read, seed=5, skip_tau=1e-2)
+    tol = TOL_F32 if hp == "f32" and read == "same" else TOL_FLIP
+    skipped = 0
+    for t in range(3 * wl.window + 5):
+        skipped += int(p.orc.skip.sum())
+        y, y_ref, _ = p.step(gdn_step_inputs(wl, t))
+        assert head_rel_err(y, y_ref).max() <= tol, f"step {t}"
+        p.check_bookkeeping(ring=(t % 8 == 7))
+    assert skipped > 0
+    if hp == "f32":
+        p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
+def test_skip_verify_commit_flush(cuda_ok):
+    """Random verify/commit rounds with T in {1, 2, 4, 8}, steps between them and a flush, with skipping on."""
+    wl = FAST_DECAY
+    p = Pair(wl, max_draft=8, seed=5, skip_tau=2e-2)
+    rng = np.random.default_rng(3)
+    skipped = 0
+    for rnd in range(12):
+        T = int(rng.choice([1, 2, 4, 8]))
+        skipped += int(p.orc.skip.sum())
+        y, y_ref, _ = p.verify(T, gdn_draft_inputs(wl, rnd, T))
+        assert head_rel_err(y, y_ref).max() <= TOL_F32, f"round {rnd}"
+        p.check_bookkeeping(ring=False)
+        p.commit(accepted_lengths(wl, rnd, T))
+        for k in range(int(rng.integers(0, 4))):
+            y, y_ref, _ = p.step(gdn_step_inputs(wl, 100 + 4 * rnd + k))
+            assert head_rel_err(y, y_ref).max() <= TOL_F32
+        p.check_bookkeeping(ring=True)
+    assert skipped > 0
+    p.flush()
+    p.check_bookkeeping()
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
 @pytest.mark.slow
 def test_full_size_sampled(cuda_ok):
     """The GDN layer (batch 256, 32 heads, d 128, L 16), 1024 steps, sampled sequences and heads."""
