@@ -538,17 +538,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               return make_float4(f0.x, f0.y, f1.x, f1.y);
             }
             if (srcfmt == SRC_F8) {  // E4M3 codes times the tile scale
-              const uint32_t cw = *reinterpret_cast<const uint32_t *>(st + row * kCols + col);
-              return make_float4(__fmul_rn(e4m3_signed_value(cw & 0xFFu), g_tile),
-                                 __fmul_rn(e4m3_signed_value((cw >> 8) & 0xFFu), g_tile),
-                                 __fmul_rn(e4m3_signed_value((cw >> 16) & 0xFFu), g_tile),
-                                 __fmul_rn(e4m3_signed_value(cw >> 24), g_tile));
+              const float4 e = e4m3x4_to_float4(*reinterpret_cast<const uint32_t *>(st + row * kCols + col));
+              return make_float4(__fmul_rn(e.x, g_tile), __fmul_rn(e.y, g_tile), __fmul_rn(e.z, g_tile),
+                                 __fmul_rn(e.w, g_tile));
             }
+            // NVFP4: E2M1 codes times the block step d_b = E4M3 block scale times the tile scale
             const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + col / 2);
             const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + col / 16];
-            const float d_b = __fmul_rn(e4m3_value(sc), g_tile);
-            return make_float4(nvfp4_value(cw & 15u, d_b), nvfp4_value((cw >> 4) & 15u, d_b),
-                               nvfp4_value((cw >> 8) & 15u, d_b), nvfp4_value((cw >> 12) & 15u, d_b));
+            const float d_b = __fmul_rn(e4m3_to_float(sc), g_tile);
+            const float4 e = e2m1x4_to_float4(cw);
+            return make_float4(__fmul_rn(e.x, d_b), __fmul_rn(e.y, d_b), __fmul_rn(e.z, d_b), __fmul_rn(e.w, d_b));
           };
           if (!fold) {
             // ---------------- non-fold tile: lane owns columns 4l..4l+3 of the warp's 8 rows

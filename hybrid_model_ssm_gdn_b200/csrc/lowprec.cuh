@@ -24,6 +24,8 @@
 #pragma once
 
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace rssm {
@@ -62,7 +64,8 @@ __device__ __forceinline__ __half fp16_sr(float x, uint32_t r) {
   else thr = 0;
   const uint32_t up = ((uint64_t)r < thr) ? 1u : 0u;
   const int ulp_exp = max(Eeff - 127, -14) - 10;
-  float mag = ldexpf((float)(q + up), ulp_exp);     // exact: an integer <= 2^11 times a power of two
+  // exact: an integer <= 2^11 times 2^ulp_exp (ulp_exp >= -24, a normal fp32 power of two)
+  float mag = (float)(q + up) * __int_as_float((ulp_exp + 127) << 23);
   mag = fminf(mag, 65504.f);
   return __float2half_rn(sign ? -mag : mag);          // exact: the value lies on the fp16 grid
 }
@@ -126,6 +129,28 @@ __device__ __forceinline__ uint32_t e4m3_code(float q) {  // q >= 0 on the E4M3 
   const int E = e - 1 + 7;
   const uint32_t m = (uint32_t)ldexpf(q, 4 - e) - 8u;
   return ((uint32_t)E << 3) | m;
+}
+
+// Decoders for the kernels' tile reads, through the hardware pair conversions to f16x2 (every
+// E4M3 and E2M1 value is exactly an f16 value).  The first element sits in the low byte / low
+// nibble, as the tiles store it.
+__device__ __forceinline__ float4 e4m3x4_to_float4(uint32_t w) {  // four codes, byte i = element i
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(__half2(lo)), b = __half22float2(__half2(hi));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint32_t code) {  // one unsigned code
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(code & 0xFFu), __NV_E4M3);
+  return __low2float(__half2(h));
+}
+
+__device__ __forceinline__ float4 e2m1x4_to_float4(uint32_t w) {  // four codes, nibble i = element i
+  const __half2_raw lo = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(w & 0xFFu), __NV_E2M1);
+  const __half2_raw hi = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w >> 8) & 0xFFu), __NV_E2M1);
+  const float2 a = __half22float2(__half2(lo)), b = __half22float2(__half2(hi));
+  return make_float4(a.x, a.y, b.x, b.y);
 }
 
 __device__ __forceinline__ float e4m3_value(uint32_t code) {
