@@ -612,11 +612,21 @@ def skip_section(windows_timed: int = 8, tau: float = 1e-2) -> dict:
             skipped.append(int(layer.export_skip().sum().item()) if t > 0 else 0)
             step(i)
         K = L * windows_timed
-        ms = timed(step, K, stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(K):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[K]) / K
+        per = [sorted(ev[w * L + i].elapsed_time(ev[w * L + i + 1]) for w in range(windows_timed)) for i in range(L)]
         nbytes = sum(gdn_traffic(wl, i) - skipped[i] * head_bytes for i in range(L)) / L
         out[name] = {"ms_per_step": ms, "tokens_per_s": wl.batch / (ms * 1e-3), "bytes_per_step": nbytes,
                      "GBps": nbytes / (ms * 1e-3) / 1e9,
-                     "skipped_fraction": sum(skipped) / (L * wl.batch * wl.nheads), "device_error": layer.get_error()}
+                     "skipped_fraction": sum(skipped) / (L * wl.batch * wl.nheads),
+                     "launch_ms_by_position": [p[len(p) // 2] for p in per], "skipped_heads_by_position": skipped,
+                     "device_error": layer.get_error()}
         del layer
     out["speedup"] = out["off"]["ms_per_step"] / out["on"]["ms_per_step"]
     return out
