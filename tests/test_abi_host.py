@@ -61,12 +61,33 @@ def test_arena_size_and_validation(lib):
     assert _arena(lib, kind=abi.GDN, headdim=128, ngroups=2)[0] == 2
 
 
+def test_precision_and_skip_modes_validation(lib):
+    """The FP8 checkpoint and decay-aware skipping are GDN modes: Mamba-2 contexts refuse them; a negative,
+    NaN or infinite threshold is an argument error.  The FP8 arena holds a quarter of the fp32 checkpoint plus
+    one fp32 scale per 64-row tile; skipping adds one flag byte per head."""
+    gdn = dict(kind=abi.GDN, headdim=128, ngroups=1, A=None, D=None)
+    assert _arena(lib, hp=abi.HP_F8_SR)[0] == 3
+    assert _arena(lib, skip_tau=1e-3)[0] == 3
+    assert _arena(lib, skip_tau=-1.0, **gdn)[0] == 1
+    assert _arena(lib, skip_tau=float("nan"), **gdn)[0] == 1
+    assert _arena(lib, skip_tau=float("inf"), **gdn)[0] == 1
+    _, n32 = _arena(lib, **gdn)
+    st, n8 = _arena(lib, hp=abi.HP_F8_SR, **gdn)
+    assert st == 0
+    state = 2 * 4 * 128 * 128
+    assert n32 - n8 >= state * 3 - 256 and n32 - n8 <= state * 3 + 256
+    st, nsk = _arena(lib, skip_tau=1e-2, **gdn)
+    assert st == 0 and 2 * 4 <= nsk - n32 <= 256
+    assert _arena(lib, hp=5, **gdn)[0] == 1
+
+
 def test_null_arguments_are_rejected_without_launch(lib):
     assert lib.rssm_create(None, None, 0, None) == 1
     assert lib.rssm_create(C.byref(_cfg()), None, 0, C.byref(C.c_void_p())) == 1
     assert lib.rssm_destroy(None) == 1
     assert lib.rssm_mamba2_step(None, None, None, None, None, None, None) == 1
     assert lib.rssm_commit(None, None, None) == 1
+    assert lib.rssm_export_skip(None, None, None) == 1
     code, seq = C.c_int(), C.c_int()
     assert lib.rssm_get_error(None, C.byref(code), C.byref(seq), None) == 1
     assert lib.rssm_conv_mamba2_step(C.byref(_cfg()), None, None, None, None, None, None, None) == 1
