@@ -632,6 +632,73 @@ def skip_section(windows_timed: int = 8, tau: float = 1e-2) -> dict:
     return out
 
 
+def graph_section(batches=(1, 16, 256), n_mamba2: int = 6, n_gdn: int = 2, windows: int = 4) -> dict:
+    """A hybrid stack's state-space layers (6 Mamba-2 layers of the 120B-class shape and 2 GDN layers, L 16)
+    decoding token by token: every layer's step launched eagerly, and the same window of steps captured
+    once in a CUDA graph and replayed.  ms per token of the whole stack at several batch sizes."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    out = {"workload": f"{n_mamba2} mamba2 layers (128 heads, P 64, N 128, 8 groups) + {n_gdn} gdn layers "
+                       "(32 heads, d 128), L 16, bf16 inputs, fp32 checkpoints; eager launches vs one CUDA graph "
+                       "per window"}
+    L = WL.window
+    for Bt in batches:
+        wm, wg = WL.replace(batch=Bt), GDN_B256.replace(batch=Bt)
+        p = mamba2_params(wm)
+        A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
+        Sm = torch.from_numpy(mamba2_initial_state(wm)).to(dev)
+        Sg = torch.from_numpy(gdn_initial_state(wg)).to(dev)
+        layers = []
+        for _ in range(n_mamba2):
+            c = ReplaySSM("mamba2", Bt, wm.nheads, wm.headdim, wm.dstate, wm.ngroups, L, 0, bf, A=A, D=D)
+            c.load_checkpoint(Sm)
+            layers.append(c)
+        for _ in range(n_gdn):
+            c = ReplaySSM("gdn", Bt, wg.nheads, wg.dv, wg.dk, 1, L, 0, bf)
+            c.load_checkpoint(Sg)
+            layers.append(c)
+        del Sm, Sg
+        pm = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in mamba2_step_inputs(wm, t).items()} for t in range(L)]
+        pg = [{k: torch.from_numpy(v).to(dev).to(torch.float32 if k in ("alpha", "beta") else bf)
+               for k, v in gdn_step_inputs(wg, t).items()} for t in range(L)]
+        ym = torch.empty(Bt, wm.nheads, wm.headdim, device=dev)
+        yg = torch.empty(Bt, wg.nheads, wg.dv, device=dev)
+
+        def token(i):
+            for c in layers:
+                if c.kind == "mamba2":
+                    t = pm[i % L]
+                    c.mamba2_step(t["x"], t["B"], t["C"], t["dt"], ym)
+                else:
+                    t = pg[i % L]
+                    c.gdn_step(t["q"], t["k"], t["v"], t["alpha"], t["beta"], yg)
+
+        stream = torch.cuda.current_stream()
+        for i in range(2 * L):
+            token(i)
+        ms_eager = timed(token, windows * L, stream)
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for i in range(L):  # one window: an even number of calls per layer keeps each context's parity
+                    token(i)
+        stream.wait_stream(side)
+        for _ in range(2):
+            graph.replay()
+        ms_graph = timed(lambda i: graph.replay(), windows, stream) / L
+        errs = [c.get_error() for c in layers]
+        out[f"B{Bt}"] = {"eager_ms_per_token": ms_eager, "graph_ms_per_token": ms_graph,
+                         "graph_speedup": ms_eager / ms_graph, "launches_per_token": len(layers),
+                         "device_error": max(errs)}
+        del graph, layers
+        torch.cuda.synchronize()
+    return out
+
+
 def verify_section(rounds: int, kinds=("mamba2", "gdn")) -> dict:
     """Speculative verify + commit (T = 4, 8) vs snapshot-per-draft: the Mamba-2 shape at batch 512 and the
     Gated DeltaNet layer at batch 256."""
@@ -789,7 +856,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN, speculative-verify, precision and read-skipping sections")
     ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch",
-                                                  "precision", "skip"], default=None,
+                                                  "precision", "skip", "graph"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -810,7 +877,8 @@ def main():
                    verify_section(args.steps, (args.only.split("-")[1],)) if args.only.startswith("verify-") else
                    batch_section() if args.only == "batch" else
                    precision_section() if args.only == "precision" else
-                   skip_section() if args.only == "skip" else window_section())
+                   skip_section() if args.only == "skip" else
+                   graph_section() if args.only == "graph" else window_section())
             print(json.dumps(out))
         return
 
