@@ -35,9 +35,13 @@ def _stream():
     return C.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _dev(t, dtype, name):
+def _dev(t, dtype, name, need=None):
+    """``t`` after checking that it is a contiguous CUDA tensor of ``dtype`` with at least ``need`` elements
+    (what the kernels read or write through it; a smaller buffer would be overrun on the device)."""
     if t is None:
         return None
+    if need is not None and t.numel() < need:
+        raise ValueError(f"{name}: needs at least {need} elements, got {t.numel()} (shape {tuple(t.shape)})")
     if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous CUDA tensor of {dtype}, got {t.dtype} on {t.device}")
     return t
@@ -79,6 +83,7 @@ class ReplaySSM:
                   "rssm_create")
         self.handle = h
         self.rows = headdim
+        self.dstate = dstate
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -88,44 +93,61 @@ class ReplaySSM:
 
     # ------------------------------------------------------------------ calls
     def load_checkpoint(self, S):
-        S = _dev(S, torch.float32, "S")
+        S = _dev(S, torch.float32, "S", self.batch * self.nheads * self.rows * self.dstate)
         abi.check(self.lib.rssm_load_checkpoint(self.handle, _ptr(S), _stream()), "rssm_load_checkpoint")
 
     def _out(self, y, lead):
         if y is None:
             y = torch.empty(*lead, self.nheads, self.rows, dtype=torch.float32, device=self.device)
-        return _dev(y, torch.float32, "y")
+        n = self.nheads * self.rows
+        for s in lead:
+            n *= s
+        return _dev(y, torch.float32, "y", n)
+
+    def _need(self, name, lead):
+        """Elements of token input ``name`` with leading dims ``lead`` ([Bt] or [Bt][T])."""
+        n = 1
+        for s in lead:
+            n *= s
+        per = {"x": self.nheads * self.rows, "B": self.ngroups * self.dstate, "C": self.ngroups * self.dstate,
+               "dt": self.nheads, "q": self.nheads * self.dstate, "k": self.nheads * self.dstate,
+               "v": self.nheads * self.rows, "alpha": self.nheads, "beta": self.nheads}[name]
+        return n * per
 
     def mamba2_step(self, x, B, C_, dt, y=None):
         d = self.in_dtype
-        args = [_dev(x, d, "x"), _dev(B, d, "B"), _dev(C_, d, "C"), _dev(dt, d, "dt")]
-        y = self._out(y, (self.batch,))
+        lead = (self.batch,)
+        args = [_dev(x, d, "x", self._need("x", lead)), _dev(B, d, "B", self._need("B", lead)),
+                _dev(C_, d, "C", self._need("C", lead)), _dev(dt, d, "dt", self._need("dt", lead))]
+        y = self._out(y, lead)
         abi.check(self.lib.rssm_mamba2_step(self.handle, *map(_ptr, args), _ptr(y), _stream()), "rssm_mamba2_step")
         return y
 
     def gdn_step(self, q, k, v, alpha, beta, y=None):
         d = self.in_dtype
-        args = [_dev(q, d, "q"), _dev(k, d, "k"), _dev(v, d, "v"), _dev(alpha, torch.float32, "alpha"),
-                _dev(beta, torch.float32, "beta")]
-        y = self._out(y, (self.batch,))
+        lead = (self.batch,)
+        args = [_dev(q, d, "q", self._need("q", lead)), _dev(k, d, "k", self._need("k", lead)),
+                _dev(v, d, "v", self._need("v", lead)), _dev(alpha, torch.float32, "alpha", self._need("alpha", lead)),
+                _dev(beta, torch.float32, "beta", self._need("beta", lead))]
+        y = self._out(y, lead)
         abi.check(self.lib.rssm_gdn_step(self.handle, *map(_ptr, args), _ptr(y), _stream()), "rssm_gdn_step")
         return y
 
     def verify(self, T, y=None, **tok):
         d = self.in_dtype
         f32 = {"alpha", "beta"}
-        t = {k: _dev(v, torch.float32 if k in f32 else d, k) for k, v in tok.items()}
+        t = {k: _dev(v, torch.float32 if k in f32 else d, k, self._need(k, (self.batch, T))) for k, v in tok.items()}
         toks = abi.Tokens(**{k: v.data_ptr() for k, v in t.items()})
         y = self._out(y, (self.batch, T))
         abi.check(self.lib.rssm_verify(self.handle, T, C.byref(toks), _ptr(y), _stream()), "rssm_verify")
         return y
 
     def commit(self, accepted):
-        a = _dev(accepted, torch.int32, "accepted")
+        a = _dev(accepted, torch.int32, "accepted", self.batch)
         abi.check(self.lib.rssm_commit(self.handle, _ptr(a), _stream()), "rssm_commit")
 
     def flush(self, mask=None):
-        m = _dev(mask, torch.uint8, "mask")
+        m = _dev(mask, torch.uint8, "mask", self.batch)
         abi.check(self.lib.rssm_flush(self.handle, _ptr(m), _stream()), "rssm_flush")
 
     # ------------------------------------------------------------------ inspection

@@ -91,3 +91,27 @@ def test_null_arguments_are_rejected_without_launch(lib):
     code, seq = C.c_int(), C.c_int()
     assert lib.rssm_get_error(None, C.byref(code), C.byref(seq), None) == 1
     assert lib.rssm_conv_mamba2_step(C.byref(_cfg()), None, None, None, None, None, None, None) == 1
+
+
+def test_binding_input_sizes_match_the_workloads():
+    """The binding's per-input element counts (checked before any device call, so that a short buffer cannot
+    be overrun) agree with the seeded workloads that the tests and the bench pass, for steps and drafts."""
+    import types
+
+    import numpy as np
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM, _dev
+    from synth import GDN_B256, MAMBA2_120B, gdn_draft_inputs, gdn_step_inputs, mamba2_draft_inputs, mamba2_step_inputs
+
+    for wl, step, drafts in ((MAMBA2_120B.replace(batch=3), mamba2_step_inputs, mamba2_draft_inputs),
+                             (GDN_B256.replace(batch=3, nheads=4), gdn_step_inputs, gdn_draft_inputs)):
+        m2 = wl.kind == "mamba2"
+        fake = types.SimpleNamespace(batch=wl.batch, nheads=wl.nheads, rows=wl.headdim if m2 else wl.dv,
+                                     dstate=128, ngroups=wl.ngroups if m2 else 1)
+        for name, v in step(wl, 0).items():
+            assert ReplaySSM._need(fake, name, (wl.batch,)) == np.asarray(v).size, name
+        for name, v in drafts(wl, 0, 4).items():
+            assert ReplaySSM._need(fake, name, (wl.batch, 4)) == np.asarray(v).size, name
+    with pytest.raises(ValueError, match="needs at least 8 elements"):
+        _dev(torch.zeros(7), torch.float32, "x", 8)
