@@ -109,9 +109,9 @@ class ReplaySSM:
         n = 1
         for s in lead:
             n *= s
-        per = {"x": self.nheads * self.rows, "B": self.ngroups * self.dstate, "C": self.ngroups * self.dstate,
-               "dt": self.nheads, "q": self.nheads * self.dstate, "k": self.nheads * self.dstate,
-               "v": self.nheads * self.rows, "alpha": self.nheads, "beta": self.nheads}[name]
+        H, R, N, G = self.nheads, self.rows, self.dstate, self.ngroups
+        per = {"x": H * R, "B": G * N, "C": G * N, "dt": H, "q": H * N, "k": H * N, "v": H * R,
+               "alpha": H, "beta": H}[name]
         return n * per
 
     def mamba2_step(self, x, B, C_, dt, y=None):
