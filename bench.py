@@ -233,6 +233,16 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
                       f"(float64 step-by-step + replay bookkeeping), {dt:.1f} s on 1 host thread"}
 
 
+def arm_config(world: int) -> dict:
+    """The workload both arms report (the reference arm samples it; its cpu_baseline says how)."""
+    return {"workload": "mamba2 replay decode, batch 256 per GPU, 128 heads, P 64, N 128, 8 groups, L 16, "
+                        "bf16 inputs, fp32 checkpoint 1 GiB", "batch_per_gpu": WL.batch,
+            "global_batch": WL.batch * world, "nheads": WL.nheads, "headdim": WL.headdim,
+            "dstate": WL.dstate, "ngroups": WL.ngroups, "window": WL.window,
+            "parallelism": f"replicas x{world} (batch shards, no collective)",
+            "l2": "checkpoint stream (1 GiB/step) exceeds L2; no flush"}
+
+
 def reference_arm(args) -> dict:
     """--impl reference: the oracle timed per step on a bounded sample sized so the run takes ~2 minutes."""
     with _limits():
@@ -256,8 +266,7 @@ def reference_arm(args) -> dict:
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "mamba2 replay decode, batch 256, 128 heads, P 64, N 128, 8 groups, L 16 "
-                                   "(oracle: sampled sequences per step)"},
+            "config": arm_config(max(1, args.gpus)),
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -403,12 +412,7 @@ def run_gpu(args, rank, world):
         "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; bf16 token inputs, fp32 checkpoint)",
-        "config": {"workload": "mamba2 replay decode, batch 256 per GPU, 128 heads, P 64, N 128, 8 groups, L 16, "
-                               "bf16 inputs, fp32 checkpoint 1 GiB", "batch_per_gpu": WL.batch,
-                   "global_batch": WL.batch * world, "nheads": WL.nheads, "headdim": WL.headdim,
-                   "dstate": WL.dstate, "ngroups": WL.ngroups, "window": WL.window,
-                   "parallelism": f"replicas x{world} (batch shards, no collective)",
-                   "l2": "checkpoint stream (1 GiB/step) exceeds L2; no flush"},
+        "config": arm_config(world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic("m2_replay_kernel__mamba2_b256_L16.md",

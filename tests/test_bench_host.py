@@ -70,3 +70,11 @@ def test_committed_profile_matches_kernel_source():
     assert t is not None
     model = sum(sum(bench.traffic_model(MAMBA2_120B, c).values()) for c in range(MAMBA2_120B.window)) / 16
     assert 0.9 * model < t < 1.1 * model
+
+
+def test_both_arms_report_the_same_workload():
+    """The GPU arm and the oracle reference arm carry one config; only the batch total scales with ranks."""
+    one, four = bench.arm_config(1), bench.arm_config(4)
+    assert one["global_batch"] == 256 and four["global_batch"] == 1024
+    assert {k: v for k, v in one.items() if k not in ("global_batch", "parallelism")} == \
+        {k: v for k, v in four.items() if k not in ("global_batch", "parallelism")}
