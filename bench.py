@@ -144,41 +144,94 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
+def gpu_selector(dev_index: int) -> str:
+    """nvidia-smi ``-i`` selector of a torch device: its UUID (indices differ under CUDA_VISIBLE_DEVICES)."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:  # noqa: BLE001 - fall back to the index
+        return str(dev_index)
+
+
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms by a reader thread.
+
+    Enter it before the warm-up: ``wait_first()`` blocks until nvidia-smi has produced a sample (its
+    start-up takes longer than a short timed region), ``mark()`` brackets the timed region, and on exit
+    the sampler keeps reading until one sample after the region has arrived.  The summary covers the
+    samples from the one just before the region to the one just after it, so a region shorter than the
+    sampling period is still described by its neighbouring samples."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, selector: str):
+        self.selector = selector
         self.proc = None
+        self.samples = []          # (time, line)
+        self.t0 = self.t1 = None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.selector, f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+
+        def reader():
+            for line in self.proc.stdout:
+                if line.strip():
+                    self.samples.append((time.perf_counter(), line.strip()))
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
         return self
 
+    def wait_first(self, timeout: float = 5.0):
+        t = time.perf_counter()
+        while self.proc is not None and not self.samples and time.perf_counter() - t < timeout:
+            time.sleep(0.01)
+
+    def mark(self, which: str):
+        if which == "start":
+            self.t0 = time.perf_counter()
+        else:
+            self.t1 = time.perf_counter()
+
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self.proc is None:
+            return
+        t = time.perf_counter()
+        end = self.t1 if self.t1 is not None else t
+        while not any(ts > end for ts, _ in self.samples) and time.perf_counter() - t < 1.0:
+            time.sleep(0.01)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.proc.wait()
+
+    def window(self):
+        """Sample lines from the last one before the timed region to the first one after it."""
+        if self.t0 is None:
+            return [l for _, l in self.samples]
+        t1 = self.t1 if self.t1 is not None else self.t0
+        before = [i for i, (ts, _) in enumerate(self.samples) if ts <= self.t0]
+        after = [i for i, (ts, _) in enumerate(self.samples) if ts >= t1]
+        lo = before[-1] if before else 0
+        hi = after[0] if after else len(self.samples) - 1
+        return [l for _, l in self.samples[lo:hi + 1]]
 
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        for l in self.window():
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9:
                 continue
@@ -199,15 +252,16 @@ class ClockSampler:
 # ------------------------------------------------------------------------------ CPU oracle (baseline leg)
 
 class OracleArm:
-    """The float64 oracle, as it stands, decoding ``nseq`` sequences (all heads) of the workload on one host thread."""
+    """The float64 oracle, as it stands, decoding sequences ``first .. first + nseq - 1`` (all heads) of the
+    workload."""
 
-    def __init__(self, nseq: int):
+    def __init__(self, nseq: int, first: int = 0):
         from oracle.decoder import ReplayOracle
-        self.seqs = list(range(nseq))
+        self.seqs = list(range(first, first + nseq))
         S0 = mamba2_initial_state(WL, seqs=self.seqs)
         self.inputs = [{k: v[self.seqs] for k, v in mamba2_step_inputs(WL, t).items()} for t in range(4)]
         self.orc = ReplayOracle("mamba2", S0, WL.window, nheads=WL.nheads, ngroups=WL.ngroups,
-                                params=mamba2_params(WL))
+                                params=mamba2_params(WL), seq_ids=self.seqs)
         self.i = 0
 
     def step(self):
@@ -220,21 +274,77 @@ def _limits():
     return threadpool_limits(1)
 
 
-def cpu_baseline(budget_s: float = 12.0) -> dict:
-    """Oracle tokens/s on a bounded sample: 4 sequences x all heads, whole decode steps for ~budget_s."""
+def host_workers(nseq: int) -> int:
+    """Oracle worker processes for ``nseq`` sequences: one per usable host core, at most 32 and at most nseq."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return max(1, min(cores, 32, nseq))
+
+
+def _oracle_worker(first, nseq, warmup, steps, budget_s, barrier, out):
+    """One host process: the oracle on its own sequences, one BLAS thread.  Times ``steps`` steps after
+    ``warmup``, or (steps = 0) as many steps as fit in ``budget_s``."""
+    sys.path.insert(0, ROOT)
     with _limits():
-        arm = OracleArm(4)
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < budget_s:
+        arm = OracleArm(nseq, first)
+        for _ in range(warmup):
             arm.step()
-        dt = time.perf_counter() - t0
-    return {"value": len(arm.seqs) * arm.i / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{len(arm.seqs)} of {WL.batch} sequences x all {WL.nheads} heads, {arm.i} decode steps "
-                      f"(float64 step-by-step + replay bookkeeping), {dt:.1f} s on 1 host thread"}
+        barrier.wait()
+        t0 = time.perf_counter()
+        if steps:
+            for _ in range(steps):
+                arm.step()
+        else:
+            while time.perf_counter() - t0 < budget_s:
+                arm.step()
+        out.put((first, nseq, arm.i - warmup, time.perf_counter() - t0))
+
+
+def oracle_pool(nseq_total: int, warmup: int, steps: int, budget_s: float = 0.0) -> dict:
+    """The oracle on ``nseq_total`` sequences split over host worker processes (spawned: the parent may already
+    hold a CUDA context), started together.  Returns tokens, the slowest worker's seconds and the cores used."""
+    import multiprocessing as mp
+    w = host_workers(nseq_total)
+    ctx = mp.get_context("spawn")
+    barrier, out = ctx.Barrier(w), ctx.Queue()
+    per = [nseq_total // w + (1 if i < nseq_total % w else 0) for i in range(w)]
+    firsts = [sum(per[:i]) for i in range(w)]
+    procs = [ctx.Process(target=_oracle_worker, args=(firsts[i], per[i], warmup, steps, budget_s, barrier, out))
+             for i in range(w)]
+    for p in procs:
+        p.start()
+    res = [out.get(timeout=600) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    tokens = sum(n * k for _, n, k, _ in res)
+    secs = max(t for _, _, _, t in res)
+    return {"tokens": tokens, "seconds": secs, "cores": w, "seqs": nseq_total,
+            "steps": min(k for _, _, k, _ in res)}
+
+
+def cpu_baseline(budget_s: float = 10.0) -> dict:
+    """Oracle tokens/s on a bounded sample of the workload: one host process per core (at most 32), two
+    sequences (all heads) each, whole decode steps for ~budget_s; plus the same oracle on one thread."""
+    w = host_workers(64)
+    r = oracle_pool(2 * w, 2, 0, budget_s)
+    with _limits():
+        arm = OracleArm(2)
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget_s / 2:
+            arm.step()
+        dt1 = time.perf_counter() - t0
+    one = len(arm.seqs) * arm.i / dt1
+    return {"value": r["tokens"] / r["seconds"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+            "one_thread_tokens_per_s": one,
+            "sample": f"{r['seqs']} of {WL.batch} sequences x all {WL.nheads} heads on {r['cores']} host processes "
+                      f"(one BLAS thread each), >= {r['steps']} decode steps in {r['seconds']:.1f} s (float64 "
+                      f"step-by-step + replay bookkeeping); one thread alone: {one:.1f} tokens/s"}
 
 
 def arm_config(world: int) -> dict:
-    """The workload both arms report (the reference arm samples it; its cpu_baseline says how)."""
+    """The workload of the GPU arm (the reference arm times a sample of it; see reference_config)."""
     return {"workload": "mamba2 replay decode, batch 256 per GPU, 128 heads, P 64, N 128, 8 groups, L 16, "
                         "bf16 inputs, fp32 checkpoint 1 GiB", "batch_per_gpu": WL.batch,
             "global_batch": WL.batch * world, "nheads": WL.nheads, "headdim": WL.headdim,
@@ -243,30 +353,37 @@ def arm_config(world: int) -> dict:
             "l2": "checkpoint stream (1 GiB/step) exceeds L2; no flush"}
 
 
+def reference_config(nseq: int) -> dict:
+    """The reference arm's config: the GPU arm's layer shape, with the sample it actually times."""
+    c = {k: v for k, v in arm_config(1).items() if k not in ("batch_per_gpu", "global_batch", "parallelism", "l2")}
+    c["workload"] = (f"mamba2 replay decode (oracle, host cores), {nseq} of the 256 sequences per step, 128 heads, "
+                     "P 64, N 128, 8 groups, L 16, bf16 inputs, fp32 checkpoint")
+    c["sampled_sequences"] = nseq
+    return c
+
+
 def reference_arm(args) -> dict:
-    """--impl reference: the oracle timed per step on a bounded sample sized so the run takes ~2 minutes."""
+    """--impl reference: the oracle timed per step on the host cores, on a sample of the sequences sized so the
+    whole run takes about two minutes."""
     with _limits():
         probe = OracleArm(1)
         t0 = time.perf_counter()
         for _ in range(3):
             probe.step()
         per_seq_step = (time.perf_counter() - t0) / 3
-        nseq = int(max(1, min(WL.batch, 120.0 / ((args.steps + args.warmup) * per_seq_step))))
-        arm = OracleArm(nseq)
-        for _ in range(args.warmup):
-            arm.step()
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
-            arm.step()
-        dt = time.perf_counter() - t0
-    v = nseq * args.steps / dt
-    cb = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-          "sample": f"{nseq} of {WL.batch} sequences x all {WL.nheads} heads per step, {args.steps} steps, "
-                    f"{dt:.1f} s on 1 host thread"}
+    w = host_workers(WL.batch)
+    nseq = int(max(1, min(WL.batch, 100.0 * w / ((args.steps + args.warmup) * per_seq_step))))
+    r = oracle_pool(nseq, args.warmup, args.steps)
+    v = r["tokens"] / r["seconds"]
+    ms = r["seconds"] / args.steps * 1e3
+    cb = {"value": v, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+          "sample": f"{nseq} of {WL.batch} sequences x all {WL.nheads} heads per step on {r['cores']} host processes "
+                    f"(one BLAS thread each), {args.steps} steps after {args.warmup} warm-up, {r['seconds']:.1f} s"}
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 0,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "ms_per_sequence_step": ms / nseq,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": arm_config(max(1, args.gpus)),
+            "config": reference_config(nseq),
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -280,6 +397,7 @@ def run_gpu(args, rank, world):
     torch.cuda.set_device(rank % torch.cuda.device_count())
     dev = torch.device("cuda")
     bf = torch.bfloat16
+    L = WL.window
     p = mamba2_params(WL)
     A = torch.from_numpy(p["A"]).to(dev)
     D = torch.from_numpy(p["D"]).to(dev)
@@ -287,46 +405,62 @@ def run_gpu(args, rank, world):
                       A=A, D=D)
     S0 = torch.from_numpy(mamba2_initial_state(WL)).to(dev)
     layer.load_checkpoint(S0)
+    # each rank decodes its own batch shard: its own seeded inputs
     host_pool = [mamba2_step_inputs(WL.replace(seed=WL.seed + 1000 * rank), t) for t in range(POOL)]
     pool = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in inp.items()} for inp in host_pool]
     y = torch.empty(WL.batch, WL.nheads, WL.headdim, device=dev)
     stream = torch.cuda.current_stream()
+    pos = [0]  # steps run on the layer so far (its window position is pos % L)
 
     def step(i):
         t = pool[i % POOL]
         layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], y)
+        pos[0] += 1
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    # the timed region starts at a window boundary so that the fold count is exact
-    count0 = args.warmup % WL.window
     K = args.steps
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
-    def timed_region(first_step):
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+    with ClockSampler(gpu_selector(torch.cuda.current_device())) as clk:
+        # warm-up: at least W steps, extended to a window boundary so that the timed region starts at window
+        # position 0 (the fold falls on every L-th timed step)
+        warm = -(-args.warmup // L) * L
+        for i in range(warm):
+            step(i)
         torch.cuda.synchronize()
-        with ClockSampler(torch.cuda.current_device()) as clk:
+        clk.wait_first()
+
+        def timed_region(first_step):
+            if world > 1:
+                import torch.distributed as dist
+                dist.barrier()
+            torch.cuda.synchronize()
+            clk.mark("start")
             ev[0].record(stream)
             for i in range(K):
                 step(first_step + i)
                 ev[i + 1].record(stream)
             torch.cuda.synchronize()
-        return [ev[i].elapsed_time(ev[i + 1]) for i in range(K)], ev[0].elapsed_time(ev[K]), clk.summary()
+            clk.mark("end")
+            return [ev[i].elapsed_time(ev[i + 1]) for i in range(K)], ev[0].elapsed_time(ev[K])
 
-    per, total_ms, clocks = timed_region(args.warmup)
-    # a region that saw a hardware or thermal slowdown is measured once more (same fold phase: K steps
-    # later, a whole number of windows when K is); every rank takes the same decision
+        count0 = pos[0] % L
+        per, total_ms = timed_region(warm)
+    clocks = clk.summary()
+    # a region that saw a hardware or thermal slowdown is measured once more (from the next window boundary);
+    # every rank takes the same decision
     bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
     retry = max_over_ranks([1.0 if bad & set(clocks["reasons"]) else 0.0], device=dev)[0] > 0
     if retry:
-        per, total_ms, clocks = timed_region(args.warmup + K)
-        count0 = (args.warmup + K) % WL.window
+        with ClockSampler(gpu_selector(torch.cuda.current_device())) as clk:
+            while pos[0] % L:
+                step(pos[0])
+            torch.cuda.synchronize()
+            clk.wait_first()
+            count0 = pos[0] % L
+            per, total_ms = timed_region(pos[0])
+        clocks = clk.summary()
         clocks["remeasured"] = True
     total_ms = max_over_ranks([total_ms], device=dev)[0]
-    model = [traffic_model(WL, (count0 + i) % WL.window) for i in range(K)]
+    model = [traffic_model(WL, (count0 + i) % L) for i in range(K)]
     bytes_avg = sum(sum(m.values()) for m in model) / K
     step_ms = total_ms / K
     mean_launch_ms = sum(per) / K
@@ -334,6 +468,11 @@ def run_gpu(args, rank, world):
     achieved = bytes_avg / (mean_launch_ms * 1e-3) / 1e9
     fold_ms = [d for d, m in zip(per, model) if m["state_write"]]
     plain_ms = [d for d, m in zip(per, model) if not m["state_write"]]
+    # the same launches weighted as in a whole window ((L - 1) plain steps, one fold), whatever K is
+    window_ms = None
+    if fold_ms and plain_ms:
+        window_ms = ((L - 1) * statistics.mean(plain_ms) + statistics.mean(fold_ms)) / L
+        window_ms = max_over_ranks([window_ms], device=dev)[0]
     err = layer.get_error()
 
     # conventional step-by-step kernel on the same layer (comparison)
@@ -354,57 +493,9 @@ def run_gpu(args, rank, world):
     conv_ms = e0.elapsed_time(e1) / Kc
     del S
 
-    # end to end through the public API: every step's inputs are copied from pinned host memory and its
-    # output read back to pinned host memory inside the timed region; the copies of neighbouring steps
-    # overlap the decode on separate host->device and device->host streams (double-buffered device inputs)
-    pinned = [{k: torch.from_numpy(v).to(bf).pin_memory() for k, v in inp.items()} for inp in host_pool[:8]]
-    y_host = [torch.empty(WL.batch, WL.nheads, WL.headdim, dtype=torch.float32).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in pinned[0].values())
-    d2h = y_host[0].numel() * 4
-    Ke = max(16, K // 4)
-    bufs = [{k: torch.empty_like(v, device=dev) for k, v in pinned[0].items()} for _ in range(2)]
-    ys = [torch.empty(WL.batch, WL.nheads, WL.headdim, device=dev) for _ in range(2)]
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    copied = [torch.cuda.Event() for _ in range(2)]
-    used = [torch.cuda.Event() for _ in range(2)]
-    read = [torch.cuda.Event() for _ in range(2)]
-
-    def h2d_copy(i):
-        b = i % 2
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(used[b])           # step i-2 has consumed this buffer
-            for k, v in pinned[i % len(pinned)].items():
-                bufs[b][k].copy_(v, non_blocking=True)
-            copied[b].record(s_in)
-
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    stream.wait_event(t0)
-    s_in.wait_stream(stream)
-    s_out.wait_stream(stream)
-    h2d_copy(0)
-    for i in range(Ke):
-        b = i % 2
-        if i + 1 < Ke:
-            h2d_copy(i + 1)
-        stream.wait_event(copied[b])
-        if i >= 2:
-            stream.wait_event(read[b])             # y of step i-2 has been read back
-        t = bufs[b]
-        layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], ys[b])
-        used[b].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(used[b])
-            y_host[b].copy_(ys[b], non_blocking=True)
-            read[b].record(s_out)
-    stream.wait_stream(s_out)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = t0.elapsed_time(t1) / Ke
-    e2e_ms, conv_ms = max_over_ranks([e2e_ms, conv_ms], device=dev)
+    e2e = e2e_leg(layer, host_pool, pos, step, stream, dev)
+    e2e_ms, conv_ms = max_over_ranks([e2e["ms_per_step"], conv_ms], device=dev)
+    e2e["ms_per_step"] = e2e_ms
 
     tokens = WL.batch * world
     res = {
@@ -412,7 +503,10 @@ def run_gpu(args, rank, world):
         "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; bf16 token inputs, fp32 checkpoint)",
-        "config": arm_config(world),
+        "config": dict(arm_config(world), warmup_run=warm, timed_from_window_position=count0),
+        "window_weighted": None if window_ms is None else {
+            "tokens_per_s": tokens / (window_ms * 1e-3), "ms_per_step": window_ms,
+            "note": f"the timed launches weighted {L - 1} plain : 1 fold, as in a whole window"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic("m2_replay_kernel__mamba2_b256_L16.md",
@@ -425,13 +519,104 @@ def run_gpu(args, rank, world):
                        "conventional_bytes_per_step": conventional_bytes(WL),
                        "conventional_GBps": conventional_bytes(WL) / (conv_ms * 1e-3) / 1e9,
                        "replay_speedup": conv_ms / step_ms},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": dict(e2e, value=tokens / (e2e_ms * 1e-3), unit="tokens/s"),
         "gpu_launches": K,
         "clocks": clocks,
         "device_error": err,
     }
     return res
+
+
+def e2e_leg(layer, host_pool, pos, step, stream, dev, windows: int = 4) -> dict:
+    """End to end through the public API: every step's inputs are copied from pinned host memory and its output
+    read back to pinned host memory inside the timed region.  The copies of neighbouring steps overlap the
+    decode on separate host-to-device and device-to-host streams (double-buffered device inputs and outputs).
+    Timed over whole windows from a window boundary, after one untimed window; the same copies and the step
+    are also timed on their own, so the line shows which of them bounds the pipeline."""
+    import torch
+    bf = torch.bfloat16
+    L = WL.window
+    pinned = [{k: torch.from_numpy(v).to(bf).pin_memory() for k, v in inp.items()} for inp in host_pool[:8]]
+    y_host = [torch.empty(WL.batch, WL.nheads, WL.headdim, dtype=torch.float32).pin_memory() for _ in range(2)]
+    h2d = sum(v.numel() * v.element_size() for v in pinned[0].values())
+    d2h = y_host[0].numel() * 4
+    bufs = [{k: torch.empty_like(v, device=dev) for k, v in pinned[0].items()} for _ in range(2)]
+    ys = [torch.empty(WL.batch, WL.nheads, WL.headdim, device=dev) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(n):
+        copied = [torch.cuda.Event() for _ in range(2)]
+        used = [torch.cuda.Event() for _ in range(2)]
+        read = [torch.cuda.Event() for _ in range(2)]
+
+        def h2d_copy(i):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(used[b])           # step i-2 has consumed this buffer
+                for k, v in pinned[i % len(pinned)].items():
+                    bufs[b][k].copy_(v, non_blocking=True)
+                copied[b].record(s_in)
+
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        h2d_copy(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                h2d_copy(i + 1)
+            stream.wait_event(copied[b])
+            if i >= 2:
+                stream.wait_event(read[b])             # y of step i-2 has been read back
+            t = bufs[b]
+            layer.mamba2_step(t["x"], t["B"], t["C"], t["dt"], ys[b])
+            pos[0] += 1
+            used[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(used[b])
+                y_host[b].copy_(ys[b], non_blocking=True)
+                read[b].record(s_out)
+        stream.wait_stream(s_out)
+
+    torch.cuda.synchronize()
+    run((-pos[0]) % L + L)                             # untimed: to the next window boundary, then one window
+    torch.cuda.synchronize()
+    Ke = windows * L
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    run(Ke)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1) / Ke
+
+    def alone(fn, s, n=32):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(s)
+        for i in range(n):
+            fn(i)
+        b.record(s)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    def copy_in(i):
+        with torch.cuda.stream(s_in):
+            for k, v in pinned[i % len(pinned)].items():
+                bufs[0][k].copy_(v, non_blocking=True)
+
+    def copy_out(i):
+        with torch.cuda.stream(s_out):
+            y_host[i % 2].copy_(ys[i % 2], non_blocking=True)
+
+    h2d_ms = alone(copy_in, s_in)
+    d2h_ms = alone(copy_out, s_out)
+    while pos[0] % L:
+        step(pos[0])
+    step_alone = alone(lambda i: step(i), stream, 2 * L)
+    return {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": Ke,
+            "breakdown_ms_per_step": {"h2d_copy_alone": h2d_ms, "d2h_copy_alone": d2h_ms,
+                                      "decode_step_alone": step_alone},
+            "h2d_GBps_alone": h2d / (h2d_ms * 1e-3) / 1e9, "d2h_GBps_alone": d2h / (d2h_ms * 1e-3) / 1e9}
 
 
 # bytes per state element of each stored format: fp32, fp16, E4M3 with one fp32 scale per 64 x 128 tile,

@@ -68,8 +68,13 @@ class ReplaySSM:
         self.ngroups, self.window, self.max_draft, self.in_dtype = ngroups, window, max_draft, in_dtype
         self.device = torch.device(device or "cuda")
         if kind == "mamba2":
-            self.A = _dev(A.to(self.device, torch.float32).contiguous(), torch.float32, "A")
-            self.D = _dev(D.to(self.device, torch.float32).contiguous(), torch.float32, "D")
+            # the kernels read nheads floats from each through raw pointers: check before any device copy
+            for name, t in (("A", A), ("D", D)):
+                if t is None or t.numel() < nheads:
+                    raise ValueError(f"{name}: needs at least {nheads} elements (one per head), got "
+                                     f"{None if t is None else t.numel()}")
+            self.A = _dev(A.to(self.device, torch.float32).contiguous(), torch.float32, "A", nheads)
+            self.D = _dev(D.to(self.device, torch.float32).contiguous(), torch.float32, "D", nheads)
         else:
             self.A = self.D = None
         self.cfg = make_config(kind, batch, nheads, headdim, dstate, ngroups, window, max_draft, in_dtype, hp, read,

@@ -3,73 +3,114 @@
 // The replay kernels hand (sequence, head-group) units to their persistent blocks through
 // a counter in the context's arena (sched_grab / sched_finish in common.cuh): every unit
 // goes to exactly one block, and the last block to finish re-arms the counter for the next
-// launch on the stream.  rssm_sched_probe runs the same two helpers on counters, claim
-// marks and per-block tallies held in file-scope device arrays, so a caller can check the
-// mechanism on a device without allocating anything.  Calls must not overlap (one stream,
-// or ordered streams): the arrays are shared by every caller of the library.
+// launch on the stream.  rssm_sched_probe runs the same two helpers on a counter, claim
+// marks and per-block tallies held in one file-scope device array, so that a caller which
+// cannot allocate device memory (a host process that only holds a driver context, or code
+// that runs where allocation is forbidden, such as inside a memory-pool-managed region)
+// can still check the mechanism on its device.
+//
+// The array lives in the library's device image: every device that loads the library
+// holds it until the process exits, and every call shares it, so calls must not overlap
+// on the GPU (one stream, or streams ordered by the caller); overlapping calls race on the
+// counter and the marks.  Host code never names the array as if it were a device address:
+// the first call on a device looks its address up once with cudaGetSymbolAddress (with
+// that device current) and passes it to the kernels, so that first call should come
+// before any stream capture.
+#include <mutex>
+
 #include "sched.h"
 
 namespace rssm {
 
 namespace {
 
-// [0] unused (the error-word slot of the arena layout), [1] next unit, [2] blocks finished
-static __device__ int g_probe_sched[4];
-static __device__ unsigned int g_probe_claims[kProbeMaxUnits];
-static __device__ int g_probe_per_block[kProbeMaxBlocks];
-static __device__ int g_probe_bad;
+// Layout (ints): [0] unused (the arena's error-word slot), [1] next unit, [2] blocks finished,
+// [3] units drawn twice or more / never (filled by the check), [4] 1 if the counter was not
+// re-armed; per-block tallies from kPerBlockOff, claim marks from kClaimsOff.
+constexpr int kPerBlockOff = 64;
+constexpr int kClaimsOff = kPerBlockOff + kProbeMaxBlocks;
+constexpr int kScratchInts = kClaimsOff + kProbeMaxUnits;
+static __device__ __align__(256) int g_probe_scratch[kScratchInts];
 
-__global__ void probe_clear_kernel(int units) {
-  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x) g_probe_claims[u] = 0u;
-  if (blockIdx.x == 0 && threadIdx.x == 0) g_probe_bad = 0;
+constexpr int kMaxDevices = 64;
+std::mutex g_addr_mu;
+int *g_addr[kMaxDevices];  // device address of g_probe_scratch, per device ordinal
+
+// Clears the marks, the result words and the counter, so that a launch that never finished
+// (for instance one cut short by an error) leaves nothing behind for the next probe.
+__global__ void probe_clear_kernel(int *sc, int units) {
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x) sc[kClaimsOff + u] = 0;
+  if (blockIdx.x == 0 && threadIdx.x < 8) sc[threadIdx.x] = 0;
 }
 
 // Each block draws units until the counter runs past `units`, marking every unit it draws.
-__global__ void probe_draw_kernel(int units) {
+__global__ void probe_draw_kernel(int *sc, int units) {
   __shared__ int drawn_unit;
   int drawn = 0;
   for (;;) {
-    if (threadIdx.x == 0) drawn_unit = sched_grab(g_probe_sched);
+    if (threadIdx.x == 0) drawn_unit = sched_grab(sc);
     __syncthreads();
     const int u = drawn_unit;
     __syncthreads();
     if (u >= units) break;
     if (threadIdx.x == 0) {
-      atomicAdd(&g_probe_claims[u], 1u);
+      atomicAdd(&sc[kClaimsOff + u], 1);
       ++drawn;
     }
   }
   if (threadIdx.x == 0) {
-    g_probe_per_block[blockIdx.x] = drawn;
-    sched_finish(g_probe_sched);
+    sc[kPerBlockOff + blockIdx.x] = drawn;
+    sched_finish(sc);
   }
 }
 
-// Counts units not drawn exactly once.
-__global__ void probe_check_kernel(int units) {
+// Counts units not drawn exactly once, and checks that the last block re-armed the counter.
+__global__ void probe_check_kernel(int *sc, int units) {
   int bad = 0;
   for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < units; u += gridDim.x * blockDim.x)
-    bad += g_probe_claims[u] != 1u;
-  if (bad) atomicAdd(&g_probe_bad, bad);
+    bad += sc[kClaimsOff + u] != 1;
+  if (bad) atomicAdd(&sc[3], bad);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && (sc[1] != 0 || sc[2] != 0)) sc[4] = 1;
+}
+
+// Device address of the scratch array on the current device, looked up once per device.
+cudaError_t scratch_address(int **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_addr_mu);
+  if (g_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_probe_scratch);
+    if (e != cudaSuccess) return e;
+    g_addr[dev] = static_cast<int *>(p);
+  }
+  *out = g_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t launch_sched_probe(int units, int blocks, int *per_block, int *bad_units, cudaStream_t st) {
-  probe_clear_kernel<<<64, 256, 0, st>>>(units);
-  cudaError_t e = cudaGetLastError();
+  int *sc = nullptr;
+  cudaError_t e = scratch_address(&sc);
+  if (e != cudaSuccess) return e;
+  probe_clear_kernel<<<64, 256, 0, st>>>(sc, units);
+  e = cudaGetLastError();
   if (e == cudaSuccess) {
-    probe_draw_kernel<<<blocks, 32, 0, st>>>(units);
+    probe_draw_kernel<<<blocks, 32, 0, st>>>(sc, units);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) {
-    probe_check_kernel<<<64, 256, 0, st>>>(units);
+    probe_check_kernel<<<64, 256, 0, st>>>(sc, units);
     e = cudaGetLastError();
   }
-  if (e == cudaSuccess)
-    e = cudaMemcpyFromSymbolAsync(per_block, g_probe_per_block, sizeof(int) * blocks, 0, cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbolAsync(bad_units, g_probe_bad, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+  int words[2] = {0, 0};
+  if (e == cudaSuccess) e = cudaMemcpyAsync(per_block, sc + kPerBlockOff, sizeof(int) * blocks, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(words, sc + 3, sizeof(words), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) *bad_units = words[0] + words[1];
   return e;
 }
 

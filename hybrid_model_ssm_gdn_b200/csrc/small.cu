@@ -49,17 +49,19 @@ __global__ void export_meta_kernel(const int4 *meta, int *out, int Bt, int L) {
   out[4 * b + 3] = (m.y & 1) * L;
 }
 
-// out[(b*X + x)][s] = in[(b*X + x)][base_b + s], rows of slot_bytes (multiple of 4)
+// out[(b*X + x)][s] = in[(b*X + x)][base_b + s], rows of slot_bytes (multiple of 4); a capped grid
+// strides over the rows, so any row count the host API accepts fits one launch
 __global__ void gather_window_kernel(const unsigned char *in, unsigned char *out, const int4 *meta, int Bt, int X,
-                                     size_t in_group_bytes, int slot_bytes, int L) {
-  const size_t row = blockIdx.x;  // (b*X + x)*L + s
-  const int s = (int)(row % L);
-  const size_t grp = row / L;
-  const int b = (int)(grp / X);
-  const int base = (meta[b].y & 1) * L;
-  const uint32_t *src = reinterpret_cast<const uint32_t *>(in + grp * in_group_bytes + (size_t)(base + s) * slot_bytes);
-  uint32_t *dst = reinterpret_cast<uint32_t *>(out + row * slot_bytes);
-  for (int w = threadIdx.x; w < slot_bytes / 4; w += blockDim.x) dst[w] = src[w];
+                                     size_t in_group_bytes, int slot_bytes, int L, size_t rows) {
+  for (size_t row = blockIdx.x; row < rows; row += gridDim.x) {  // row = (b*X + x)*L + s
+    const int s = (int)(row % L);
+    const size_t grp = row / L;
+    const int b = (int)(grp / X);
+    const int base = (meta[b].y & 1) * L;
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(in + grp * in_group_bytes + (size_t)(base + s) * slot_bytes);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(out + row * slot_bytes);
+    for (int w = threadIdx.x; w < slot_bytes / 4; w += blockDim.x) dst[w] = src[w];
+  }
 }
 
 }  // namespace
@@ -84,7 +86,8 @@ cudaError_t launch_gather_window(const unsigned char *in, unsigned char *out, co
                                  size_t in_group_bytes, int slot_bytes, int L, cudaStream_t stream) {
   const size_t rows = (size_t)Bt * X * L;
   if (rows == 0) return cudaSuccess;
-  gather_window_kernel<<<(unsigned)rows, 64, 0, stream>>>(in, out, meta, Bt, X, in_group_bytes, slot_bytes, L);
+  const unsigned grid = (unsigned)(rows < (size_t)(1u << 20) ? rows : (size_t)(1u << 20));
+  gather_window_kernel<<<grid, 64, 0, stream>>>(in, out, meta, Bt, X, in_group_bytes, slot_bytes, L, rows);
   return cudaGetLastError();
 }
 

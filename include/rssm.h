@@ -236,12 +236,22 @@ rssm_status rssm_snap_commit(const rssm_config *cfg, int *cur, const int *accept
 
 /* Run the unit scheduler of the replay kernels on its own: `blocks` blocks draw `units` work
  * units from a counter with one atomic per unit, and the last block to finish re-arms the
- * counter (the mechanism the replay kernels use on the counter in the context's arena).  Needs
- * no caller device memory: the counter, per-unit claim marks and per-block tallies live in
- * file-scope device arrays of the library, so calls must not overlap in time.
- *   units 1 .. 65536, blocks 1 .. 1024;
+ * counter (the mechanism the replay kernels use on the counter in the context's arena).  The
+ * pages have no counterpart: this is a check of this library's own scheduling.
+ *
+ * It allocates nothing and needs no caller device memory, for callers that cannot allocate
+ * on the device (for instance a process that only holds a driver context, or code running
+ * where device allocation is forbidden): the counter, per-unit claim marks and per-block
+ * tallies live in one file-scope device array of the library, of fixed size (about 260 KiB,
+ * for at most 65536 units and 1024 blocks), which every device that loads the library holds
+ * until the process exits.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress, with the device current); make that first call before any stream
+ * capture.  Every call clears the array before use, and all calls share it: calls that
+ * overlap on the GPU race, so order them on one stream.
+ *   units 1 .. 65536, blocks 1 .. 1024 (RSSM_ERR_ARG beyond these limits, before any device work);
  *   per_block host int [blocks]: units each block drew (they sum to `units`);
- *   bad_units host int [1]: number of units not drawn exactly once (0 when correct).
+ *   bad_units host int [1]: units not drawn exactly once, plus one if the last block did not
+ *     re-arm the counter (0 when correct).
  * Synchronises `stream`.  RSSM_ERR_ARG on a count out of range or a null pointer. */
 rssm_status rssm_sched_probe(int units, int blocks, int *per_block, int *bad_units, rssm_stream stream);
 

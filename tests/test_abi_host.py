@@ -115,3 +115,15 @@ def test_binding_input_sizes_match_the_workloads():
             assert ReplaySSM._need(fake, name, (wl.batch, 4)) == np.asarray(v).size, name
     with pytest.raises(ValueError, match="needs at least 8 elements"):
         _dev(torch.zeros(7), torch.float32, "x", 8)
+
+
+def test_short_per_head_parameters_are_rejected_before_any_device_call():
+    """Mamba-2 contexts read nheads floats from A and D through raw pointers: shorter tensors are refused on the
+    host, before the binding touches the device."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM
+    ok, short = torch.full((4,), -1.0), torch.zeros(3)
+    for A, D, name in ((short, ok, "A"), (ok, short, "D"), (None, ok, "A")):
+        with pytest.raises(ValueError, match=f"{name}: needs at least 4 elements"):
+            ReplaySSM("mamba2", 2, 4, 64, 128, 1, 16, 0, torch.bfloat16, A=A, D=D)

@@ -72,9 +72,31 @@ def test_committed_profile_matches_kernel_source():
     assert 0.9 * model < t < 1.1 * model
 
 
-def test_both_arms_report_the_same_workload():
-    """The GPU arm and the oracle reference arm carry one config; only the batch total scales with ranks."""
+def test_both_arms_report_the_same_layer_shape():
+    """The GPU arm and the oracle reference arm time the same layer shape; the reference arm's config says how
+    many of the sequences it samples, and carries no replica or batch fields of the GPU arm."""
     one, four = bench.arm_config(1), bench.arm_config(4)
     assert one["global_batch"] == 256 and four["global_batch"] == 1024
-    assert {k: v for k, v in one.items() if k not in ("global_batch", "parallelism")} == \
-        {k: v for k, v in four.items() if k not in ("global_batch", "parallelism")}
+    ref = bench.reference_config(12)
+    shape = ("nheads", "headdim", "dstate", "ngroups", "window")
+    assert {k: ref[k] for k in shape} == {k: one[k] for k in shape} == {k: four[k] for k in shape}
+    assert ref["sampled_sequences"] == 12 and "12 of the 256 sequences" in ref["workload"]
+    assert not {"parallelism", "global_batch", "batch_per_gpu"} & set(ref)
+
+
+def test_clock_window_uses_neighbouring_samples():
+    """A timed region shorter than the sampling period is described by the samples just before and after it."""
+    c = bench.ClockSampler("0")
+    line = "0, {sm}, 1965, 700, 0x0, Not Active, Not Active, Not Active, {cap}"
+    c.samples = [(1.0, line.format(sm=1800, cap="Not Active")), (2.0, line.format(sm=1900, cap="Active")),
+                 (3.0, line.format(sm=1950, cap="Not Active")), (4.0, line.format(sm=1000, cap="Not Active"))]
+    c.t0, c.t1 = 2.2, 2.3
+    s = c.summary()
+    assert s["samples"] == 2 and s["sm_mhz"] == 1925 and s["reasons"] == ["sw_power_cap"]
+    c.t0, c.t1 = 0.5, 0.6                      # region before the first sample: the first sample stands for it
+    assert bench.ClockSampler.summary(c)["samples"] == 1
+
+
+def test_host_workers_bounds():
+    assert bench.host_workers(1) == 1
+    assert 1 <= bench.host_workers(1000) <= 32
