@@ -104,6 +104,11 @@ def max_over_ranks(values, device=None):
     return [float(v) for v in t.cpu()]
 
 
+def rank_workload(rank: int):
+    """The workload rank ``rank`` decodes: the same layer with its own input seed (its own batch shard)."""
+    return WL.replace(seed=WL.seed + 1000 * rank)
+
+
 def weak_scaling_value(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
     """Whole-job tokens/s: every rank decodes its own batch shard; time is the slowest rank's."""
     return tokens_per_rank_step * world * steps / (max_ms * 1e-3)
@@ -406,7 +411,7 @@ def run_gpu(args, rank, world):
     S0 = torch.from_numpy(mamba2_initial_state(WL)).to(dev)
     layer.load_checkpoint(S0)
     # each rank decodes its own batch shard: its own seeded inputs
-    host_pool = [mamba2_step_inputs(WL.replace(seed=WL.seed + 1000 * rank), t) for t in range(POOL)]
+    host_pool = [mamba2_step_inputs(rank_workload(rank), t) for t in range(POOL)]
     pool = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in inp.items()} for inp in host_pool]
     y = torch.empty(WL.batch, WL.nheads, WL.headdim, device=dev)
     stream = torch.cuda.current_stream()
@@ -623,6 +628,7 @@ def e2e_leg(layer, host_pool, pos, step, stream, dev, windows: int = 4) -> dict:
 # and NVFP4 (E2M1 codes, an E4M3 scale per 16 elements, one fp32 scale per tile)
 HP_BYTES = {"f32": 4.0, "f16sr": 2.0, "f8sr": 1.0 + 4.0 / (64 * 128)}
 NVFP4_BYTES = 0.5 + 1.0 / 16 + 4.0 / (64 * 128)
+NVFP4D_BYTES = NVFP4_BYTES + 1.0 / 16     # plus one E4M3 column-group scale per 16 elements
 
 
 def gdn_traffic(wl, count_before: int, hp: str = "f32", read: str = "same") -> float:
@@ -634,11 +640,11 @@ def gdn_traffic(wl, count_before: int, hp: str = "f32", read: str = "same") -> f
     esz = 2 if wl.in_dtype == "bf16" else 4
     elems = Bt * H * dv * dk
     ckpt = elems * (NVFP4_BYTES if read == "shared_nvfp4" else HP_BYTES[hp])
-    copy = elems * NVFP4_BYTES if read == "nvfp4" else 0.0
+    copy = elems * {"nvfp4": NVFP4_BYTES, "nvfp4d": NVFP4D_BYTES}.get(read, 0.0)
     rec = Bt * H * (dk * esz + dv * esz + 8)
     tok = Bt * H * (2 * dk * esz + dv * esz + 8)
     fold = count_before + 1 == L
-    state = ckpt + ckpt + copy if fold else (copy if read == "nvfp4" else ckpt)
+    state = ckpt + ckpt + copy if fold else (copy if read in ("nvfp4", "nvfp4d") else ckpt)
     return state + count_before * rec + tok + rec + Bt * H * dv * 4
 
 
@@ -713,7 +719,7 @@ def gdn_section(steps: int) -> dict:
 
 
 PRECISION_MODES = (("f32", "same"), ("f16sr", "same"), ("f8sr", "same"), ("f32", "nvfp4"), ("f16sr", "nvfp4"),
-                   ("f8sr", "nvfp4"), ("f32", "shared_nvfp4"))
+                   ("f8sr", "nvfp4"), ("f32", "shared_nvfp4"), ("f32", "nvfp4d"))
 
 
 def precision_section(windows_timed: int = 4) -> dict:
@@ -815,6 +821,60 @@ def skip_section(windows_timed: int = 8, tau: float = 1e-2) -> dict:
                      "GBps": nbytes / (ms * 1e-3) / 1e9,
                      "skipped_fraction": sum(skipped) / (L * wl.batch * wl.nheads),
                      "launch_ms_by_position": [p[len(p) // 2] for p in per], "skipped_heads_by_position": skipped,
+                     "device_error": layer.get_error()}
+        del layer
+    out["speedup"] = out["off"]["ms_per_step"] / out["on"]["ms_per_step"]
+    return out
+
+
+def skip_mamba2_section(windows_timed: int = 8, tau: float = 1e-2, decay_scale: float = 8.0) -> dict:
+    """Mamba-2 layer (batch 256, 128 heads, P 64, N 128, 8 groups, L 16) with faster-decaying heads (A times
+    ``decay_scale``): decay-aware read skipping off and on.  As in the GDN section, one untimed window of flag
+    exports gives the skipped heads at each window position (the inputs cycle with period L)."""
+    import torch
+
+    from hybrid_model_ssm_gdn_b200 import ReplaySSM
+    wl, dev, bf = WL.replace(decay_scale=decay_scale), torch.device("cuda"), torch.bfloat16
+    L = wl.window
+    p = mamba2_params(wl)
+    A, D = torch.from_numpy(p["A"]).to(dev), torch.from_numpy(p["D"]).to(dev)
+    S0 = torch.from_numpy(mamba2_initial_state(wl)).to(dev)
+    pool = [{k: torch.from_numpy(v).to(dev).to(bf) for k, v in mamba2_step_inputs(wl, t).items()} for t in range(L)]
+    y = torch.empty(wl.batch, wl.nheads, wl.headdim, device=dev)
+    stream = torch.cuda.current_stream()
+    head_bytes = wl.headdim * wl.dstate * 4
+    out = {"workload": f"mamba2 replay decode, batch 256, 128 heads, P 64, N 128, 8 groups, L 16, bf16 inputs, "
+                       f"fp32 checkpoint, A x {decay_scale}", "tau": tau}
+    for name, t in (("off", 0.0), ("on", tau)):
+        layer = ReplaySSM("mamba2", wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups, L, 0, bf, A=A, D=D,
+                          skip_tau=t)
+        layer.load_checkpoint(S0)
+
+        def step(i):
+            q = pool[i % L]
+            layer.mamba2_step(q["x"], q["B"], q["C"], q["dt"], y)
+
+        for i in range(2 * L):
+            step(i)
+        skipped = []
+        for i in range(L):
+            skipped.append(int(layer.export_skip().sum().item()) if t > 0 else 0)
+            step(i)
+        K = L * windows_timed
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(K):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[K]) / K
+        per = [sorted(ev[w * L + i].elapsed_time(ev[w * L + i + 1]) for w in range(windows_timed)) for i in range(L)]
+        nbytes = sum(sum(traffic_model(wl, i).values()) - skipped[i] * head_bytes for i in range(L)) / L
+        out[name] = {"ms_per_step": ms, "tokens_per_s": wl.batch / (ms * 1e-3), "bytes_per_step": nbytes,
+                     "GBps": nbytes / (ms * 1e-3) / 1e9,
+                     "skipped_fraction": sum(skipped) / (L * wl.batch * wl.nheads),
+                     "launch_ms_by_position": [q[len(q) // 2] for q in per], "skipped_heads_by_position": skipped,
                      "device_error": layer.get_error()}
         del layer
     out["speedup"] = out["off"]["ms_per_step"] / out["on"]["ms_per_step"]
@@ -1045,7 +1105,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN, speculative-verify, precision and read-skipping sections")
     ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch",
-                                                  "precision", "skip", "graph"], default=None,
+                                                  "precision", "skip", "skip-mamba2", "graph"], default=None,
                     help="run only one extra section and print its JSON (for profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -1067,6 +1127,7 @@ def main():
                    batch_section() if args.only == "batch" else
                    precision_section() if args.only == "precision" else
                    skip_section() if args.only == "skip" else
+                   skip_mamba2_section() if args.only == "skip-mamba2" else
                    graph_section() if args.only == "graph" else window_section())
             print(json.dumps(out))
         return
@@ -1082,6 +1143,7 @@ def main():
         res["verify"] = verify_section(512)
         res["precision"] = precision_section()
         res["skip"] = skip_section()
+        res["skip_mamba2"] = skip_mamba2_section()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline()
     if rank == 0:

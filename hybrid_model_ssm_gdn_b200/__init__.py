@@ -24,7 +24,8 @@ __all__ = ["ReplaySSM", "RSSMError", "conv_mamba2_step", "conv_gdn_step", "snap_
 
 _DT = {torch.float32: abi.F32, torch.bfloat16: abi.BF16}
 _HP = {"f32": abi.HP_F32, "f16sr": abi.HP_F16_SR, "f8sr": abi.HP_F8_SR}
-_READ = {"same": abi.READ_SAME, "nvfp4": abi.READ_NVFP4, "shared_nvfp4": abi.READ_SHARED_NVFP4}
+_READ = {"same": abi.READ_SAME, "nvfp4": abi.READ_NVFP4, "shared_nvfp4": abi.READ_SHARED_NVFP4,
+         "nvfp4d": abi.READ_NVFP4D}
 
 
 def _ptr(t):
@@ -193,6 +194,12 @@ class ReplaySSM:
         abi.check(self.lib.rssm_export_read_copy(self.handle, _ptr(codes), _ptr(scales), _ptr(g), _stream()),
                   "rssm_export_read_copy")
         return {"packed": codes, "scales": scales, "g": g}
+
+    def export_column_scales(self):
+        """Column-group scales of the two-axis read copy: uint8 E4M3 [Bt][H][ceil(rows/16)][128]."""
+        cs = torch.empty(self.batch, self.nheads, (self.rows + 15) // 16, 128, dtype=torch.uint8, device=self.device)
+        abi.check(self.lib.rssm_export_column_scales(self.handle, _ptr(cs), _stream()), "rssm_export_column_scales")
+        return cs
 
     def export_skip(self):
         """Decay-aware skip flags uint8 [Bt][H] (1 = the next call skips that head's checkpoint read)."""

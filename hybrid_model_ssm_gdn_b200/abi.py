@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libr
 MAMBA2, GDN = 0, 1
 F32, BF16 = 0, 1
 HP_F32, HP_F16_SR, HP_F8_SR = 0, 1, 2
-READ_SAME, READ_NVFP4, READ_SHARED_NVFP4 = 0, 1, 2
+READ_SAME, READ_NVFP4, READ_SHARED_NVFP4, READ_NVFP4D = 0, 1, 2, 3
 STATUS = {0: "RSSM_OK", 1: "RSSM_ERR_ARG", 2: "RSSM_ERR_SHAPE", 3: "RSSM_ERR_UNSUPPORTED",
           4: "RSSM_ERR_ARENA_TOO_SMALL", 5: "RSSM_ERR_CUDA", 6: "RSSM_ERR_DEVICE"}
 DEV_OK, DEV_PENDING, DEV_NO_VERIFY, DEV_ACCEPTED, DEV_TIMEOUT = 0, 1, 2, 3, 4
@@ -56,6 +56,7 @@ _SIGS = {
     "rssm_export": [_P, _P, _P, _P, _P],
     "rssm_export_read_copy": [_P, _P, _P, _P, _P],
     "rssm_export_skip": [_P, _P, _P],
+    "rssm_export_column_scales": [_P, _P, _P],
     "rssm_get_error": [_P, C.POINTER(C.c_int), C.POINTER(C.c_int), _P],
     "rssm_conv_mamba2_step": [C.POINTER(Config), _P, _P, _P, _P, _P, _P, _P],
     "rssm_conv_gdn_step": [C.POINTER(Config), _P, _P, _P, _P, _P, _P, _P, _P],

@@ -2,6 +2,7 @@
 //
 // Validates arguments, carves the caller's arena, keeps the bookkeeping parity bit and
 // launches the kernels on the caller's stream.  Nothing here allocates device memory.
+#include <math.h>
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -20,6 +21,10 @@ struct rssm_ctx {
   int smem_optin;
   int nstage_override;
   int loaded;    // set by the first successful rssm_load_checkpoint
+  float skip_ln_tau;       // Mamba-2 decay-aware skipping: ln(skip_tau) in fp32
+  long long wait_cycles;   // bound of the kernels' waits (RSSM_WAIT_CYCLES, default ~1 s)
+  unsigned int suspend_ns; // suspend-time hint of the kernels' barrier polls (RSSM_SUSPEND_NS)
+  int withhold;            // test hook RSSM_WITHHOLD_TILE (-1: off)
 };
 
 namespace {
@@ -40,7 +45,7 @@ rssm_status validate(const rssm_config *c) {
   if (c->kind != RSSM_MAMBA2 && c->kind != RSSM_GDN) return RSSM_ERR_ARG;
   if (c->in_dtype != RSSM_F32 && c->in_dtype != RSSM_BF16) return RSSM_ERR_ARG;
   if (c->hp != RSSM_HP_F32 && c->hp != RSSM_HP_F16_SR && c->hp != RSSM_HP_F8_SR) return RSSM_ERR_ARG;
-  if (c->read < RSSM_READ_SAME || c->read > RSSM_READ_SHARED_NVFP4) return RSSM_ERR_ARG;
+  if (c->read < RSSM_READ_SAME || c->read > RSSM_READ_NVFP4D) return RSSM_ERR_ARG;
   if (!(c->skip_tau >= 0.f) || c->skip_tau > 3.0e38f) return RSSM_ERR_ARG;  // NaN, negative or infinite
   if (c->batch < 1 || c->nheads < 1) return RSSM_ERR_SHAPE;
   if ((long long)c->batch * c->nheads > (1LL << 26)) return RSSM_ERR_SHAPE;
@@ -53,7 +58,7 @@ rssm_status validate(const rssm_config *c) {
     if (c->headdim > 64) return RSSM_ERR_SHAPE;
     if (c->ngroups < 1 || c->nheads % c->ngroups != 0) return RSSM_ERR_SHAPE;
     if (!c->A || !c->D) return RSSM_ERR_ARG;
-    if (c->hp != RSSM_HP_F32 || c->read != RSSM_READ_SAME || c->skip_tau != 0.f) return RSSM_ERR_UNSUPPORTED;
+    if (c->hp != RSSM_HP_F32 || c->read != RSSM_READ_SAME) return RSSM_ERR_UNSUPPORTED;
   } else {
     if (c->headdim > 128) return RSSM_ERR_SHAPE;
     if (c->ngroups != 1) return RSSM_ERR_SHAPE;
@@ -82,6 +87,10 @@ rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, c
   a.ring_x = x->arena + x->lay.ring_a; a.ring_B = x->arena + x->lay.ring_b;
   a.ring_dt = reinterpret_cast<float *>(x->arena + x->lay.ring_c);
   a.x = xin; a.Bin = B; a.C = C; a.dt = dt; a.mask = mask; a.A = c.A; a.D = c.D; a.y = y;
+  a.skip = c.skip_tau > 0.f ? x->arena + x->lay.skip : nullptr;
+  a.skip_ln_tau = x->skip_ln_tau;
+  a.wait_cycles = x->wait_cycles; a.suspend_ns = x->suspend_ns; a.withhold = x->withhold;
+  x->withhold = -1;  // the test hook fires on one launch only
   cudaError_t e = launch_m2_replay(a, esz, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity ^= 1;
@@ -99,18 +108,24 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   a.grid = a.units < x->num_sms ? a.units : x->num_sms;
   a.hp_mode = c.hp; a.read_mode = c.read; a.seed = c.seed; a.q_scale = c.q_scale;
   const int esz = esize(c);
-  a.nstage = x->nstage_override > 0 ? x->nstage_override : g_max_stages(a.DV, a.L, a.tmax, esz, x->smem_optin - 1024);
-  if (a.nstage < 2 || a.nstage > 8 || g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) > x->smem_optin) return RSSM_ERR_SHAPE;
+  const int extra = g_extra_smem_bytes(c.read);
+  a.nstage = x->nstage_override > 0 ? x->nstage_override
+                                    : g_max_stages(a.DV, a.L, a.tmax, esz, x->smem_optin - 1024 - extra);
+  if (a.nstage < 2 || a.nstage > 8 || g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) + extra > x->smem_optin)
+    return RSSM_ERR_SHAPE;
   a.meta_in = meta_cur(x); a.meta_out = meta_next(x); a.err = err_word(x);
   a.hp = x->arena + x->lay.hp;
   a.hs = reinterpret_cast<float *>(x->arena + x->lay.hs);
   a.rq = x->arena + x->lay.rq; a.rs = x->arena + x->lay.rs; a.rg = reinterpret_cast<float *>(x->arena + x->lay.rg);
+  a.rc = x->arena + x->lay.rc;
   a.ring_k = x->arena + x->lay.ring_a; a.ring_v = x->arena + x->lay.ring_b;
   a.ring_a = reinterpret_cast<float *>(x->arena + x->lay.ring_c);
   a.ring_b = reinterpret_cast<float *>(x->arena + x->lay.ring_d);
   a.skip = c.skip_tau > 0.f ? x->arena + x->lay.skip : nullptr;
   a.skip_tau = c.skip_tau;
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.beta = beta; a.mask = mask; a.y = y;
+  a.wait_cycles = x->wait_cycles; a.suspend_ns = x->suspend_ns; a.withhold = x->withhold;
+  x->withhold = -1;  // the test hook fires on one launch only
   cudaError_t e = launch_gdn_replay(a, esz, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity ^= 1;
@@ -164,6 +179,19 @@ rssm_status rssm_create(const rssm_config *cfg, void *arena, size_t arena_bytes,
   x->smem_optin = optin;
   const char *ns = getenv("RSSM_NSTAGE");
   x->nstage_override = ns ? atoi(ns) : 0;
+  // the rule is A_h * sum(dt) < ln(tau) in fp32; ln is taken in double by the C library and rounded once
+  x->skip_ln_tau = cfg->skip_tau > 0.f ? (float)log((double)cfg->skip_tau) : 0.f;
+  x->wait_cycles = kWaitCycles;
+  const char *wc = getenv("RSSM_WAIT_CYCLES");
+  if (wc) {
+    const long long v = atoll(wc);
+    x->wait_cycles = v < 100000LL ? 100000LL : v > kWaitCycles ? kWaitCycles : v;
+  }
+  const char *sn = getenv("RSSM_SUSPEND_NS");
+  x->suspend_ns = sn ? (unsigned)atoi(sn) : kSuspendNs;
+  // test hook for the timeout path: honoured only together with a shortened wait bound
+  const char *wh = getenv("RSSM_WITHHOLD_TILE");
+  x->withhold = (wh && wc) ? atoi(wh) : -1;
   *out = x;
   return RSSM_OK;
 }
@@ -185,8 +213,8 @@ rssm_status rssm_load_checkpoint(rssm_ctx *x, const float *S, rssm_stream stream
   else
     e = launch_store_state(S, x->arena + x->lay.hp, reinterpret_cast<float *>(x->arena + x->lay.hs), c.hp,
                            x->arena + x->lay.rq, x->arena + x->lay.rs,
-                           reinterpret_cast<float *>(x->arena + x->lay.rg), c.read, (int)units, c.headdim, c.seed,
-                           c.nheads, st);
+                           reinterpret_cast<float *>(x->arena + x->lay.rg), x->arena + x->lay.rc, c.read, (int)units,
+                           c.headdim, c.seed, c.nheads, st);
   if (e == cudaSuccess)  // empty ring: count = 0 everywhere; zeroed so exports are deterministic
     e = cudaMemsetAsync(x->arena + x->lay.ring_a, 0, x->lay.total - x->lay.ring_a, st);
   if (e == cudaSuccess) e = launch_meta_reset(reinterpret_cast<int4 *>(x->arena + x->lay.meta), c.batch, err_word(x), st);
@@ -307,6 +335,16 @@ rssm_status rssm_export_read_copy(rssm_ctx *x, unsigned char *codes, unsigned ch
                         cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_fail(e);
   return RSSM_OK;
+}
+
+rssm_status rssm_export_column_scales(rssm_ctx *x, unsigned char *colscales, rssm_stream stream) {
+  if (!x || !colscales) return RSSM_ERR_ARG;
+  const rssm_config &c = x->cfg;
+  if (c.read != RSSM_READ_NVFP4D || !x->loaded) return RSSM_ERR_UNSUPPORTED;
+  const size_t bytes = (size_t)c.batch * c.nheads * ((c.headdim + 15) / 16) * kCols;
+  const cudaError_t e = cudaMemcpyAsync(colscales, x->arena + x->lay.rc, bytes, cudaMemcpyDeviceToDevice,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RSSM_OK : cuda_fail(e);
 }
 
 rssm_status rssm_export_skip(rssm_ctx *x, unsigned char *flags, rssm_stream stream) {

@@ -27,7 +27,8 @@ constexpr int kMaxDraft = 8;
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;  // + one producer warp
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at B200 clocks
+constexpr long long kWaitCycles = 2000000000LL;  // default bound of every wait, ~1 s at B200 clocks
+constexpr unsigned int kSuspendNs = 0;           // default suspend-time hint of a barrier poll (hardware default)
 
 // error word: min over (seq * 16 + code); 0x7fffffff = clean
 constexpr int kErrClean = 0x7fffffff;
@@ -44,11 +45,12 @@ struct ArenaLayout {
   size_t rq;       // NVFP4 codes u8 [Bt][H][R][64]
   size_t rs;       // NVFP4 block scales u8 [Bt][H][R][8]
   size_t rg;       // NVFP4 tile scale fp32 [Bt][H][ceil(R/64)] (padded to 16 bytes)
+  size_t rc;       // two-axis copy: column-group scales u8 [Bt][H][ceil(R/16)][128]
   size_t ring_a;   // Mamba-2 x [Bt][H][2L][P] / GDN k [Bt][H][2L][128]   (input dtype)
   size_t ring_b;   // Mamba-2 B [Bt][G][2L][128] / GDN v [Bt][H][2L][d_v] (input dtype)
   size_t ring_c;   // Mamba-2 dt / GDN alpha: fp32 [Bt][H][dt_stride(L)]
   size_t ring_d;   // GDN beta: fp32 [Bt][H][dt_stride(L)]
-  size_t skip;     // GDN decay-aware skip flags u8 [Bt][H] (only with skip_tau > 0)
+  size_t skip;     // decay-aware skip flags u8 [Bt][H] (only with skip_tau > 0)
   size_t total;
 };
 
@@ -70,6 +72,7 @@ inline ArenaLayout make_layout(const rssm_config &c) {
   a.rs = take(fp4 ? units * R * kCols / 16 : 0);
   const size_t nrb = (R + 63) / 64;  // NVFP4 tiles (64-row blocks) per head
   a.rg = take(fp4 ? align_up(units * nrb, 4) * 4 : 0);
+  a.rc = take(c.read == RSSM_READ_NVFP4D ? units * ((R + 15) / 16) * kCols : 0);
   if (c.kind == RSSM_MAMBA2) {
     a.ring_a = take(units * 2 * L * R * esz);
     a.ring_b = take(Bt * c.ngroups * 2 * L * kCols * esz);
@@ -81,7 +84,7 @@ inline ArenaLayout make_layout(const rssm_config &c) {
     a.ring_c = take(units * dt_stride(c.window) * 4);
     a.ring_d = take(units * dt_stride(c.window) * 4);
   }
-  a.skip = take(c.kind == RSSM_GDN && c.skip_tau > 0.f ? units : 0);
+  a.skip = take(c.skip_tau > 0.f ? units : 0);
   a.total = off;
   return a;
 }
@@ -143,35 +146,53 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+// How a wait spins: `limit` clock cycles in all, and each try_wait may suspend the warp for up to
+// `hint_ns` nanoseconds until the phase completes (0: the hardware's default), so that waiting warps
+// take fewer issue slots from working ones.
+struct WaitSpec {
+  long long limit;
+  uint32_t hint_ns;
+};
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
+  if (hint_ns)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait for the phase with the given parity: false after ws.limit clock cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, WaitSpec ws) {
+  if (mbar_try_wait(bar, parity, ws.hint_ns)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+  while (!mbar_try_wait(bar, parity, ws.hint_ns)) {
+    if (clock64() - t0 > ws.limit) return false;
   }
   return true;
 }
 
 // Bounded wait that also gives up as soon as another warp of the block has flagged an abort.
-__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                   WaitSpec ws) {
+  if (mbar_try_wait(bar, parity, ws.hint_ns)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait(bar, parity, ws.hint_ns)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > ws.limit) return false;
   }
   return true;
 }

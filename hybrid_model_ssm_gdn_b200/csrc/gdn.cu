@@ -99,7 +99,13 @@ constexpr int kBarBytesG = 512;  // mbarriers (29 x 8 B) + armed phases + abort 
 constexpr int kGBG = 3;  // group buffers: the producer loads a unit's group data one unit ahead
 
 // tile source formats
-enum { SRC_F32 = 0, SRC_F16 = 1, SRC_FP4 = 2, SRC_F8 = 3 };
+enum { SRC_F32 = 0, SRC_F16 = 1, SRC_FP4 = 2, SRC_F8 = 3, SRC_FP4D = 4 };
+// two-axis copy: where a tile's column-group scales land in a stage (after the row-block scales)
+constexpr int kColScaleOff = kTileMaxBytes / 2 + 1024;
+// fold scratch of the two-axis copy: column maxima of a tile in three rotating slots, then the tile's
+// column-group steps (read by every consumer warp after a rendezvous)
+constexpr int kCmSlotWords = (kFp4Rows / 16) * kCols;
+constexpr int kCmBytes = 3 * kCmSlotWords * 4 + kCmSlotWords * 4;
 
 template <typename TI>
 __device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 consecutive elements
@@ -131,12 +137,17 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   unsigned char *tabs = smem + kBarBytesG;
   unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
   unsigned char *stages = gbuf + kGBG * lay.gb_bytes;
+  unsigned int *cmx = reinterpret_cast<unsigned int *>(stages + (size_t)NS * lay.stage_bytes);  // two-axis copy only
+  float *kvals = reinterpret_cast<float *>(cmx + 3 * kCmSlotWords);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitSpec ws{a.wait_cycles, a.suspend_ns};
   const int chunks = (a.H + HG - 1) / HG;
   const int units = a.Bt * chunks;
   const bool fp4_read = LP && a.read_mode != RSSM_READ_SAME;
   const bool shared_fp4 = LP && a.read_mode == RSSM_READ_SHARED_NVFP4;
+  const bool fp4d = LP && a.read_mode == RSSM_READ_NVFP4D;
+  const int read_fmt = fp4d ? SRC_FP4D : SRC_FP4;  // format of the read copy
   const bool hp16 = LP && a.hp_mode == RSSM_HP_F16_SR;
   const bool hp8 = LP && a.hp_mode == RSSM_HP_F8_SR;
   const int hp_fmt = hp16 ? SRC_F16 : hp8 ? SRC_F8 : SRC_F32;  // format of the stored checkpoint
@@ -160,6 +171,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (fp4d)
+    for (int q = threadIdx.x; q < 3 * kCmSlotWords; q += blockDim.x) cmx[q] = 0u;
   __syncthreads();
 
   if (warp == kGProducer) {
@@ -228,7 +241,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     // group data of unit u: k records and q of every head, alpha / beta ring rows
     auto issue_group = [&](int u, int gi, Sched &S) -> bool {
       const int gs = gi % kGBG;
-      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGBG) & 1) ^ 1), abort_flag)) return false;
+      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGBG) & 1) ^ 1), abort_flag, ws)) return false;
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       schedule(u, S, reinterpret_cast<int *>(gb));
       __syncwarp();
@@ -293,14 +306,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         const int n_rec = S.n_ring + S.n_new;
         const bool fold = S.m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : hp_fmt)
-                                : (fp4_read ? SRC_FP4 : hp_fmt);
+                                : (fp4_read ? read_fmt : hp_fmt);
+        const bool fp4src = srcfmt == SRC_FP4 || srcfmt == SRC_FP4D;
         for (int tt = 0; tt < S.nh * nrb; ++tt, ++ti) {
           const int i = tt / nrb, t = tt % nrb;
           const int rows = min(kFp4Rows, R - kFp4Rows * t);
           const size_t unit = (size_t)S.b * a.H + S.h0 + i;
           const size_t row_abs = unit * R + (size_t)kFp4Rows * t;  // first state row of the tile
+          const uint32_t cs_bytes = srcfmt == SRC_FP4D ? (uint32_t)((rows + 15) / 16) * kCols : 0u;
           const int s = ti % NS;
-          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag, ws)) {
             ok = false;
             break;
           }
@@ -311,12 +326,13 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           } else if (srcfmt == SRC_F32) tb += rows * kCols * 4;
           else if (srcfmt == SRC_F16) tb += rows * kCols * 2;
           else if (srcfmt == SRC_F8) tb += rows * kCols + 16;
-          else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16;
+          else tb += rows * (kCols / 2) + rows * (kCols / 16) + 16 + cs_bytes;
           if (lane == 0) {
             armed[s] = ti / NS;
             mbar_arrive_expect_tx(&full[s], tb);
           }
           __syncwarp();
+          if (ti == a.withhold) continue;  // test hook: this stage is never filled
           if (lane == 0 && !skp) {
             if (srcfmt == SRC_F32)
               bulk_g2s(st, reinterpret_cast<const float *>(a.hp) + row_abs * kCols, rows * kCols * 4, &full[s], pol_stream);
@@ -327,11 +343,15 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             else
               bulk_g2s(st, a.rq + row_abs * (kCols / 2), rows * (kCols / 2), &full[s], pol_stream);
           }
-          if (lane == 1 && srcfmt == SRC_FP4 && !skp)
+          if (lane == 1 && fp4src && !skp) {
             bulk_g2s(st + kTileMaxBytes / 2, a.rs + row_abs * (kCols / 16), rows * (kCols / 16), &full[s], pol_stream);
-          if (lane == 2 && (srcfmt == SRC_FP4 || srcfmt == SRC_F8) && !skp) {
+            if (cs_bytes)
+              bulk_g2s(st + kColScaleOff, a.rc + (unit * ((R + 15) / 16) + (size_t)t * (kFp4Rows / 16)) * kCols,
+                       cs_bytes, &full[s], pol_stream);
+          }
+          if (lane == 2 && (fp4src || srcfmt == SRC_F8) && !skp) {
             const size_t gi4 = (unit * nrb + t) & ~(size_t)3;   // 16-byte chunk holding the tile scale
-            bulk_g2s(st + lay.st_g, (srcfmt == SRC_FP4 ? a.rg : a.hs) + gi4, 16, &full[s], pol_keep);
+            bulk_g2s(st + lay.st_g, (fp4src ? a.rg : a.hs) + gi4, 16, &full[s], pol_keep);
           }
           if (lane == 3 && S.n_ring)
             bulk_g2s(st + lay.st_v, reinterpret_cast<const unsigned char *>(a.ring_v) + (unit * 2 * L + S.base_e) * vrow,
@@ -361,14 +381,14 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     auto prep_sync = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(psync);
-      const bool ok = mbar_wait_or_abort(psync, (uint32_t)(rdv & 1), abort_flag);
+      const bool ok = mbar_wait_or_abort(psync, (uint32_t)(rdv & 1), abort_flag, ws);
       ++rdv;
       return ok;
     };
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
-      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGBG) & 1), abort_flag) ||
-          !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
+      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGBG) & 1), abort_flag, ws) ||
+          !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag, ws)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -481,10 +501,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     const int row0 = warp * 8;
     const uint64_t pol_wr = policy_evict_first();
     const uint64_t pol_ring = policy_evict_last();
-    int ti = 0, rdv = 0;
+    int ti = 0, rdv = 0, fd = 0;  // fd: fold tiles done (the two-axis copy's scratch slot rotates with it)
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
-      if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+      if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag, ws)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -499,7 +519,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         const unsigned skm = (unsigned)gh[Q_SKIP];
         const bool fold = m > 0;
         const int srcfmt = fold ? (shared_fp4 ? SRC_FP4 : hp_fmt)
-                                : (fp4_read ? SRC_FP4 : hp_fmt);
+                                : (fp4_read ? read_fmt : hp_fmt);
         const float *u0t = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_u0);
         const float *cot = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_coef);
         float *amx = reinterpret_cast<float *>(tabs + lay.tb_amax);  // [2 slots][8 warps], table buffer 0
@@ -510,7 +530,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           const int h = h0 + i;
           const size_t unit = (size_t)b * a.H + h;
           const int s = ti % NS;
-          if (!mbar_wait_or_abort(&full[s], (uint32_t)((ti / NS) & 1), abort_flag)) {
+          if (!mbar_wait_or_abort(&full[s], (uint32_t)((ti / NS) & 1), abort_flag, ws)) {
             if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
             break;
           }
@@ -542,14 +562,51 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               return make_float4(__fmul_rn(e.x, g_tile), __fmul_rn(e.y, g_tile), __fmul_rn(e.z, g_tile),
                                  __fmul_rn(e.w, g_tile));
             }
-            // NVFP4: E2M1 codes times the block step d_b = E4M3 block scale times the tile scale
+            // NVFP4: E2M1 codes times the block step d_b = E4M3 block scale times the tile scale (two-axis
+            // copy: times 2^-8; its column-group step is applied to the vector the row is multiplied with)
             const uint32_t cw = *reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + col / 2);
             const uint32_t sc = st[kTileMaxBytes / 2 + row * (kCols / 16) + col / 16];
-            const float d_b = __fmul_rn(e4m3_to_float(sc), g_tile);
+            const float d_b = __fmul_rn(e4m3_to_float(sc), srcfmt == SRC_FP4D ? 0.00390625f : g_tile);
             const float4 e = e2m1x4_to_float4(cw);
             return make_float4(__fmul_rn(e.x, d_b), __fmul_rn(e.y, d_b), __fmul_rn(e.z, d_b), __fmul_rn(e.w, d_b));
           };
-          if (!fold) {
+          if (NO == 1 && !fold) {
+            // ---------------- non-fold tile, one output: four lanes per row, 32 columns each (chunks rotated by
+            // lane, as in fold tiles), the buffered term split over the four lanes by record; two shuffles
+            // finish the row (rows is a multiple of 8, so a warp's rows are all live or all past the tile)
+            const int qtr = lane & 3;
+            const int row = row0 + (lane >> 2);
+            const int rowg = kFp4Rows * t + row;
+            if (row0 < rows && t_out > 0) {
+              float z0 = 0.f, z1 = 0.f;
+              if (!((skm >> i) & 1u)) {  // a skipped head's checkpoint term is zero
+                const float *uq = u0_h + qtr * 32;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const int ch = (c + lane) & 7;
+                  float4 u4 = *reinterpret_cast<const float4 *>(uq + ch * 4);
+                  if (srcfmt == SRC_FP4D) {  // column-group steps k = E4M3 * g of this row's 16-row group
+                    const float4 c4 = e4m3x4_to_float4(*reinterpret_cast<const uint32_t *>(
+                        st + kColScaleOff + (row >> 4) * kCols + qtr * 32 + ch * 4));
+                    u4.x *= __fmul_rn(c4.x, g_tile); u4.y *= __fmul_rn(c4.y, g_tile);
+                    u4.z *= __fmul_rn(c4.z, g_tile); u4.w *= __fmul_rn(c4.w, g_tile);
+                  }
+                  const float4 s4 = srcfmt == SRC_F32
+                                        ? *reinterpret_cast<const float4 *>(st + (row * kCols + qtr * 32 + ch * 4) * 4)
+                                        : load_row4(row, qtr * 32 + ch * 4);
+                  z0 = fmaf(s4.x, u4.x, z0);
+                  z1 = fmaf(s4.y, u4.y, z1);
+                  z0 = fmaf(s4.z, u4.z, z0);
+                  z1 = fmaf(s4.w, u4.w, z1);
+                }
+              }
+              float z = z0 + z1;
+              for (int r = qtr; r < n_rec; r += 4) z = fmaf(co_h[r], to_f32(vr[r * R + rowg]), z);
+              z += __shfl_xor_sync(0xffffffffu, z, 1);
+              z += __shfl_xor_sync(0xffffffffu, z, 2);
+              if (qtr == 0) a.y[((size_t)b * a.T * a.H + h) * R + rowg] = z;
+            }
+          } else if (!fold) {
             // ---------------- non-fold tile: lane owns columns 4l..4l+3 of the warp's 8 rows
             if (row0 < rows) {
               constexpr int V = 8 * NO;
@@ -559,6 +616,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
 #pragma unroll
               for (int j = 0; j < NO; ++j)
                 uv[j] = (j < t_out) ? *reinterpret_cast<const float4 *>(u0_h + j * kCols + 4 * lane) : make_float4(0, 0, 0, 0);
+              if (srcfmt == SRC_FP4D) {  // column-group steps k = E4M3 * g of this warp's 16-row group
+                const float4 c4 = e4m3x4_to_float4(
+                    *reinterpret_cast<const uint32_t *>(st + kColScaleOff + (row0 >> 4) * kCols + 4 * lane));
+                const float4 k4 = make_float4(__fmul_rn(c4.x, g_tile), __fmul_rn(c4.y, g_tile), __fmul_rn(c4.z, g_tile),
+                                              __fmul_rn(c4.w, g_tile));
+#pragma unroll
+                for (int j = 0; j < NO; ++j) {
+                  uv[j].x *= k4.x; uv[j].y *= k4.y; uv[j].z *= k4.z; uv[j].w *= k4.w;
+                }
+              }
               float4 sv[8];
               if ((skm >> i) & 1u) {  // skipped head: the checkpoint term is zero
 #pragma unroll
@@ -685,15 +752,54 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               for (int off = 16; off >= 1; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
               const int slot = rdv & 1;
               if (lane == 0) amx[slot * 8 + warp] = am;
+              if (fp4d) {
+                // two-axis copy: column maxima of each 16-row group into this tile's slot, and the slot of the
+                // fold tile after next cleared (every warp has read it before the previous rendezvous)
+                unsigned int *cm = cmx + (fd % 3) * kCmSlotWords + (row >> 4) * kCols + qtr * 32;
+                if (live) {
+#pragma unroll
+                  for (int c = 0; c < 8; ++c) {
+                    unsigned int *cc = cm + ((c + lane) & 7) * 4;
+                    atomicMax(cc, __float_as_uint(fabsf(sv[c].x)));
+                    atomicMax(cc + 1, __float_as_uint(fabsf(sv[c].y)));
+                    atomicMax(cc + 2, __float_as_uint(fabsf(sv[c].z)));
+                    atomicMax(cc + 3, __float_as_uint(fabsf(sv[c].w)));
+                  }
+                }
+                unsigned int *cz = cmx + ((fd + 1) % 3) * kCmSlotWords;
+                for (int q = warp * 32 + lane; q < kCmSlotWords; q += kConsumers) cz[q] = 0u;
+                __threadfence_block();
+              }
               __syncwarp();
               if (lane == 0) mbar_arrive(fsync);  // every consumer warp has posted its maximum
-              if (!mbar_wait_or_abort(fsync, (uint32_t)(rdv & 1), abort_flag)) {
+              if (!mbar_wait_or_abort(fsync, (uint32_t)(rdv & 1), abort_flag, ws)) {
                 if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
                 break;
               }
               ++rdv;
 #pragma unroll
               for (int w = 0; w < kConsumerWarps; ++w) tmax = fmaxf(tmax, amx[slot * 8 + w]);
+              if (fp4d) {
+                // the column-group steps k = E4M3 * g (two per thread) and their codes; every warp reads the
+                // steps after a second rendezvous
+                const unsigned int *cm = cmx + (fd % 3) * kCmSlotWords;
+                const float g = nvfp4_tile_scale(tmax);
+                unsigned char *rcd = a.rc + (unit * ((R + 15) / 16) + (size_t)t * (kFp4Rows / 16)) * kCols;
+                for (int q = warp * 32 + lane; q < ((rows + 15) >> 4) * kCols; q += kConsumers) {
+                  float k;
+                  rcd[q] = (unsigned char)nvfp4d_col_scale(__uint_as_float(cm[q]), g, &k);
+                  kvals[q] = k;
+                }
+                ++fd;
+                __threadfence_block();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(fsync);
+                if (!mbar_wait_or_abort(fsync, (uint32_t)(rdv & 1), abort_flag, ws)) {
+                  if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+                  break;
+                }
+                ++rdv;
+              }
             }
             // write the new state in the checkpoint format: each lane puts its values back where it
             // read them in the stage, then one bulk store per warp moves the warp's rows (contiguous
@@ -748,6 +854,17 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             if (fp4_read) {
               const float g = nvfp4_tile_scale(tmax);
               if (warp == 0 && lane == 0) a.rg[unit * nrb + t] = g;
+              if (live && fp4d) {  // two-axis copy: the blocks are formed on x' = x / k
+                const float *kr = kvals + (row >> 4) * kCols + qtr * 32;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const float4 k4 = *reinterpret_cast<const float4 *>(kr + ((c + lane) & 7) * 4);
+                  sv[c].x = k4.x > 0.f ? __fdiv_rn(sv[c].x, k4.x) : 0.f;
+                  sv[c].y = k4.y > 0.f ? __fdiv_rn(sv[c].y, k4.y) : 0.f;
+                  sv[c].z = k4.z > 0.f ? __fdiv_rn(sv[c].z, k4.z) : 0.f;
+                  sv[c].w = k4.w > 0.f ? __fdiv_rn(sv[c].w, k4.w) : 0.f;
+                }
+              }
               if (live) {
                 // this lane's 32 columns are blocks qtr*2 and qtr*2+1; chunk ch lies in block ch >> 2
                 float bam0 = 0.f, bam1 = 0.f;
@@ -758,7 +875,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                   if (ch < 4) bam0 = fmaxf(bam0, mq); else bam1 = fmaxf(bam1, mq);
                 }
                 float db0, db1;
-                const uint32_t sc0 = nvfp4_block_scale(bam0, g, &db0), sc1 = nvfp4_block_scale(bam1, g, &db1);
+                const uint32_t sc0 = fp4d ? nvfp4d_block_scale(bam0, &db0) : nvfp4_block_scale(bam0, g, &db0);
+                const uint32_t sc1 = fp4d ? nvfp4d_block_scale(bam1, &db1) : nvfp4_block_scale(bam1, g, &db1);
                 *reinterpret_cast<uint16_t *>(a.rs + (unit * R + rowg) * (kCols / 16) + qtr * 2) =
                     (uint16_t)(sc0 | (sc1 << 8));
                 unsigned char *cd = a.rq + (unit * R + rowg) * (kCols / 2) + qtr * 16;
@@ -790,9 +908,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
     for (int s = 0; s < 8; ++s)
-      if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1));
+      if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1), ws);
     for (int s = 0; s < kGBG; ++s)
-      if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
+      if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1), ws);
   }
   if (threadIdx.x == 0) sched_finish(a.err);
 }
@@ -810,6 +928,8 @@ int g_max_stages(int R, int L, int tmax, int esz, int budget) {
   return n;
 }
 
+int g_extra_smem_bytes(int read_mode) { return read_mode == RSSM_READ_NVFP4D ? kCmBytes : 0; }
+
 int g_units(int Bt, int H, int tmax) {
   const int no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
   const int hg = g_heads_per_unit(no);
@@ -818,7 +938,7 @@ int g_units(int Bt, int H, int tmax) {
 
 cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream) {
   const int no = a.tmax <= 1 ? 1 : a.tmax <= 2 ? 2 : a.tmax <= 4 ? 4 : 8;
-  const size_t smem = g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage);
+  const size_t smem = g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) + g_extra_smem_bytes(a.read_mode);
   void (*kern)(GArgs) = nullptr;
   const bool lp = a.hp_mode != RSSM_HP_F32 || a.read_mode != RSSM_READ_SAME;
 #define RSSM_PICK(TI, NOV) \

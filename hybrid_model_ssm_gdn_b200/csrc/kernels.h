@@ -25,6 +25,11 @@ struct M2Args {
   const unsigned char *mask;      // flush only, may be null
   const float *A, *D;
   float *y;                       // [Bt][T][H][P]
+  unsigned char *skip;            // decay-aware skip flags [Bt][H], or null when skipping is off
+  float skip_ln_tau;              // flag threshold on A_h times the sum of dt over the committed records
+  long long wait_cycles;          // bound of every wait on an asynchronous copy or another warp
+  unsigned int suspend_ns;        // suspend-time hint of each try_wait (0: the hardware's default)
+  int withhold;                   // test hook: no block fills its tile with this index (-1: off)
 };
 int m2_smem_bytes(int P, int L, int tmax, int esz, int nstage);
 int m2_max_stages(int P, int L, int tmax, int esz, int smem_budget);
@@ -45,6 +50,7 @@ struct GArgs {
   float *hs;                      // E4M3 checkpoint tile scales [Bt][H][ceil(DV/64)]
   unsigned char *rq, *rs;         // NVFP4 codes [Bt][H][DV][64], scales [Bt][H][DV][8]
   float *rg;                      // tile scales [Bt][H][ceil(DV/64)]
+  unsigned char *rc;              // two-axis copy: column-group scales [Bt][H][ceil(DV/16)][128]
   unsigned char *skip;            // decay-aware skip flags [Bt][H], or null when skipping is off
   float skip_tau;                 // flag threshold on the product of alpha over the committed records
   void *ring_k, *ring_v;          // input dtype [Bt][H][2L][128], [Bt][H][2L][DV]
@@ -53,8 +59,12 @@ struct GArgs {
   const float *alpha, *beta;      // [Bt][T][H]
   const unsigned char *mask;
   float *y;                       // [Bt][T][H][DV]
+  long long wait_cycles;          // bound of every wait on an asynchronous copy or another warp
+  unsigned int suspend_ns;        // suspend-time hint of each try_wait (0: the hardware's default)
+  int withhold;                   // test hook: no block fills its tile with this index (-1: off)
 };
 int g_smem_bytes(int R, int L, int tmax, int esz, int nstage);
+int g_extra_smem_bytes(int read_mode);  // fold scratch of the two-axis read copy
 int g_max_stages(int R, int L, int tmax, int esz, int budget);
 int g_units(int Bt, int H, int tmax);  // work units: (sequence, chunk of heads)
 cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream);
@@ -67,8 +77,8 @@ cudaError_t launch_export_meta(const int4 *meta, int *out, int Bt, int L, cudaSt
 cudaError_t launch_gather_window(const unsigned char *in, unsigned char *out, const int4 *meta, int Bt, int X,
                                  size_t in_group_bytes, int slot_bytes, int L, cudaStream_t stream);
 cudaError_t launch_store_state(const float *S, void *hp, float *hs, int hp_mode, unsigned char *rq, unsigned char *rs,
-                               float *rg, int read_mode, int units, int rows, unsigned long long seed, int H,
-                               cudaStream_t stream);
+                               float *rg, unsigned char *rc, int read_mode, int units, int rows, unsigned long long seed,
+                               int H, cudaStream_t stream);
 cudaError_t launch_widen_state(const void *hp, const float *hs, int hp_mode, const unsigned char *rq,
                                const unsigned char *rs, const float *rg, int read_mode, float *out, int units, int rows,
                                cudaStream_t stream);

@@ -11,7 +11,7 @@ namespace rssm {
 namespace {
 
 __global__ void store_state_kernel(const float *S, void *hp, float *hs, int hp_mode, unsigned char *rq,
-                                   unsigned char *rs, float *rg, int read_mode, int rows_per_head,
+                                   unsigned char *rs, float *rg, unsigned char *rc, int read_mode, int rows_per_head,
                                    unsigned long long seed) {
   const int nrb = (rows_per_head + kFp4Rows - 1) / kFp4Rows;
   const size_t unit = blockIdx.x / nrb;
@@ -64,6 +64,41 @@ __global__ void store_state_kernel(const float *S, void *hp, float *hs, int hp_m
   if (read_mode == RSSM_READ_SAME) return;
   const float g = nvfp4_tile_scale(tmax);
   if (row == 0) rg[unit * nrb + t] = g;
+  if (read_mode == RSSM_READ_NVFP4D) {
+    // column maxima per group of 16 rows, the column-group steps k, then NVFP4 blocks of x / k
+    __shared__ unsigned int cmax[kFp4Rows / 16][kCols];
+    __shared__ float kst[kFp4Rows / 16][kCols];
+    for (int q = row; q < kFp4Rows / 16 * kCols; q += kFp4Rows) cmax[q / kCols][q % kCols] = 0u;
+    __syncthreads();
+    if (live)
+      for (int c = 0; c < kCols; ++c) atomicMax(&cmax[row >> 4][c], __float_as_uint(fabsf(src[c])));
+    __syncthreads();
+    const int ngr = (rows_per_head + 15) / 16, ngr_t = (rows + 15) / 16;
+    for (int q = row; q < ngr_t * kCols; q += kFp4Rows) {
+      float k;
+      const uint32_t code = nvfp4d_col_scale(__uint_as_float(cmax[q / kCols][q % kCols]), g, &k);
+      kst[q / kCols][q % kCols] = k;
+      rc[(unit * ngr + (size_t)t * (kFp4Rows / 16)) * kCols + q] = (unsigned char)code;
+    }
+    __syncthreads();
+    if (!live) return;
+    const float *kr = kst[row >> 4];
+    for (int blk = 0; blk < kCols / 16; ++blk) {
+      float xv[16], bam = 0.f;
+      for (int c = 0; c < 16; ++c) {
+        const float k = kr[blk * 16 + c];
+        xv[c] = k > 0.f ? __fdiv_rn(src[blk * 16 + c], k) : 0.f;
+        bam = fmaxf(bam, fabsf(xv[c]));
+      }
+      float d_b;
+      rs[(unit * rows_per_head + rowg) * (kCols / 16) + blk] = (unsigned char)nvfp4d_block_scale(bam, &d_b);
+      for (int c = 0; c < 16; c += 2) {
+        const uint32_t lo = nvfp4_code(xv[c], d_b), hi = nvfp4_code(xv[c + 1], d_b);
+        rq[(unit * rows_per_head + rowg) * (kCols / 2) + (blk * 16 + c) / 2] = (unsigned char)(lo | (hi << 4));
+      }
+    }
+    return;
+  }
   if (!live) return;
   for (int blk = 0; blk < kCols / 16; ++blk) {
     float bam = 0.f;
@@ -113,10 +148,10 @@ __global__ void widen_state_kernel(const void *hp, const float *hs, int hp_mode,
 }  // namespace
 
 cudaError_t launch_store_state(const float *S, void *hp, float *hs, int hp_mode, unsigned char *rq, unsigned char *rs,
-                               float *rg, int read_mode, int units, int rows, unsigned long long seed, int /*H*/,
-                               cudaStream_t stream) {
+                               float *rg, unsigned char *rc, int read_mode, int units, int rows, unsigned long long seed,
+                               int /*H*/, cudaStream_t stream) {
   const int nrb = (rows + kFp4Rows - 1) / kFp4Rows;
-  store_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(S, hp, hs, hp_mode, rq, rs, rg,
+  store_state_kernel<<<(unsigned)((size_t)units * nrb), kFp4Rows, 0, stream>>>(S, hp, hs, hp_mode, rq, rs, rg, rc,
                                                                                  read_mode, rows, seed);
   return cudaGetLastError();
 }

@@ -18,6 +18,10 @@
 // * NVFP4 tile (64 consecutive rows x 128 columns of one head's state), blocks of 16
 //   columns: g = amax(tile)/2688 (1 if amax = 0); s_b = E4M3(amax_b / (6 g));
 //   d_b = s_b g; code = sign | E2M1(|x| / d_b) (all zero if s_b = 0); value = E2M1 * d_b.
+// * Two-axis NVFP4 tile (separate scales along the channel and state axes): g as above;
+//   per column and group of 16 rows c = E4M3(amax_group / (6 g)), step k = c g;
+//   x' = x / k (0 where k = 0); per row block s_b = E4M3(amax_b(x') / (6 * 2^-8)),
+//   d_b = s_b * 2^-8; code = sign(x') | E2M1(|x'| / d_b); value = (E2M1 * d_b) * k.
 // * Random words: Philox4x32-10 (Salmon, Moraes, Dror & Shaw, SC'11), counter
 //   (sequence*H + head, epoch written, element/4, 0), key = the 64-bit seed; element e
 //   uses output word e % 4.
@@ -189,6 +193,20 @@ __device__ __forceinline__ uint32_t nvfp4_code(float x, float d_b) {
   if (d_b == 0.f) return 0u;
   const uint32_t idx = e2m1_index(__fdiv_rn(fabsf(x), d_b));
   return idx | (x < 0.f ? 8u : 0u);
+}
+
+// Two-axis copy: column-group scale code and step k = c * g from the group's largest magnitude.
+__device__ __forceinline__ uint32_t nvfp4d_col_scale(float amax_grp, float g, float *k) {
+  const float c = e4m3_round(__fdiv_rn(amax_grp, __fmul_rn(6.f, g)));
+  *k = __fmul_rn(c, g);
+  return e4m3_code(c);
+}
+
+// Two-axis copy: row-block scale code and block step d_b = s_b * 2^-8 (exact) of the divided values.
+__device__ __forceinline__ uint32_t nvfp4d_block_scale(float amax_b, float *d_b) {
+  const float sb = e4m3_round(__fdiv_rn(amax_b, 0.0234375f));   // 6 * 2^-8
+  *d_b = sb * 0.00390625f;
+  return e4m3_code(sb);
 }
 
 __device__ __forceinline__ float nvfp4_value(uint32_t code, float d_b) {

@@ -47,7 +47,7 @@ constexpr int kGHdr = 1024;      // group header bytes
 // group header: ints then floats
 enum {
   G_ACTIVE = 0, G_NREC, G_M, G_NRING, G_NNEW, G_TOUT, G_SLOT0, G_MC, G_ME, G_MP, G_B, G_G, G_H0, G_NH,
-  G_BASE, G_WMETA, G_WB, G_END,
+  G_BASE, G_WMETA, G_WB, G_SKIP, G_END,  // G_SKIP: bit i set = head h0 + i skips its checkpoint read
   G_A = 32,                  // floats: A[16]
   G_D = G_A + kHG,           // D[16]
   G_DT = G_D + kHG           // dt of new tokens [8][16]
@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitSpec ws{a.wait_cycles, a.suspend_ns};
   const int hpg = a.H / a.G;
   const int chunks = (hpg + kHG - 1) / kHG;
   const int units = a.Bt * a.G * chunks;
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     const int L = a.L, dts = dt_stride(L);
     struct Sched {
       int b, g, h0, nh, active, n_ring, n_new, m, t_out, slot0, base_e;
+      unsigned skip;
     };
     // schedule of unit u (identical for every head of the sequence) from the sequence's
     // bookkeeping word; u >= units writes the end marker
@@ -172,11 +174,14 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       const int b = u / (a.G * chunks), g = (u / chunks) % a.G, ch = u % chunks;
       S.b = b; S.g = g; S.h0 = g * hpg + ch * kHG; S.nh = min(kHG, hpg - ch * kHG);
       int4 mw = make_int4(0, 0, 0, 0);
-      int mk = 1;
+      int mk = 1, fl = 0;
       if (lane == 0) {
         mw = a.meta_in[b];
         mk = (a.mask == nullptr) ? 1 : (int)a.mask[b];
       }
+      // skip flags left by the previous call, loaded beside the bookkeeping word
+      if (a.skip != nullptr && lane < S.nh) fl = a.skip[(size_t)b * a.H + S.h0 + lane];
+      const unsigned skm = __ballot_sync(0xffffffffu, fl != 0);
       const int c = __shfl_sync(0xffffffffu, mw.x, 0), e = __shfl_sync(0xffffffffu, mw.y, 0);
       const int pend = __shfl_sync(0xffffffffu, mw.z, 0), msk = __shfl_sync(0xffffffffu, mk, 0);
       int active = 1, n_ring = 0, n_new = 0, m = 0, t_out = 0, slot0 = 0;
@@ -205,17 +210,18 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       }
       S.active = active; S.n_ring = n_ring; S.n_new = n_new; S.m = m; S.t_out = t_out; S.slot0 = slot0;
       S.base_e = base_e;
+      S.skip = active ? skm : 0u;
       if (lane == 0) {
         hdr[G_ACTIVE] = active; hdr[G_NREC] = n_ring + n_new; hdr[G_M] = m; hdr[G_NRING] = n_ring;
         hdr[G_NNEW] = n_new; hdr[G_TOUT] = t_out; hdr[G_SLOT0] = slot0; hdr[G_MC] = mc; hdr[G_ME] = me;
         hdr[G_MP] = mp; hdr[G_B] = b; hdr[G_G] = g; hdr[G_H0] = S.h0; hdr[G_NH] = S.nh; hdr[G_BASE] = base_e;
-        hdr[G_WMETA] = (S.h0 == 0); hdr[G_WB] = (ch == 0); hdr[G_END] = 0;
+        hdr[G_WMETA] = (S.h0 == 0); hdr[G_WB] = (ch == 0); hdr[G_SKIP] = (int)S.skip; hdr[G_END] = 0;
       }
     };
     // group data of unit u into buffer gi % kGB (B records, B and C of the new tokens, dt rows)
     auto issue_group = [&](int u, int gi, Sched &S) -> bool {
       const int gs = gi % kGB;
-      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGB) & 1) ^ 1), abort_flag)) return false;
+      if (!mbar_wait_or_abort(&gempty[gs], (uint32_t)(((gi / kGB) & 1) ^ 1), abort_flag, ws)) return false;
       unsigned char *gb = gbuf + (size_t)gs * lay.gb_bytes;
       schedule(u, S, reinterpret_cast<int *>(gb));
       __syncwarp();
@@ -268,10 +274,12 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
       const Sched S = Sc;
       if (S.active) {
         const int n_rec = S.n_ring + S.n_new;
-        const uint32_t tbytes = (uint32_t)lay.tile_bytes + n_rec * xrow;
         for (int i = 0; i < S.nh; ++i, ++ti) {
+          const bool skp = (S.skip >> i) & 1u;  // decay-aware skip: no checkpoint tile for this head
+          const bool hold = ti == a.withhold;  // test hook: this stage is never filled
+          const uint32_t tbytes = (skp ? 0u : (uint32_t)lay.tile_bytes) + n_rec * xrow;
           const int s = ti % NS;
-          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag)) {
+          if (!mbar_wait_or_abort(&empty[s], (uint32_t)(((ti / NS) & 1) ^ 1), abort_flag, ws)) {
             ok = false;
             break;
           }
@@ -282,7 +290,8 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
             mbar_arrive_expect_tx(&full[s], tbytes);
           }
           __syncwarp();
-          if (lane == 0) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
+          if (hold) continue;
+          if (lane == 0 && !skp) bulk_g2s(st, a.hp + unit * a.P * kCols, lay.tile_bytes, &full[s], pol_stream);
           if (lane == 1 && S.n_ring)
             bulk_g2s(st + lay.xr, reinterpret_cast<const unsigned char *>(a.ring_x) + (unit * 2 * L + S.base_e) * xrow,
                      S.n_ring * xrow, &full[s], pol_keep);
@@ -306,8 +315,8 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     // ================================================================== prep warp
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGB, tsl = gi & 1;
-      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGB) & 1), abort_flag) ||
-          !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag)) {
+      if (!mbar_wait_or_abort(&gfull[gs], (uint32_t)((gi / kGB) & 1), abort_flag, ws) ||
+          !mbar_wait_or_abort(&tempty[tsl], (uint32_t)(((gi >> 1) & 1) ^ 1), abort_flag, ws)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -478,6 +487,14 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
             T.ao[i * NO + j] = __expf(A * sfx);
           }
         }
+        if (a.skip != nullptr && lane < nh) {
+          // skip flag for the next call: A_h times the fp32 sum of dt, in record order, over the records
+          // committed after this call (records m.. ; a verify's drafts are not committed)
+          const int n_comm = a.op == OP_VERIFY ? n_ring : n_rec;
+          float sdt = 0.f;
+          for (int r = m; r < n_comm; ++r) sdt = __fadd_rn(sdt, dt_of(lane, r));
+          a.skip[(size_t)b * a.H + h0 + lane] = __fmul_rn(gf[G_A + lane], sdt) < a.skip_ln_tau ? 1 : 0;
+        }
         if (m > 0 && lane < nh) {
           const int i = lane;
           const float A = gf[G_A + i];
@@ -500,7 +517,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     int ti = 0;
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGB, tsl = gi & 1;
-      if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag)) {
+      if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag, ws)) {
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
       }
@@ -513,6 +530,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         const float *t_coef = T.coef, *t_ao = T.ao, *t_wf = T.wf, *t_af = T.af;
         const int n_rec = gh[G_NREC], m = gh[G_M], t_out = gh[G_TOUT];
         const int n_ring = gh[G_NRING], n_new = gh[G_NNEW], slot0 = gh[G_SLOT0];
+        const unsigned skm = (unsigned)gh[G_SKIP];
         const TI *Bg = reinterpret_cast<const TI *>(gb + lay.gb_B);
         const TI *Cg = reinterpret_cast<const TI *>(gb + lay.gb_C);
         // ---- stream the heads' tiles; each warp works and releases on its own
@@ -538,7 +556,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
         constexpr int SPREAD = V >= 32 ? 1 : 32 / V;
         for (int i = 0; i < nh; ++i, ++ti) {
           const int s = ti % NS;
-          if (!mbar_wait_or_abort(&full[s], (uint32_t)((ti / NS) & 1), abort_flag)) {
+          if (!mbar_wait_or_abort(&full[s], (uint32_t)((ti / NS) & 1), abort_flag, ws)) {
             if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
             break;
           }
@@ -558,10 +576,14 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
             bulk_commit();
           }
           if (row0 < a.P) {
+            // a head flagged for decay-aware skipping has no tile in the stage: its checkpoint term is zero
+            const bool skp = (skm >> i) & 1u;
             float4 sv[8];
             if (!kMma || m > 0) {
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) sv[rr] = *reinterpret_cast<const float4 *>(tile + (row0 + rr) * kCols + 4 * lane);
+            for (int rr = 0; rr < 8; ++rr)
+              sv[rr] = skp ? make_float4(0.f, 0.f, 0.f, 0.f)
+                           : *reinterpret_cast<const float4 *>(tile + (row0 + rr) * kCols + 4 * lane);
             }
             if (m > 0) {
               const float af = t_af[i];
@@ -614,13 +636,15 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
                 const int g = lane >> 2, t4 = lane & 3;
                 float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
                 const float *srow = tile + (row0 + g) * kCols + 4 * t4;
+                if (!skp || m > 0) {  // a skipped head's folded rows were written back into the stage
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                  const float4 v = *reinterpret_cast<const float4 *>(srow + 16 * c);
-                  uint32_t h0, l0, h1, l1;
-                  split_bf16x2(v.x, v.y, h0, l0);
-                  split_bf16x2(v.z, v.w, h1, l1);
-                  mma_16816((c & 1) ? d1 : d0, h0, l0, h1, l1, ac[c][0], ac[c][1]);
+                  for (int c = 0; c < 8; ++c) {
+                    const float4 v = *reinterpret_cast<const float4 *>(srow + 16 * c);
+                    uint32_t h0, l0, h1, l1;
+                    split_bf16x2(v.x, v.y, h0, l0);
+                    split_bf16x2(v.z, v.w, h1, l1);
+                    mma_16816((c & 1) ? d1 : d0, h0, l0, h1, l1, ac[c][0], ac[c][1]);
+                  }
                 }
                 float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint4 *cf = reinterpret_cast<const uint4 *>(t_coef) + (size_t)i * lay.nq * 32;
@@ -693,9 +717,9 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   if (*abort_flag && threadIdx.x == 0) {
     // do not leave bulk copies in flight into the shared memory of an exiting block
     for (int s = 0; s < 8; ++s)
-      if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1));
+      if (armed[s] >= 0) mbar_wait(&full[s], (uint32_t)(armed[s] & 1), ws);
     for (int s = 0; s < kGB; ++s)
-      if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1));
+      if (armed[8 + s] >= 0) mbar_wait(&gfull[s], (uint32_t)(armed[8 + s] & 1), ws);
   }
   if (threadIdx.x == 0) sched_finish(a.err);
 }

@@ -80,9 +80,12 @@ typedef enum { RSSM_F32 = 0, RSSM_BF16 = 1 } rssm_dtype;
  * times one fp32 scale amax/448 per 64-row tile of a head's state, rounded stochastically with
  * the same random words (GDN only) */
 typedef enum { RSSM_HP_F32 = 0, RSSM_HP_F16_SR = 1, RSSM_HP_F8_SR = 2 } rssm_hp;
-/* copy read for outputs: the checkpoint itself, a separate NVFP4 copy, or (contrast
- * only) one NVFP4 copy that is also the checkpoint the recurrence continues from */
-typedef enum { RSSM_READ_SAME = 0, RSSM_READ_NVFP4 = 1, RSSM_READ_SHARED_NVFP4 = 2 } rssm_read;
+/* copy read for outputs: the checkpoint itself, a separate NVFP4 copy, (contrast only) one
+ * NVFP4 copy that is also the checkpoint the recurrence continues from, or a separate NVFP4
+ * copy with scales along both axes ([HMD] Interpretation 4th paragraph: separate scales along
+ * the state and channel dimensions): an E4M3 scale per column for every 16 rows of a tile,
+ * times the E4M3 block scales along each row (GDN only) */
+typedef enum { RSSM_READ_SAME = 0, RSSM_READ_NVFP4 = 1, RSSM_READ_SHARED_NVFP4 = 2, RSSM_READ_NVFP4D = 3 } rssm_read;
 
 typedef struct {
   int kind;        /* rssm_kind */
@@ -203,6 +206,13 @@ rssm_status rssm_export(rssm_ctx *ctx, float *S_out, void *ring_out, int *meta_o
  * RSSM_ERR_UNSUPPORTED if the context has no read copy. */
 rssm_status rssm_export_read_copy(rssm_ctx *ctx, unsigned char *codes, unsigned char *scales, float *g,
                                   rssm_stream stream);
+
+/* Copy the column-group scales of a two-axis read copy (RSSM_READ_NVFP4D) out: colscales uint8
+ * [Bt][H][ceil(rows/16)][128] (device), the E4M3 scale of each column for each group of 16 rows;
+ * rssm_export_read_copy gives its codes, row-block scales and tile scales (the row-block scale of
+ * this copy is d_b = E4M3 * 2^-8, in units of the column-group step E4M3 * g).
+ * RSSM_ERR_UNSUPPORTED for any other read mode. */
+rssm_status rssm_export_column_scales(rssm_ctx *ctx, unsigned char *colscales, rssm_stream stream);
 
 /* Copy the decay-aware skip flags out: flags uint8 [Bt][H] (device), 1 = the next call skips
  * that head's checkpoint read.  RSSM_ERR_UNSUPPORTED if the context has skip_tau == 0. */

@@ -47,23 +47,35 @@ rounding, random words from Philox4x32-10 with counter (sequence*H + head,
 new epoch, element/4, 0) and the 64-bit seed as key) or "f8sr" (E4M3 with a
 per-64-row-tile scale and the same stochastic rounding); read = "same" (outputs
 read the checkpoint), "nvfp4" (separate NVFP4 read copy, re-quantised from the
-fp32 fold result at every fold) or "shared_nvfp4" (the NVFP4 copy is also the
-checkpoint the recurrence continues from; contrast mode).  The NVFP4 copy is
-quantised tile by tile, a tile being 64 consecutive rows of one head's state.
+fp32 fold result at every fold), "nvfp4d" (the same with two-axis scales:
+column-group scales along the channel axis and block scales along the state
+axis, see lowprec) or "shared_nvfp4" (the NVFP4 copy is also the checkpoint
+the recurrence continues from; contrast mode).  The copies are quantised tile
+by tile, a tile being 64 consecutive rows of one head's state.
 
-Decay-aware read skipping (GDN, ``skip_tau`` > 0): a head whose gates over
-the buffered inputs have multiplied down below a threshold may skip reading
-the checkpoint, which then counts as zero; a fold of such a head writes the
-new checkpoint from the buffer alone ("SSM decoding stops writing state every
-step", Perspective, first paragraph, names this as the next step and fixes
-no rule).  Reading taken: after each step, verify or flush, a head's flag is
-set iff the product of alpha over the committed records of the current
-window, taken in fp32 in record order, is below ``skip_tau``; the next call
-reads that flag.  The product only falls as records are added, so the
-skipped term S0 u0 of any later output has norm at most
-skip_tau * ||S0|| * q_scale * ||q|| (each (I - beta k k^T) has norm <= 1 for
-||k|| = 1, 0 <= beta <= 2).  Commit leaves the flags alone; a fold that empties
-the window clears them.
+Decay-aware read skipping (``skip_tau`` > 0): a head whose decay over the
+buffered inputs has fallen below a threshold may skip reading the checkpoint,
+which then counts as zero; a fold of such a head writes the new checkpoint
+from the buffer alone ("SSM decoding stops writing state every step",
+Perspective, first paragraph, names this as a next step for heads whose decay
+is negligible, and fixes no rule).  Reading taken: after
+each step, verify or flush, a head's flag is set from the committed records of
+the current window, and the next call reads it:
+
+* GDN: iff the product of alpha over those records, taken in fp32 in record
+  order, is below ``skip_tau``.  The product only falls as records are added,
+  so the skipped term S0 u0 of any later output has norm at most
+  skip_tau * ||S0|| * q_scale * ||q|| (each (I - beta k k^T) has norm <= 1 for
+  ||k|| = 1, 0 <= beta <= 2).
+* Mamba-2: iff A_h * s < ln(skip_tau), with s the fp32 sum of dt over those
+  records in record order, the product A_h * s taken in fp32, and ln(skip_tau)
+  the double-precision natural log of the fp32 threshold rounded once to fp32.
+  Then the product of dA = exp(dt A_h) over the records is exp(A_h s) <
+  skip_tau up to that rounding, and it only falls as records are added (A_h <
+  0 < dt), so the skipped term exp(A_h s(m, e)) S0 C of any later output has
+  norm at most about skip_tau * ||S0|| * ||C||.
+
+Commit leaves the flags alone; a fold that empties the window clears them.
 
 Two outputs are produced per call: ``y`` mirrors the method (folds at the
 points above, state rounded to its stored formats, replay in float64) and
@@ -73,6 +85,8 @@ floating-point differences; the tests check it.
 """
 
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
@@ -98,8 +112,8 @@ class ReplayOracle:
     def __init__(self, kind, S0, window, *, nheads, ngroups=1, params=None, seq_ids=None, head_ids=None,
                  hp="f32", read="same", seed=0, q_scale=1.0, skip_tau=0.0):
         assert kind in ("mamba2", "gdn")
-        assert skip_tau >= 0 and (skip_tau == 0 or kind == "gdn")
-        assert hp in ("f32", "f16sr", "f8sr") and read in ("same", "nvfp4", "shared_nvfp4")
+        assert skip_tau >= 0
+        assert hp in ("f32", "f16sr", "f8sr") and read in ("same", "nvfp4", "nvfp4d", "shared_nvfp4")
         self.kind, self.L, self.H, self.G = kind, int(window), int(nheads), int(ngroups)
         S0 = np.asarray(S0, np.float64)
         self.nb = S0.shape[0]
@@ -115,6 +129,7 @@ class ReplayOracle:
         self.q_scale = float(q_scale)
         self.hp_mode, self.read_mode, self.seed = hp, read, int(seed)
         self.skip_tau = np.float32(skip_tau)
+        self.ln_tau = np.float32(math.log(float(self.skip_tau))) if skip_tau > 0 else np.float32(0)
 
         self.S_true = S0.copy()
         self.count = np.zeros(self.nb, np.int64)
@@ -170,15 +185,25 @@ class ReplayOracle:
         return np.where(self.skip[b][:, None, None], 0.0, S)
 
     def _update_skip(self, b):
-        """Flags for the next call: fp32 product of alpha over the committed records, in order, < skip_tau."""
+        """Flags for the next call from the committed records, in order: GDN, fp32 product of alpha < skip_tau;
+        Mamba-2, A_h times the fp32 sum of dt < ln(skip_tau), in fp32."""
         if self.skip_tau <= 0:
             return
-        prod = np.ones(self.nh, np.float32)
-        for rec in self.ring[b][: self.count[b]]:
-            prod = (prod * np.asarray(rec["alpha"], np.float32)).astype(np.float32)
-        self.skip[b] = prod < self.skip_tau
+        recs = self.ring[b][: self.count[b]]
+        if self.kind == "gdn":
+            prod = np.ones(self.nh, np.float32)
+            for rec in recs:
+                prod = (prod * np.asarray(rec["alpha"], np.float32)).astype(np.float32)
+            self.skip[b] = prod < self.skip_tau
+            return
+        s = np.zeros(self.nh, np.float32)
+        for rec in recs:
+            s = (s + np.asarray(rec["dt"], np.float32)).astype(np.float32)
+        self.skip[b] = (self.A.astype(np.float32) * s).astype(np.float32) < self.ln_tau
 
     def _read_copy(self, S32):
+        if self.read_mode == "nvfp4d":
+            return lowprec.nvfp4d_roundtrip_state(S32).astype(np.float64)
         return lowprec.nvfp4_roundtrip_state(S32).astype(np.float64)
 
     def _store(self, b, S_new):

@@ -42,6 +42,31 @@ consecutive elements along the contracted (contiguous) axis:
     d_b = s_b * g                               (fp32)
     q   = E2M1(|x| / d_b) with the sign of x     (fp32 divide); q = 0 if d_b = 0
     dequantised value = value(q) * d_b          (fp32)
+The tile has its own scale rather than one per head state so that a tile holds
+the scale of the rows it covers: a state whose rows differ in magnitude (the
+channels of a head) gets tighter scales, and the two-level scale stays the
+usual NVFP4 layout of a 64 x 128 operand tile.
+
+Two-axis NVFP4 read copy (finer scales: the pages name separate scales along
+the state and channel dimensions as a way to cut the remaining read error,
+"Hybrid-model decoding has a new bottleneck", Interpretation, fourth
+paragraph, and give no format).  Reading taken: one E4M3 scale per column for
+each group of 16 consecutive rows (a scale along the channel axis), then the
+usual E4M3 block scales along each row's 16 consecutive columns (the state
+axis) on the values divided by it:
+    g   = amax(tile) / 2688 in fp32, or 1 if amax = 0   (as for NVFP4)
+    c   = E4M3(amax over the group's rows of |x_ij| / (6 g))   (fp32 product, then fp32 divide)
+    k   = c * g                                         (fp32; the column-group step)
+    x'  = x / k                                         (fp32 divide; 0 where k = 0)
+    s_b = E4M3(amax_b(|x'|) / (6 * 2^-8))               (fp32 divide by an exact constant)
+    d_b = s_b * 2^-8                                    (exact)
+    q   = E2M1(|x'| / d_b) with the sign of x'          (fp32 divide); q = 0 if d_b = 0
+    dequantised value = (value(q) * d_b) * k            (fp32; the first product is exact)
+Each element's step is the product of a scale of its column group and a scale
+of its row block, so a state whose channels differ in magnitude along a column
+no longer shares one block step across them.  A tile of equal magnitudes
+2688 * 2^n round-trips exactly.  The column-group scales add one byte per 16
+elements (the copy grows from 0.5625 to 0.625 bytes per element).
 """
 
 from __future__ import annotations
@@ -238,3 +263,80 @@ def nvfp4_roundtrip_state(S) -> np.ndarray:
     rows = S.shape[-2]
     return np.concatenate([nvfp4_roundtrip(S[..., r0:r0 + NVFP4_TILE_ROWS, :])
                            for r0 in range(0, rows, NVFP4_TILE_ROWS)], axis=-2)
+
+
+# --------------------------------------------------------------------------- two-axis NVFP4 read copy
+
+NVFP4D_GROUP_ROWS = 16
+NVFP4D_BLOCK_STEP = np.float32(2.0 ** -8)
+
+
+def nvfp4d_quantize(tile) -> dict:
+    """Two-axis NVFP4 encoding of fp32 tiles [..., R, C] (R <= 64, C a multiple of 16).  Returns "codes"
+    (unpacked), "packed" [..., R, C/2], "scales" [..., R, C/16] (E4M3 row-block scales), "colscales"
+    [..., ceil(R/16), C] (E4M3 column-group scales) and "g" [...]."""
+    x = np.ascontiguousarray(tile, np.float32)
+    *lead, R, C = x.shape
+    assert C % NVFP4_BLOCK == 0
+    ax = np.abs(x)
+    amax = ax.reshape(*lead, -1).max(axis=-1) if R * C else np.zeros(lead, np.float32)
+    g = np.where(amax > 0, amax / np.float32(2688.0), np.float32(1.0)).astype(np.float32)
+    six_g = (np.float32(6.0) * g).astype(np.float32)
+    ngr = -(-R // NVFP4D_GROUP_ROWS)
+    cs = np.empty(tuple(lead) + (ngr, C), np.float32)
+    k = np.empty_like(x)
+    for gi in range(ngr):
+        rows = slice(gi * NVFP4D_GROUP_ROWS, min(R, (gi + 1) * NVFP4D_GROUP_ROWS))
+        gm = ax[..., rows, :].max(axis=-2)                                   # [..., C]
+        c = e4m3_round((gm / six_g[..., None]).astype(np.float32)).astype(np.float32)
+        cs[..., gi, :] = c
+        k[..., rows, :] = (c * g[..., None]).astype(np.float32)[..., None, :]
+    xp = np.where(k > 0, x / np.where(k > 0, k, np.float32(1.0)), np.float32(0.0)).astype(np.float32)
+    blocks = np.abs(xp).reshape(*lead, R, C // NVFP4_BLOCK, NVFP4_BLOCK)
+    amax_b = blocks.max(axis=-1)
+    s_b = e4m3_round((amax_b / np.float32(6.0 * 2.0 ** -8)).astype(np.float32)).astype(np.float32)
+    d_b = (s_b * NVFP4D_BLOCK_STEP).astype(np.float32)
+    safe = np.where(d_b > 0, d_b, np.float32(1.0)).astype(np.float32)
+    mag = e2m1_magnitude_code((blocks / safe[..., None]).astype(np.float32))
+    mag = np.where((d_b > 0)[..., None], mag, 0).astype(np.uint8)
+    neg = (xp.reshape(blocks.shape) < 0) & (d_b > 0)[..., None]
+    codes = (mag | (neg.astype(np.uint8) << 3)).reshape(x.shape).astype(np.uint8)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    return {"codes": codes, "packed": packed, "scales": e4m3_code(s_b), "colscales": e4m3_code(cs), "g": g}
+
+
+def nvfp4d_dequantize(codes, scales, colscales, g) -> np.ndarray:
+    """value(code) * (s_b * 2^-8) * (c * g) in fp32; returns float32 [..., R, C]."""
+    codes = np.asarray(codes, np.uint8)
+    *lead, R, C = codes.shape
+    d_b = (e4m3_value(scales).astype(np.float32) * NVFP4D_BLOCK_STEP).astype(np.float32)
+    mag = E2M1_VALUES[codes & 7].astype(np.float32)
+    v = (mag.reshape(*lead, R, C // NVFP4_BLOCK, NVFP4_BLOCK) * d_b[..., None]).astype(np.float32).reshape(codes.shape)
+    k = (e4m3_value(colscales).astype(np.float32) * np.asarray(g, np.float32)[..., None, None]).astype(np.float32)
+    k_rows = np.repeat(k, NVFP4D_GROUP_ROWS, axis=-2)[..., :R, :]
+    v = (v * k_rows).astype(np.float32)
+    return np.where(codes & 8, -v, v).astype(np.float32)
+
+
+def nvfp4d_quantize_state(S) -> dict:
+    """Two-axis encoding of states [..., rows, 128] by 64-row tiles: packed codes [..., rows, 64], row-block
+    scales [..., rows, 8], column-group scales [..., ceil(rows/16), 128] and g [..., tiles]."""
+    S = np.ascontiguousarray(S, np.float32)
+    rows = S.shape[-2]
+    parts = [nvfp4d_quantize(S[..., r0:r0 + NVFP4_TILE_ROWS, :]) for r0 in range(0, rows, NVFP4_TILE_ROWS)]
+    return {"codes": np.concatenate([p["codes"] for p in parts], axis=-2),
+            "packed": np.concatenate([p["packed"] for p in parts], axis=-2),
+            "scales": np.concatenate([p["scales"] for p in parts], axis=-2),
+            "colscales": np.concatenate([p["colscales"] for p in parts], axis=-2),
+            "g": np.stack([p["g"] for p in parts], axis=-1)}
+
+
+def nvfp4d_roundtrip_state(S) -> np.ndarray:
+    """fp32 values of the two-axis read copy of states [..., rows, 128]."""
+    S = np.ascontiguousarray(S, np.float32)
+    rows = S.shape[-2]
+    out = []
+    for r0 in range(0, rows, NVFP4_TILE_ROWS):
+        q = nvfp4d_quantize(S[..., r0:r0 + NVFP4_TILE_ROWS, :])
+        out.append(nvfp4d_dequantize(q["codes"], q["scales"], q["colscales"], q["g"]))
+    return np.concatenate(out, axis=-2)

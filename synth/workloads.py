@@ -16,12 +16,16 @@ Distributions (per workload family):
 * Mamba-2: x ~ N(0,1); B, C ~ N(0, 1/N); dt = clamp(softplus(z + dt_bias_h),
   1e-3, 0.1) with z ~ N(0,1) and dt_bias_h = softplus^-1(exp(U(ln 1e-3, ln 0.1)))
   (log-uniform time-step bias, the usual Mamba-2 initialisation); A_h =
-  -exp(U(0, ln 16)); D_h ~ N(0,1).  Initial checkpoint zero (tiny workload) or
+  -exp(U(0, ln 16)) (times decay_scale, 1 unless a case asks for faster decay);
+  D_h ~ N(0,1).  Initial checkpoint zero (tiny workload) or
   N(0, 0.05^2).
 * Gated DeltaNet: q, k = z/||z|| per head with z ~ N(0, I), normalised in fp32
   and then rounded; v ~ N(0,1); beta = sigmoid(N(0,1)); alpha =
   exp(-softplus(N(0,1)) * decay_scale) with decay_scale 0.05 (alpha mostly in
-  (0.9, 1)).  Initial checkpoint N(0, 1/d_k).
+  (0.9, 1)).  Initial checkpoint N(0, 1/d_k).  Optionally the state gets row
+  and column structure: v channel i of head h scaled by exp(value_spread *
+  N(0,1)) and key dimension j of q and k by exp(key_spread * N(0,1)) before the
+  normalisation, both fixed per layer (drawn once, from the parameter stream).
 """
 
 from __future__ import annotations
@@ -58,6 +62,7 @@ class Mamba2Workload:
     init: str         # "zero" or "normal"
     seed: int
     init_std: float = 0.05
+    decay_scale: float = 1.0   # multiplies A_h (faster-decaying heads for the decay-aware skipping cases)
 
     kind = "mamba2"
 
@@ -82,6 +87,8 @@ class GDNWorkload:
     seed: int
     decay_scale: float = 0.05
     q_scale: float = 1.0
+    value_spread: float = 0.0  # sigma of a log-normal scale per (head, value channel); 0 = none
+    key_spread: float = 0.0    # sigma of a log-normal scale per (head, key dimension) of q and k; 0 = none
 
     kind = "gdn"
 
@@ -137,7 +144,7 @@ def _softplus(z: np.ndarray) -> np.ndarray:
 def mamba2_params(wl: Mamba2Workload) -> dict:
     """Per-head layer parameters: A_h < 0 and D_h (fp32), plus the dt bias used by the generator."""
     r = _rng(wl.seed, _S_PARAMS, 0)
-    A = -np.exp(r.uniform(0.0, np.log(16.0), wl.nheads))
+    A = -np.exp(r.uniform(0.0, np.log(16.0), wl.nheads)) * wl.decay_scale
     D = r.standard_normal(wl.nheads)
     dt0 = np.exp(r.uniform(np.log(1e-3), np.log(0.1), wl.nheads))
     dt_bias = dt0 + np.log(-np.expm1(-dt0))  # inverse softplus
@@ -196,11 +203,29 @@ def _unit_rows(z: np.ndarray) -> np.ndarray:
     return z / n
 
 
+def gdn_structure(wl: GDNWorkload):
+    """Per-layer scales (value channels [H][d_v], key dimensions [H][d_k]) of a structured GDN workload, or
+    None where the spread is 0."""
+    r = _rng(wl.seed, _S_PARAMS, 1)
+    vs = r.standard_normal((wl.nheads, wl.dv))
+    ks = r.standard_normal((wl.nheads, wl.dk))
+    v_scale = np.exp(wl.value_spread * vs).astype(np.float32) if wl.value_spread else None
+    k_scale = np.exp(wl.key_spread * ks).astype(np.float32) if wl.key_spread else None
+    return v_scale, k_scale
+
+
 def _gdn_tokens(wl: GDNWorkload, stream_base: int, index: int, lead: tuple) -> dict:
     hd = lead + (wl.nheads,)
-    q = _unit_rows(_rng(wl.seed, stream_base + _S_Q, index).standard_normal(hd + (wl.dk,), dtype=np.float32))
-    k = _unit_rows(_rng(wl.seed, stream_base + _S_K, index).standard_normal(hd + (wl.dk,), dtype=np.float32))
+    v_scale, k_scale = gdn_structure(wl)
+    zq = _rng(wl.seed, stream_base + _S_Q, index).standard_normal(hd + (wl.dk,), dtype=np.float32)
+    zk = _rng(wl.seed, stream_base + _S_K, index).standard_normal(hd + (wl.dk,), dtype=np.float32)
+    if k_scale is not None:
+        zq, zk = zq * k_scale, zk * k_scale
+    q = _unit_rows(zq)
+    k = _unit_rows(zk)
     v = _rng(wl.seed, stream_base + _S_V, index).standard_normal(hd + (wl.dv,), dtype=np.float32)
+    if v_scale is not None:
+        v = v * v_scale
     zb = _rng(wl.seed, stream_base + _S_BETA, index).standard_normal(hd)
     za = _rng(wl.seed, stream_base + _S_ALPHA, index).standard_normal(hd)
     beta = (1.0 / (1.0 + np.exp(-zb))).astype(np.float32)

@@ -52,11 +52,11 @@ class Pair:
             S_full = mamba2_initial_state(wl) if S0 is None else S0
             self.gpu = ReplaySSM("mamba2", wl.batch, wl.nheads, wl.headdim, 128, wl.ngroups, wl.window, max_draft,
                                  self.dt, hp, read, seed, 1.0, torch.from_numpy(self.params["A"]),
-                                 torch.from_numpy(self.params["D"]))
+                                 torch.from_numpy(self.params["D"]), skip_tau=skip_tau)
             S_sel = S_full[self.seq_ids][:, self.head_ids]
             self.orc = ReplayOracle("mamba2", S_sel, wl.window, nheads=wl.nheads, ngroups=wl.ngroups,
                                     params=self.params, seq_ids=self.seq_ids, head_ids=self.head_ids, hp=hp,
-                                    read=read, seed=seed)
+                                    read=read, seed=seed, skip_tau=skip_tau)
         else:
             S_full = gdn_initial_state(wl) if S0 is None else S0
             self.gpu = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, 128, 1, wl.window, max_draft, self.dt, hp, read,
@@ -122,7 +122,8 @@ class Pair:
             return
         fields = (("x", "x", True), ("dt", "dt", True), ("B", "B", False)) if self.kind == "mamba2" else \
             (("k", "k", True), ("v", "v", True), ("alpha", "alpha", True), ("beta", "beta", True))
-        views = {name: ex["ring_" + name].float().cpu().numpy()[self.seq_ids] for name, _, _ in fields}
+        sel = torch.from_numpy(self.seq_ids).cuda()
+        views = {name: ex["ring_" + name].index_select(0, sel).float().cpu().numpy() for name, _, _ in fields}
         for i in range(len(self.seq_ids)):
             for slot in range(self.orc.live_slots(i)):
                 rec = self.orc.ring[i][slot]
@@ -133,8 +134,14 @@ class Pair:
                         got = got[self.head_ids]
                     np.testing.assert_array_equal(got, want, err_msg=f"ring {name} seq {i} slot {slot}")
 
+    def selected_state(self):
+        """The exported fp32 checkpoint of the sampled sequences and heads (sliced on the device)."""
+        S = self.gpu.export(state=True, ring=False)["S"]
+        S = S.index_select(0, torch.from_numpy(self.seq_ids).cuda())
+        return S.index_select(1, torch.from_numpy(self.head_ids).cuda()).cpu().numpy()
+
     def check_checkpoint(self, tol=TOL_CKPT):
-        S = self.gpu.export(state=True, ring=False)["S"].cpu().numpy()[self.seq_ids][:, self.head_ids]
+        S = self.selected_state()
         rows = S.shape[2]
         err = head_rel_err(S.reshape(S.shape[0], S.shape[1], -1),
                            self.orc.hp[..., :rows, :].reshape(S.shape[0], S.shape[1], -1))

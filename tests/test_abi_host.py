@@ -62,12 +62,15 @@ def test_arena_size_and_validation(lib):
 
 
 def test_precision_and_skip_modes_validation(lib):
-    """The FP8 checkpoint and decay-aware skipping are GDN modes: Mamba-2 contexts refuse them; a negative,
-    NaN or infinite threshold is an argument error.  The FP8 arena holds a quarter of the fp32 checkpoint plus
-    one fp32 scale per 64-row tile; skipping adds one flag byte per head."""
+    """The FP8 checkpoint is a GDN mode: Mamba-2 contexts refuse it.  Decay-aware skipping serves both kinds; a
+    negative, NaN or infinite threshold is an argument error.  The FP8 arena holds a quarter of the fp32
+    checkpoint plus one fp32 scale per 64-row tile; skipping adds one flag byte per head."""
     gdn = dict(kind=abi.GDN, headdim=128, ngroups=1, A=None, D=None)
     assert _arena(lib, hp=abi.HP_F8_SR)[0] == 3
-    assert _arena(lib, skip_tau=1e-3)[0] == 3
+    st, m_plain = _arena(lib)
+    st2, m_skip = _arena(lib, skip_tau=1e-3)
+    assert st == st2 == 0 and 2 * 4 <= m_skip - m_plain <= 256
+    assert _arena(lib, skip_tau=-1.0)[0] == 1
     assert _arena(lib, skip_tau=-1.0, **gdn)[0] == 1
     assert _arena(lib, skip_tau=float("nan"), **gdn)[0] == 1
     assert _arena(lib, skip_tau=float("inf"), **gdn)[0] == 1

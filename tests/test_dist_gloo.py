@@ -27,6 +27,48 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
+def _shard_worker(rank, world, port, q):
+    """What run_gpu does per rank, without the GPU: draw this rank's seeded inputs, time its replica (a fake
+    duration that differs by rank), and aggregate with max_over_ranks into the weak-scaling value."""
+    import hashlib
+
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        from synth import mamba2_step_inputs
+        wl = bench.rank_workload(rank).replace(batch=2)
+        digest = hashlib.sha1(mamba2_step_inputs(wl, 0)["x"].tobytes()).hexdigest()
+        digests = [None] * world
+        dist.all_gather_object(digests, digest)
+        my_ms = 100.0 + 25.0 * rank
+        total_ms = bench.max_over_ranks([my_ms])[0]
+        value = bench.weak_scaling_value(bench.WL.batch, world, 64, total_ms)
+        q.put((rank, digests, total_ms, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_shards_and_weak_scaling_fields_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = {r: rest for r, *rest in (q.get(timeout=120) for _ in procs)}
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    digests0, total0, value0 = out[0]
+    digests1, total1, value1 = out[1]
+    assert digests0 == digests1 and digests0[0] != digests0[1]     # each rank decodes its own shard
+    assert total0 == total1 == 125.0                                # the slowest rank's time, on every rank
+    assert value0 == value1 == pytest.approx(256 * 2 * 64 / 0.125)  # tokens of all ranks / that time
+
+
 def test_max_over_ranks_gloo_world2():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()

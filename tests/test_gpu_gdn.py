@@ -118,7 +118,7 @@ def _edge_state(shape, seed):
 
 
 @pytest.mark.parametrize("hp,read", [("f16sr", "nvfp4"), ("f32", "shared_nvfp4"), ("f16sr", "same"),
-                                     ("f8sr", "same"), ("f8sr", "nvfp4")])
+                                     ("f8sr", "same"), ("f8sr", "nvfp4"), ("f32", "nvfp4d"), ("f8sr", "nvfp4d")])
 def test_load_converters_bit_exact(cuda_ok, hp, read):
     wl = SMALL.replace(batch=2, nheads=3, dv=128)
     S = _edge_state((2, 3, 128, 128), 1)
@@ -134,7 +134,9 @@ def test_load_converters_bit_exact(cuda_ok, hp, read):
         np.testing.assert_array_equal(ex, want)
     if read != "same":
         rc = p.gpu.export_read_copy()
-        q = lp.nvfp4_quantize_state(S)
+        q = (lp.nvfp4d_quantize_state if read == "nvfp4d" else lp.nvfp4_quantize_state)(S)
+        if read == "nvfp4d":
+            np.testing.assert_array_equal(p.gpu.export_column_scales().cpu().numpy(), q["colscales"])
         np.testing.assert_array_equal(rc["packed"].cpu().numpy(), q["packed"])
         np.testing.assert_array_equal(rc["scales"].cpu().numpy(), q["scales"])
         np.testing.assert_array_equal(rc["g"].cpu().numpy(), q["g"])
@@ -153,28 +155,28 @@ TOL_FLIP = 2e-2
 FLIP_FRACTION = 0.02
 
 
-@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f16sr", "same"), ("f32", "shared_nvfp4"),
-                                     ("f8sr", "same"), ("f8sr", "nvfp4")])
-def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
-    """With stochastic rounding the oracle's trajectory is one sample among many, so the GPU is held to
-    the spread between two oracle seeds (mean error at most twice the seed-to-seed mean, plus the fp32
-    bound); without it, to rare single-code NVFP4 flips."""
+def track_lowprec(wl, hp, read, steps, seq_ids=None, head_ids=None):
+    """Steps a low-precision context beside the oracle in the same mode (on the sampled sequences and heads).
+    With stochastic rounding the oracle's trajectory is one sample among many, so the GPU is held to the
+    spread between two oracle seeds (mean error at most twice the seed-to-seed mean, plus the fp32 bound);
+    without it, to rare single-code NVFP4 flips.  Returns the per-output errors."""
     from oracle.decoder import ReplayOracle
-    wl = GDN_LOWPREC.replace(batch=4, nheads=4, window=8)
-    p = Pair(wl, hp=hp, read=read, seed=7)
+    from synth import gdn_initial_state
+    p = Pair(wl, seq_ids=seq_ids, head_ids=head_ids, hp=hp, read=read, seed=7)
     other = None
     if hp in ("f16sr", "f8sr"):
-        from synth import gdn_initial_state
-        other = ReplayOracle("gdn", gdn_initial_state(wl), wl.window, nheads=wl.nheads, hp=hp, read=read, seed=8)
+        S_sel = gdn_initial_state(wl, seqs=p.seq_ids)[:, p.head_ids]
+        other = ReplayOracle("gdn", S_sel, wl.window, nheads=wl.nheads, seq_ids=p.seq_ids, head_ids=p.head_ids,
+                             hp=hp, read=read, seed=8)
     errs, spread = [], []
-    for t in range(48):
+    for t in range(steps):
         inp = gdn_step_inputs(wl, t)
         y, y_ref, y_true = p.step(inp)
         err = head_rel_err(y, y_ref)
         errs.append(err.ravel())
         assert err.max() <= TOL_FLIP, f"step {t}: {err.max():.3e}"
         if other is not None:
-            y_other, _ = other.step(inp)
+            y_other, _ = other.step({k: v[p.seq_ids] for k, v in inp.items()})
             spread.append(head_rel_err(y_other, y_ref).ravel())
         p.check_bookkeeping(ring=(t % 8 == 7))
     errs = np.concatenate(errs)
@@ -186,6 +188,32 @@ def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
         assert errs.mean() <= 2 * spread.mean() + TOL_F32
     else:
         assert frac <= FLIP_FRACTION
+    return p, errs
+
+
+@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f16sr", "same"), ("f32", "shared_nvfp4"),
+                                     ("f8sr", "same"), ("f8sr", "nvfp4"), ("f32", "nvfp4d"), ("f16sr", "nvfp4d")])
+def test_lowprec_modes_track_oracle(cuda_ok, hp, read):
+    track_lowprec(GDN_LOWPREC.replace(batch=4, nheads=4, window=8), hp, read, 48)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "nvfp4"), ("f8sr", "nvfp4")])
+def test_lowprec_full_batch_sampled(cuda_ok, hp, read):
+    """The separate-precision GDN layer at full size (batch 256, 32 heads, d 128, L 16), four windows, on
+    sampled sequences and heads; after the last fold the sampled read copies are the NVFP4 quantisation of
+    the fp32 fold result (in fp32-checkpoint mode, of the exported checkpoint), bit for bit."""
+    wl = GDN_LOWPREC
+    p, _ = track_lowprec(wl, hp, read, 4 * wl.window, seq_ids=[0, 128, 255], head_ids=[0, 13, 31])
+    if hp == "f32":
+        S = p.selected_state()
+        rc = p.gpu.export_read_copy()
+        sel_s, sel_h = torch.from_numpy(p.seq_ids).cuda(), torch.from_numpy(p.head_ids).cuda()
+        q = lp.nvfp4_quantize_state(S)
+        for key in ("packed", "scales", "g"):
+            got = rc[key].index_select(0, sel_s).index_select(1, sel_h).cpu().numpy()
+            np.testing.assert_array_equal(got, q[key], err_msg=key)
+    assert p.gpu.get_error() == (0, -1)
 
 
 @pytest.mark.parametrize("hp,read", [("f32", "nvfp4"), ("f16sr", "same"), ("f8sr", "nvfp4")])

@@ -174,3 +174,79 @@ def test_full_size_sampled(cuda_ok):
     p.check_bookkeeping()
     p.check_checkpoint()
     print(f"worst rel err {worst:.3e}")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [4, 8])
+def test_speculative_full_size_sampled(cuda_ok, T):
+    """Speculative verify + commit on the Mamba-2 shape at batch 512 (2 GiB checkpoint, 128 heads, 8 groups,
+    L 16): 64 rounds with the seeded accepted lengths, so every round some of the 4096 units pre-fold.  Sampled
+    sequences 0, 255, 511 and one head in each of the 8 groups: every draft output within the fp32 bound, the
+    bookkeeping bit-exact after every call, the ring byte-exact and the checkpoint within 1e-5 every 16 rounds."""
+    wl = SPEC_MAMBA2_B512
+    heads = [0, 17, 35, 50, 64, 81, 99, 127]                  # groups 0..7
+    p = Pair(wl, seq_ids=[0, 255, 511], head_ids=heads, max_draft=T)
+    worst, prefolds = 0.0, 0
+    for rnd in range(64):
+        before = p.orc.epoch.copy()
+        y, _, y_true = p.verify(T, mamba2_draft_inputs(wl, rnd, T))
+        prefolds += int(np.sum(p.orc.epoch != before))
+        err = head_rel_err(y, y_true).max()
+        worst = max(worst, err)
+        assert err <= TOL_F32, f"round {rnd}: {err:.3e}"
+        p.check_bookkeeping(ring=False)
+        p.commit(accepted_lengths(wl, rnd, T))
+        p.check_bookkeeping(ring=(rnd % 16 == 15))
+        if rnd % 16 == 15:
+            p.check_checkpoint()
+    assert prefolds >= 3 * (64 * T // 2 // wl.window) // 2     # about one pre-fold per 16 / (T / 2) rounds each
+    assert p.gpu.get_error() == (0, -1)
+    print(f"T={T}: worst rel err {worst:.3e}, pre-folds on the sampled sequences {prefolds}")
+
+
+# ------------------------------------------------------------------------------------ decay-aware skipping
+
+FAST_M2 = MAMBA2_TINY.replace(batch=5, nheads=16, ngroups=2, init="normal", in_dtype="bf16", decay_scale=8.0)
+
+
+@pytest.mark.parametrize("in_dtype", ["bf16", "f32"])
+def test_skip_steps_match_oracle(cuda_ok, in_dtype):
+    """Steps over three windows with tau = 1e-2 on fast-decaying heads (A times 8): flags bit-exact after every
+    call, outputs and checkpoints against the oracle that skips the same reads, some heads skipped and some not."""
+    wl = FAST_M2.replace(in_dtype=in_dtype)
+    p = Pair(wl, skip_tau=1e-2)
+    skipped, calls = 0, 0
+    for t in range(3 * wl.window + 5):
+        skipped += int(p.orc.skip.sum())
+        calls += p.orc.skip.size
+        y, y_ref, _ = p.step(mamba2_step_inputs(wl, t))
+        assert head_rel_err(y, y_ref).max() <= TOL_F32, f"step {t}"
+        p.check_bookkeeping(ring=(t % 8 == 7))
+    assert 0 < skipped < calls
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
+@pytest.mark.parametrize("T", [4, 8])
+def test_skip_verify_commit_flush(cuda_ok, T):
+    """Verify/commit rounds (T = 8 takes the tensor-core output path), steps between them and a flush, with
+    skipping on: outputs against the skipping oracle, flags bit-exact after every call."""
+    wl = FAST_M2
+    p = Pair(wl, max_draft=T, skip_tau=2e-2)
+    rng = np.random.default_rng(4)
+    skipped = 0
+    for rnd in range(12):
+        skipped += int(p.orc.skip.sum())
+        y, y_ref, _ = p.verify(T, mamba2_draft_inputs(wl, rnd, T))
+        assert head_rel_err(y, y_ref).max() <= TOL_F32, f"round {rnd}"
+        p.check_bookkeeping(ring=False)
+        p.commit(accepted_lengths(wl, rnd, T))
+        for k in range(int(rng.integers(0, 4))):
+            y, y_ref, _ = p.step(mamba2_step_inputs(wl, 100 + 4 * rnd + k))
+            assert head_rel_err(y, y_ref).max() <= TOL_F32
+        p.check_bookkeeping(ring=True)
+    assert skipped > 0
+    p.flush()
+    p.check_bookkeeping()
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)

@@ -265,3 +265,98 @@ def test_skip_flags_under_verify_commit_and_flush():
     assert o.skip.all()
     o.flush()
     assert not o.skip.any() and (o.count == 0).all()
+
+
+# ------------------------------------------------------------------------------------ Mamba-2 decay-aware skipping
+
+M2_TAU = float(np.exp(-2.25))          # ln(tau) lies between -2.5 and -2.0
+
+
+def _mamba_A(L, A, **kw):
+    """The Mamba-2 oracle of _mamba with per-head A replaced (fp32 values)."""
+    p = dict(mamba2_params(M_WL))
+    p["A"] = np.broadcast_to(np.asarray(A, np.float32), (M_WL.nheads,)).copy()
+    rng = np.random.default_rng(0)
+    S0 = rng.standard_normal((M_WL.batch, M_WL.nheads, M_WL.headdim, M_WL.dstate)) * 0.05
+    return ReplayOracle("mamba2", S0, L, nheads=M_WL.nheads, ngroups=M_WL.ngroups, params=p, **kw), S0
+
+
+def _const_dt(t, dt=0.0625, draft=None):
+    inp = mamba2_step_inputs(M_WL, t) if draft is None else mamba2_draft_inputs(M_WL, t, draft)
+    inp["dt"] = np.full_like(inp["dt"], dt)
+    return inp
+
+
+def test_mamba2_skip_flags_follow_the_decay_and_bound_the_dropped_term():
+    """A = -8 and dt = 1/16 make A * (sum of dt) over n committed records exactly -n/2 in fp32, so with
+    ln(tau) = -2.25 a head is flagged exactly when 5 or more records are committed, and a fold clears it.
+    Within the first window the skipping oracle differs from the non-skipping one only on calls that read a
+    set flag, and there by at most tau * ||S0|| * ||C|| per head (the whole dropped term exp(A s) S0 C)."""
+    L = 8
+    sk, S0 = _mamba_A(L, -8.0, skip_tau=M2_TAU)
+    ref, _ = _mamba_A(L, -8.0)
+    for t in range(2 * L + 3):
+        inp = _const_dt(t)
+        before = sk.skip.copy()
+        y, _ = sk.step(inp)
+        y0, _ = ref.step(inp)
+        n = (t + 1) % L
+        np.testing.assert_array_equal(sk.skip, np.full((M_WL.batch, M_WL.nheads), n >= 5))
+        if t < L - 1:                                   # same checkpoint on both sides until the first fold
+            d = np.linalg.norm(y - y0, axis=-1)
+            c = np.linalg.norm(inp["C"][:, 0], axis=-1)[:, None]          # one group
+            bound = M2_TAU * np.linalg.norm(S0, axis=(-2, -1)) * c
+            assert np.all(d[~before] == 0)
+            assert np.all(d[before] <= bound[before] * (1 + 1e-9))
+            assert np.all(d[before] > 0)
+
+
+def test_mamba2_skip_with_a_vanishing_decay_changes_nothing():
+    """With A dt = -1000 on one head, exp(A dt) is exactly zero in float64, so that head's checkpoint contributes
+    nothing once a record is buffered: skipping its read (and folding from the buffer alone) gives the
+    non-skipping oracle's outputs and checkpoints exactly, and the other heads are never flagged."""
+    L = 8
+    A = np.array([-1.0, -1e4, -1.0, -1.0], np.float32)
+    sk, _ = _mamba_A(L, A, skip_tau=1e-3)
+    ref, _ = _mamba_A(L, A)
+    for t in range(3 * L):
+        inp = mamba2_step_inputs(M_WL, t)
+        inp["dt"][:, 1] = 0.1
+        y, _ = sk.step(inp)
+        y0, _ = ref.step(inp)
+        np.testing.assert_array_equal(y, y0)
+        assert not sk.skip[:, [0, 2, 3]].any()
+        np.testing.assert_array_equal(sk.skip[:, 1], (t % L) != L - 1)
+    np.testing.assert_array_equal(sk.hp, ref.hp)
+
+
+def test_mamba2_skip_flags_under_verify_commit_and_flush():
+    """Verify sets the flags from the committed records only (drafts excluded); commit leaves them; a pre-fold
+    or a flush clears them."""
+    L = 8
+    o, _ = _mamba_A(L, -8.0, skip_tau=M2_TAU)
+    for t in range(6):
+        o.step(_const_dt(t))
+    assert o.skip.all()                                 # 6 records: -3 < -2.25
+    o.verify(2, _const_dt(0, draft=2))                  # 6 + 2 <= 8: no pre-fold
+    assert o.skip.all()
+    o.commit(np.full(M_WL.batch, 2))
+    assert o.skip.all() and (o.count == 8).all()
+    o.verify(2, _const_dt(1, draft=2))                  # 8 + 2 > 8: pre-fold, nothing committed after it
+    assert not o.skip.any()
+    o.commit(np.zeros(M_WL.batch, np.int64))
+    for t in range(4):
+        o.step(_const_dt(10 + t))
+    assert not o.skip.any()                             # 4 records: -2 > -2.25
+    o.step(_const_dt(20))
+    assert o.skip.all()
+    o.flush()
+    assert not o.skip.any() and (o.count == 0).all()
+
+
+def test_skip_threshold_is_the_fp32_log():
+    """ln(tau) is the double-precision log of the fp32 threshold, rounded once to fp32."""
+    import math
+    o, _ = _mamba_A(8, -1.0, skip_tau=1e-2)
+    assert o.ln_tau == np.float32(math.log(float(np.float32(1e-2))))
+    assert o.ln_tau.dtype == np.float32 and abs(float(o.ln_tau) - math.log(1e-2)) < 1e-6

@@ -277,3 +277,85 @@ def test_fp8_state_tiles_scale_and_bound():
     step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** -6))) - 3), 2.0 ** -9)
     assert np.all(np.abs(q["values"] / s_rows - y) <= step * (1 + 1e-6))
     np.testing.assert_array_equal((lp.e4m3_value(q["codes"]).astype(np.float32) * s_rows).astype(np.float32), q["values"])
+
+
+# ------------------------------------------------------------------------------------ two-axis NVFP4 read copy
+
+def _dual_grid_tile(rng, rows=64, g_exp=-3):
+    """A tile on the two-axis grid: x = value * k_j with d_b = 1, one +-6 in every (row block) and in every
+    (column, 16-row group), column-group steps k = c * g (c E4M3, one of them 448) and g = 2^g_exp."""
+    g = np.float32(2.0 ** g_exp)
+    vals = lp.E2M1_VALUES[rng.integers(0, 8, (rows, 128))] * rng.choice([-1.0, 1.0], (rows, 128))
+    for r0 in range(0, rows, 16):                                  # in a group of m rows, row i holds a 6 at
+        m = min(16, rows - r0)                                     # every column = i (mod m): every row block
+        for i in range(m):                                         # and every column of the group has one
+            vals[r0 + i, i::m] = 6.0 * rng.choice([-1.0, 1.0], len(range(i, 128, m)))
+    grid = np.unique(np.abs(lp.e4m3_round(np.linspace(2.0 ** -6, 448.0, 4000))))
+    ngr = -(-rows // 16)
+    c = rng.choice(grid[grid > 0], (ngr, 128)).astype(np.float32)
+    c[0, 5] = 448.0
+    k = np.repeat(c * g, 16, axis=0)[:rows]
+    return (vals * k).astype(np.float32), c, g
+
+
+def test_nvfp4d_grid_tile_roundtrips_exactly():
+    """A tile built on the two-axis grid is encoded with its own column-group and row-block scales and decodes
+    exactly; so does a tile of equal magnitudes 2688 * 2^n."""
+    rng = np.random.default_rng(11)
+    for rows in (64, 40):
+        x, c, g = _dual_grid_tile(rng, rows)
+        q = lp.nvfp4d_quantize(x)
+        assert q["g"] == g
+        np.testing.assert_array_equal(lp.e4m3_value(q["colscales"]), c)
+        np.testing.assert_array_equal(lp.e4m3_value(q["scales"]), np.full((rows, 8), 256.0))   # d_b = 1
+        np.testing.assert_array_equal(lp.nvfp4d_dequantize(q["codes"], q["scales"], q["colscales"], q["g"]), x)
+    flat = (np.float32(2688 * 2.0 ** -5) * rng.choice([-1.0, 1.0], (64, 128))).astype(np.float32)
+    np.testing.assert_array_equal(lp.nvfp4d_roundtrip_state(flat[None]), flat[None])
+
+
+def test_nvfp4d_zero_groups_packing_and_state_tiles():
+    x = np.random.default_rng(2).standard_normal((2, 72, 128)).astype(np.float32)
+    x[0, 16:32, 7] = 0.0                                          # one zero column group
+    x[1] = 0.0                                                    # an all-zero state
+    q = lp.nvfp4d_quantize_state(x)
+    assert q["packed"].shape == (2, 72, 64) and q["scales"].shape == (2, 72, 8)
+    assert q["colscales"].shape == (2, 5, 128) and q["g"].shape == (2, 2)
+    np.testing.assert_array_equal(q["packed"], q["codes"][..., 0::2] | (q["codes"][..., 1::2] << 4))
+    assert q["colscales"][0, 1, 7] == 0 and not q["codes"][0, 16:32, 7].any()
+    assert not q["codes"][1].any() and np.all(q["g"][1] == 1.0)
+    r = lp.nvfp4d_roundtrip_state(x)
+    assert np.all(r[1] == 0) and np.all(r[0, 16:32, 7] == 0)
+    # rows 64..71 form their own tile: its scale comes from those rows alone
+    np.testing.assert_array_equal(r[0, 64:], lp.nvfp4d_roundtrip_state(x[0:1, 64:])[0])
+
+
+def test_nvfp4d_error_bound():
+    """Each element lies within one E2M1 step of its value in units of its step k * d_b (half a step from the
+    grid, plus the clipping of a block maximum whose scale rounded down)."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((6, 64, 128)) * np.exp(rng.standard_normal((6, 64, 1)))).astype(np.float32)
+    q = lp.nvfp4d_quantize(x)
+    k = np.repeat(lp.e4m3_value(q["colscales"]) * q["g"][:, None, None], 16, axis=-2)
+    d_b = np.repeat(lp.e4m3_value(q["scales"]) * 2.0 ** -8, 16, axis=-1)
+    step = k * d_b
+    err = np.abs(lp.nvfp4d_dequantize(q["codes"], q["scales"], q["colscales"], q["g"]) - x)
+    assert np.all(err <= 1.0 * step * (1 + 1e-6) + 0.07 * np.abs(x))
+    assert np.mean(err <= 1.0 * step * (1 + 1e-6)) > 0.999
+
+
+def test_nvfp4d_cuts_the_read_error_of_channel_structured_states():
+    """Against the one-axis copy: on states whose channels (rows) differ in magnitude, and whose state columns
+    differ too, the two-axis copy's Frobenius error is at least 15% lower; on unstructured states it is not
+    higher.  (The drift measurement on the GPU reports the effect on outputs.)"""
+    rng = np.random.default_rng(9)
+    sh = (4, 4, 128, 128)
+    iid = rng.standard_normal(sh).astype(np.float32)
+    rows = (rng.standard_normal(sh) * np.exp(rng.standard_normal(sh[:2] + (128, 1)))).astype(np.float32)
+    both = (rows * np.exp(rng.standard_normal(sh[:2] + (1, 128)))).astype(np.float32)
+
+    def rel(f, S):
+        return np.linalg.norm(f(S) - S) / np.linalg.norm(S)
+
+    for S in (rows, both):
+        assert rel(lp.nvfp4d_roundtrip_state, S) <= 0.85 * rel(lp.nvfp4_roundtrip_state, S)
+    assert rel(lp.nvfp4d_roundtrip_state, iid) <= rel(lp.nvfp4_roundtrip_state, iid)
