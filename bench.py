@@ -722,7 +722,7 @@ PRECISION_MODES = (("f32", "same"), ("f16sr", "same"), ("f8sr", "same"), ("f32",
                    ("f8sr", "nvfp4"), ("f32", "shared_nvfp4"), ("f32", "nvfp4d"))
 
 
-def precision_section(windows_timed: int = 4) -> dict:
+def precision_section(windows_timed: int = 4, modes=None) -> dict:
     """GDN layer (batch 256, 32 heads, d 128, L 16) with each checkpoint format and read mode: window-averaged
     step time, plain and fold launches, and the rate of the mode's algorithmic bytes."""
     import torch
@@ -741,6 +741,8 @@ def precision_section(windows_timed: int = 4) -> dict:
     out = {"workload": "gdn replay decode, batch 256, 32 heads, d_k = d_v = 128, L 16, bf16 inputs; checkpoint "
                        "format x read mode"}
     for hp, read in PRECISION_MODES:
+        if modes and f"{hp}/{read}" not in modes:
+            continue
         layer = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, wl.dk, 1, wl.window, 0, bf, hp, read, seed=3)
         layer.load_checkpoint(S0)
 
@@ -1103,6 +1105,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=64)
     ap.add_argument("--impl", default="rssm", choices=["rssm", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", action="append", default=None,
+                    help="with --only precision: run only this checkpoint/read mode (e.g. f32/nvfp4); repeatable")
     ap.add_argument("--no-extra", action="store_true", help="skip the GDN, speculative-verify, precision and read-skipping sections")
     ap.add_argument("--only", choices=["gdn", "verify", "verify-mamba2", "verify-gdn", "window", "batch",
                                                   "precision", "skip", "skip-mamba2", "graph"], default=None,
@@ -1125,7 +1129,7 @@ def main():
                    verify_section(args.steps) if args.only == "verify" else
                    verify_section(args.steps, (args.only.split("-")[1],)) if args.only.startswith("verify-") else
                    batch_section() if args.only == "batch" else
-                   precision_section() if args.only == "precision" else
+                   precision_section(modes=args.mode) if args.only == "precision" else
                    skip_section() if args.only == "skip" else
                    skip_mamba2_section() if args.only == "skip-mamba2" else
                    graph_section() if args.only == "graph" else window_section())

@@ -284,8 +284,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       return true;
     };
-    // units come from the launch's counter: the group data of the next unit is issued before
-    // the current unit's tiles, and the unit after that is requested (atomic in flight) meanwhile
+    // units come from the launch's counter: the group data of the next unit is issued once the current
+    // unit's first two tiles are on their way (its bookkeeping load then does not hold them up), and the
+    // unit after that is requested (atomic in flight) meanwhile
     int u_cur = 0, u_nxt = 0;
     if (lane == 0) u_cur = sched_grab(a.err);
     u_cur = __shfl_sync(0xffffffffu, u_cur, 0);
@@ -295,12 +296,14 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     bool ok = issue_group(u_cur, 0, Sc);
     int ti = 0;
     for (int gi = 0; ok && u_cur < units; ++gi) {
-      if (!issue_group(u_nxt, gi + 1, Sn)) {
-        ok = false;
-        break;
-      }
-      int u_after = units;  // read back (and so completed) at the end of the iteration on every path
-      if (lane == 0 && u_nxt < units) u_after = sched_grab(a.err);
+      int u_after = units;  // read back (and so completed) at the end of the iteration
+      bool nxt_issued = false;
+      auto issue_next = [&]() -> bool {
+        nxt_issued = true;
+        if (!issue_group(u_nxt, gi + 1, Sn)) return false;
+        if (lane == 0 && u_nxt < units) u_after = sched_grab(a.err);
+        return true;
+      };
       const Sched S = Sc;
       if (S.active) {
         const int n_rec = S.n_ring + S.n_new;
@@ -309,6 +312,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                                 : (fp4_read ? read_fmt : hp_fmt);
         const bool fp4src = srcfmt == SRC_FP4 || srcfmt == SRC_FP4D;
         for (int tt = 0; tt < S.nh * nrb; ++tt, ++ti) {
+          if (tt == 2 && !issue_next()) {
+            ok = false;
+            break;
+          }
           const int i = tt / nrb, t = tt % nrb;
           const int rows = min(kFp4Rows, R - kFp4Rows * t);
           const size_t unit = (size_t)S.b * a.H + S.h0 + i;
@@ -364,6 +371,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           }
         }
       }
+      if (ok && !nxt_issued && !issue_next()) ok = false;
+      if (!ok) break;
       Sc = Sn;
       u_cur = u_nxt;
       u_nxt = __shfl_sync(0xffffffffu, u_after, 0);
@@ -455,17 +464,38 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           float *co = cot + ((size_t)i * lay.no + j) * lay.rmax;
           for (int r = sl; r < n_rec; r += 8)
             if (r < m || r >= e_j) co[r] = 0.f;
+          // the walk-back is one dependent chain per (head, output): the next record's key and gates are
+          // loaded while the current one is reduced, and the dot product runs as four partial sums
+          auto gate = [&](int r, float &al, float &be) {
+            al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
+            be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
+          };
+          float kn[16], aln = 0.f, ben = 0.f;
+          if (e_j - 1 >= m) {
+            load_k16(kg + ((size_t)i * lay.rmax + (e_j - 1)) * kCols + sl * 16, kn);
+            gate(e_j - 1, aln, ben);
+          }
           for (int r = e_j - 1; r >= m; --r) {
             float kv[16];
-            load_k16(kg + ((size_t)i * lay.rmax + r) * kCols + sl * 16, kv);
-            float c = 0.f;
 #pragma unroll
-            for (int z = 0; z < 16; ++z) c = fmaf(u[z], kv[z], c);
+            for (int z = 0; z < 16; ++z) kv[z] = kn[z];
+            const float al = aln, be = ben;
+            if (r > m) {
+              load_k16(kg + ((size_t)i * lay.rmax + (r - 1)) * kCols + sl * 16, kn);
+              gate(r - 1, aln, ben);
+            }
+            float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll
+            for (int z = 0; z < 16; z += 4) {
+              c0 = fmaf(u[z], kv[z], c0);
+              c1 = fmaf(u[z + 1], kv[z + 1], c1);
+              c2 = fmaf(u[z + 2], kv[z + 2], c2);
+              c3 = fmaf(u[z + 3], kv[z + 3], c3);
+            }
+            float c = (c0 + c1) + (c2 + c3);
             c += __shfl_xor_sync(smask, c, 1);
             c += __shfl_xor_sync(smask, c, 2);
             c += __shfl_xor_sync(smask, c, 4);
-            const float al = r < n_ring ? ag[i * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + i];
-            const float be = r < n_ring ? bg[i * dts + base_e + r] : gf[Q_FB + (r - n_ring) * 8 + i];
             if (sl == 0) co[r] = a.q_scale * be * c;
             const float bc = be * c;
 #pragma unroll
@@ -570,43 +600,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             const float4 e = e2m1x4_to_float4(cw);
             return make_float4(__fmul_rn(e.x, d_b), __fmul_rn(e.y, d_b), __fmul_rn(e.z, d_b), __fmul_rn(e.w, d_b));
           };
-          if (NO == 1 && !fold) {
-            // ---------------- non-fold tile, one output: four lanes per row, 32 columns each (chunks rotated by
-            // lane, as in fold tiles), the buffered term split over the four lanes by record; two shuffles
-            // finish the row (rows is a multiple of 8, so a warp's rows are all live or all past the tile)
-            const int qtr = lane & 3;
-            const int row = row0 + (lane >> 2);
-            const int rowg = kFp4Rows * t + row;
-            if (row0 < rows && t_out > 0) {
-              float z0 = 0.f, z1 = 0.f;
-              if (!((skm >> i) & 1u)) {  // a skipped head's checkpoint term is zero
-                const float *uq = u0_h + qtr * 32;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                  const int ch = (c + lane) & 7;
-                  float4 u4 = *reinterpret_cast<const float4 *>(uq + ch * 4);
-                  if (srcfmt == SRC_FP4D) {  // column-group steps k = E4M3 * g of this row's 16-row group
-                    const float4 c4 = e4m3x4_to_float4(*reinterpret_cast<const uint32_t *>(
-                        st + kColScaleOff + (row >> 4) * kCols + qtr * 32 + ch * 4));
-                    u4.x *= __fmul_rn(c4.x, g_tile); u4.y *= __fmul_rn(c4.y, g_tile);
-                    u4.z *= __fmul_rn(c4.z, g_tile); u4.w *= __fmul_rn(c4.w, g_tile);
-                  }
-                  const float4 s4 = srcfmt == SRC_F32
-                                        ? *reinterpret_cast<const float4 *>(st + (row * kCols + qtr * 32 + ch * 4) * 4)
-                                        : load_row4(row, qtr * 32 + ch * 4);
-                  z0 = fmaf(s4.x, u4.x, z0);
-                  z1 = fmaf(s4.y, u4.y, z1);
-                  z0 = fmaf(s4.z, u4.z, z0);
-                  z1 = fmaf(s4.w, u4.w, z1);
-                }
-              }
-              float z = z0 + z1;
-              for (int r = qtr; r < n_rec; r += 4) z = fmaf(co_h[r], to_f32(vr[r * R + rowg]), z);
-              z += __shfl_xor_sync(0xffffffffu, z, 1);
-              z += __shfl_xor_sync(0xffffffffu, z, 2);
-              if (qtr == 0) a.y[((size_t)b * a.T * a.H + h) * R + rowg] = z;
-            }
-          } else if (!fold) {
+          if (!fold) {
             // ---------------- non-fold tile: lane owns columns 4l..4l+3 of the warp's 8 rows
             if (row0 < rows) {
               constexpr int V = 8 * NO;
@@ -627,6 +621,9 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                 }
               }
               float4 sv[8];
+              float dstep[8];  // NVFP4 copies: the row's block step, applied to the row's dot product
+#pragma unroll
+              for (int rr = 0; rr < 8; ++rr) dstep[rr] = 1.f;
               if ((skm >> i) & 1u) {  // skipped head: the checkpoint term is zero
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) sv[rr] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -634,6 +631,16 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr)
                   sv[rr] = *reinterpret_cast<const float4 *>(st + ((row0 + rr) * kCols + 4 * lane) * 4);
+              } else if (srcfmt == SRC_FP4 || srcfmt == SRC_FP4D) {
+                // the lane's 4 columns lie in one 16-element block of each row: E2M1 values here, the block
+                // step once per row
+                const float dmul = srcfmt == SRC_FP4D ? 0.00390625f : g_tile;
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                  const int row = row0 + rr;
+                  sv[rr] = e2m1x4_to_float4(*reinterpret_cast<const uint16_t *>(st + row * (kCols / 2) + 2 * lane));
+                  dstep[rr] = __fmul_rn(e4m3_to_float(st[kTileMaxBytes / 2 + row * (kCols / 16) + (lane >> 2)]), dmul);
+                }
               } else {
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) sv[rr] = load_row4(row0 + rr, 4 * lane);
@@ -643,7 +650,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               for (int rr = 0; rr < 8; ++rr)
 #pragma unroll
                 for (int j = 0; j < NO; ++j)
-                  part[rr * NO + j] = sv[rr].x * uv[j].x + sv[rr].y * uv[j].y + sv[rr].z * uv[j].z + sv[rr].w * uv[j].w;
+                  part[rr * NO + j] =
+                      dstep[rr] * (sv[rr].x * uv[j].x + sv[rr].y * uv[j].y + sv[rr].z * uv[j].z + sv[rr].w * uv[j].w);
               // buffered part: lane r adds coef_{j,r} v_r[row] for the 8 rows (one 16-byte load of v_r)
               for (int r = lane; r < n_rec; r += 32) {
                 float vv[8];

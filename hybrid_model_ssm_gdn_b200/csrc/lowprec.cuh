@@ -55,6 +55,14 @@ __device__ __forceinline__ __half fp16_sr(float x, uint32_t r) {
   const uint32_t bits = __float_as_uint(x);
   const uint32_t sign = bits >> 31;
   const int E = (int)((bits >> 23) & 0xFFu);
+  if ((uint32_t)(E - 113) <= 29u) {
+    // |x| in [2^-14, 2^16): the fp16 spacing leaves 13 fp32 mantissa bits F below it, and the rule rounds up
+    // iff (r >> 19) < F.  Adding 2^13 - 1 - (r >> 19) = (~r) >> 19 to the magnitude's bits carries into bit 13
+    // exactly then (a carry out of the mantissa moves to the next binade); truncating the 13 bits finishes it.
+    const uint32_t m = ((bits & 0x7FFFFFFFu) + ((~r) >> 19)) & ~0x1FFFu;
+    const float mag = fminf(__uint_as_float(m), 65504.f);
+    return __float2half_rn(sign ? -mag : mag);                 // exact: the value lies on the fp16 grid
+  }
   const uint32_t mant = bits & 0x7FFFFFu;
   if (E == 255) return mant ? __ushort_as_half(0x7E00) : __ushort_as_half(sign ? 0xFBFF : 0x7BFF);
   const uint32_t M = E ? (mant | 0x800000u) : mant;  // |x| = M * 2^(Eeff - 150)
@@ -80,6 +88,13 @@ __device__ __forceinline__ uint32_t fp8_sr_code(float y, uint32_t r) {
   const uint32_t bits = __float_as_uint(y);
   const uint32_t sign = bits >> 31;
   const int E = (int)((bits >> 23) & 0xFFu);
+  if ((uint32_t)(E - 121) <= 14u) {
+    // |y| in [2^-6, 2^9): 20 fp32 mantissa bits F lie below the E4M3 spacing; round up iff (r >> 12) < F, by
+    // the same carry as the fp16 rule, then take exponent and 3 mantissa bits, saturating at 448 (0x7E)
+    const uint32_t m = ((bits & 0x7FFFFFFFu) + ((~r) >> 12)) & ~0xFFFFFu;
+    const uint32_t code = m > 0x43E00000u ? 0x7Eu : ((((m >> 23) - 120u) << 3) | ((m >> 20) & 7u));
+    return code | (sign << 7);
+  }
   const uint32_t mant = bits & 0x7FFFFFu;
   const uint32_t M = E ? (mant | 0x800000u) : mant;  // |y| = M * 2^(Eeff - 150)
   const int Eeff = E ? E : 1;
