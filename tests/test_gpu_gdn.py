@@ -144,15 +144,21 @@ def test_load_converters_bit_exact(cuda_ok, hp, read):
 
 # ------------------------------------------------------------------------------------ separate precision
 
-# Bound for low-precision modes: GPU vs the oracle in the same mode.  The two fold in
-# different arithmetic (fp32 vs float64), so now and then one element lands on the other
-# side of an NVFP4 or stochastic-rounding decision boundary.  A flipped NVFP4 code moves
-# one element by one E2M1 step (at most a third of its block maximum), which moves that
-# head's output by up to ~1e-2 relative; a flipped fp16 rounding moves it by one fp16
-# ulp.  So: every head within TOL_FLIP, and all but a small fraction of (step, sequence,
-# head) outputs within the fp32 bound.
-TOL_FLIP = 2e-2
+# Bounds for the low-precision modes, GPU against the oracle in the same mode.
+#
+# Without stochastic rounding the two differ only in the fold's arithmetic (fp32 on the GPU, float64 in the
+# oracle): now and then an element of the new state lands on the other side of an NVFP4 decision, which moves
+# it by one E2M1 step (at most a third of its block's maximum).  The converters themselves are pinned bit for
+# bit (tests/test_gpu_fold_converters.py).  Measured on the small and full-batch cases: at most 3.5e-3 per
+# head, 0.9% of (step, sequence, head) outputs above 1e-4.  Bounds: 1e-2 per head, 2% above 1e-4.
+TOL_FLIP = 1e-2
 FLIP_FRACTION = 0.02
+# With stochastic rounding the oracle's trajectory is one sample among many: one rounding decision taken
+# differently changes the checkpoint by one fp16 (or E4M3) step, and the trajectories then differ within the
+# seed-to-seed spread.  The criterion is the mean error against that spread (at most twice it, plus the fp32
+# bound); the per-head cap only catches a gross error.  Measured: at most 1.8e-2 per head, mean at most
+# 1.6e-4 against spreads of 3e-3 to 7e-2.
+TOL_SR_HEAD = 3e-2
 
 
 def track_lowprec(wl, hp, read, steps, seq_ids=None, head_ids=None):
@@ -169,12 +175,13 @@ def track_lowprec(wl, hp, read, steps, seq_ids=None, head_ids=None):
         other = ReplayOracle("gdn", S_sel, wl.window, nheads=wl.nheads, seq_ids=p.seq_ids, head_ids=p.head_ids,
                              hp=hp, read=read, seed=8)
     errs, spread = [], []
+    cap = TOL_SR_HEAD if other is not None else TOL_FLIP
     for t in range(steps):
         inp = gdn_step_inputs(wl, t)
         y, y_ref, y_true = p.step(inp)
         err = head_rel_err(y, y_ref)
         errs.append(err.ravel())
-        assert err.max() <= TOL_FLIP, f"step {t}: {err.max():.3e}"
+        assert err.max() <= cap, f"step {t}: {err.max():.3e}"
         if other is not None:
             y_other, _ = other.step({k: v[p.seq_ids] for k, v in inp.items()})
             spread.append(head_rel_err(y_other, y_ref).ravel())
@@ -223,14 +230,16 @@ def test_verify_lowprec_modes(cuda_ok, hp, read):
     wl = GDN_LOWPREC.replace(batch=3, nheads=4, window=8)
     p = Pair(wl, hp=hp, read=read, seed=7, max_draft=8)
     errs = []
+    cap = TOL_FLIP if hp == "f32" else TOL_SR_HEAD
     for rnd in range(10):
         y, y_ref, _ = p.verify(8, gdn_draft_inputs(wl, rnd, 8))
         err = head_rel_err(y, y_ref)
-        assert err.max() <= TOL_FLIP, f"round {rnd}: {err.max():.3e}"
+        assert err.max() <= cap, f"round {rnd}: {err.max():.3e}"
         errs.append(err.ravel())
         p.commit(accepted_lengths(wl, rnd, 8))
         p.check_bookkeeping(ring=False)
     errs = np.concatenate(errs)
+    print(f"verify {hp}/{read}: max {errs.max():.3e}, fraction above 1e-4 {float(np.mean(errs > TOL_F32)):.4f}")
     if hp == "f32":
         assert float(np.mean(errs > TOL_F32)) <= FLIP_FRACTION
     assert p.gpu.get_error() == (0, -1)
@@ -247,13 +256,15 @@ def test_skip_steps_match_oracle(cuda_ok, hp, read):
     and checkpoints against the oracle that skips the same reads, and some heads really skipped."""
     wl = FAST_DECAY
     p = Pair(wl, hp=hp, read=read, seed=5, skip_tau=1e-2)
-    tol = TOL_F32 if hp == "f32" and read == "same" else TOL_FLIP
-    skipped = 0
+    tol = TOL_F32 if hp == "f32" and read == "same" else TOL_FLIP if hp == "f32" else TOL_SR_HEAD
+    skipped, worst = 0, 0.0
     for t in range(3 * wl.window + 5):
         skipped += int(p.orc.skip.sum())
         y, y_ref, _ = p.step(gdn_step_inputs(wl, t))
+        worst = max(worst, head_rel_err(y, y_ref).max())
         assert head_rel_err(y, y_ref).max() <= tol, f"step {t}"
         p.check_bookkeeping(ring=(t % 8 == 7))
+    print(f"skip {hp}/{read}: max {worst:.3e}")
     assert skipped > 0
     if hp == "f32":
         p.check_checkpoint()
