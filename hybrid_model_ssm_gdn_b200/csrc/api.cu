@@ -108,10 +108,11 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   a.grid = a.units < x->num_sms ? a.units : x->num_sms;
   a.hp_mode = c.hp; a.read_mode = c.read; a.seed = c.seed; a.q_scale = c.q_scale;
   const int esz = esize(c);
-  const int extra = g_extra_smem_bytes(c.read);
+  const int extra = g_extra_smem_bytes(a.L, esz, c.hp, c.read);
   a.nstage = x->nstage_override > 0 ? x->nstage_override
-                                    : g_max_stages(a.DV, a.L, a.tmax, esz, x->smem_optin - 1024 - extra);
-  if (a.nstage < 2 || a.nstage > 8 || g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) + extra > x->smem_optin)
+                                    : g_max_stages(a.DV, a.L, a.tmax, esz, c.hp, c.read, x->smem_optin - 1024 - extra);
+  if (a.nstage < 2 || a.nstage > 8 ||
+      g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage, c.hp, c.read) + extra > x->smem_optin)
     return RSSM_ERR_SHAPE;
   a.meta_in = meta_cur(x); a.meta_out = meta_next(x); a.err = err_word(x);
   a.hp = x->arena + x->lay.hp;

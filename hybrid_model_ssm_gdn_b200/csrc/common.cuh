@@ -92,6 +92,7 @@ inline ArenaLayout make_layout(const rssm_config &c) {
 // ------------------------------------------------------------------------------------------
 // loads / conversions
 
+__device__ __forceinline__ float4 f4zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
@@ -279,6 +280,24 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// four 8x8 b16 matrices from shared memory; lane l gives the (16-byte aligned) address of row l & 7 of
+// matrix l >> 3, and register q of lane 4g+t receives elements 2t, 2t+1 of row g of matrix q
+__device__ __forceinline__ void ldmatrix_x4(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p))
+               : "memory");
+}
+
+// the same with each 8x8 matrix transposed: register q of lane 4g+t receives rows 2t, 2t+1 of column g
+__device__ __forceinline__ void ldmatrix_x4_trans(const void *p, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                                  uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(p))
+               : "memory");
+}
+
 // ---- register-operand tensor-core tile (warp-wide): d[16x8] += a[16x16] b[16x8], bf16 in, fp32 accumulate.
 // Lane 4g+t holds a = {A[g][2t..2t+1], A[g+8][2t..2t+1], A[g][2t+8..2t+9], A[g+8][2t+8..2t+9]},
 // b = {B[2t..2t+1][g], B[2t+8..2t+9][g]}, d = {D[g][2t..2t+1], D[g+8][2t..2t+1]}; the lower-indexed
@@ -299,6 +318,19 @@ __device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t &hi, uin
   const __nv_bfloat162 l = __floats2bfloat162_rn(x - __uint_as_float(hb << 16), y - __uint_as_float(hb & 0xffff0000u));
   hi = hb;
   lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// fp32 pair -> bf16 pairs hi + mid + lo, each piece the leading 16 bits of what the previous ones left.
+// The split is exact: a fp32 significand has 24 bits, each piece takes the leading 8 of the remainder,
+// and the subtractions x - piece are exact, so hi + mid + lo == x.
+__device__ __forceinline__ void split3_bf16x2(float x, float y, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
+  const uint32_t xb = __float_as_uint(x), yb = __float_as_uint(y);
+  hi = __byte_perm(xb, yb, 0x7632);
+  const float x1 = x - __uint_as_float(xb & 0xffff0000u), y1 = y - __uint_as_float(yb & 0xffff0000u);
+  const uint32_t x1b = __float_as_uint(x1), y1b = __float_as_uint(y1);
+  mid = __byte_perm(x1b, y1b, 0x7632);
+  const float x2 = x1 - __uint_as_float(x1b & 0xffff0000u), y2 = y1 - __uint_as_float(y1b & 0xffff0000u);
+  lo = __byte_perm(__float_as_uint(x2), __float_as_uint(y2), 0x7632);
 }
 
 }  // namespace rssm

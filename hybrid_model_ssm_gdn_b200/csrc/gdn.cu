@@ -65,22 +65,39 @@ constexpr int kTileMaxBytes = kFp4Rows * kCols * 4;  // a 64-row fp32 tile
 
 __host__ __device__ inline int g_heads_per_unit(int no) { return no == 1 ? 4 : no == 2 ? 4 : no == 4 ? 2 : 1; }
 
+// Chunked fold.  Folding m records into a row s of the state is, with a_r = prod_{j<=r} alpha_j,
+// b_r = prod_{r<j<m} alpha_j, z_r = s . k_r and u the per-record coefficients of the sequential rule,
+//     u = T rt,  rt_r = beta_r (v_r[row] - a_r z_r),  T = (I + L)^-1,
+//     L_ri = beta_r (prod_{i<j<=r} alpha_j) (k_i . k_r)  (i < r),
+//     s' = a_{m-1} s + sum_r b_r u_r k_r,
+// the rank-m form of the delta rule's product of elementary factors.  For an fp32 checkpoint with bf16
+// inputs and m <= kChMax the consumers run it on the tensor cores per 16-row block: Z = S K^T, U = RT T^T and
+// S' = a_{m-1} S + W K with W = b U, each fp32 operand cut into three bf16 pieces whose sum is exact.  Per
+// head the prep warps leave T (16 x 16, zero past m), a_r and b_r in the tables, and reorder the folded K rows
+// in the group buffer (pitch 272 bytes) so that both K operands load with ldmatrix, free of bank conflicts.
+constexpr int kChMax = 16;
+constexpr int kChT = kChMax * kChMax;               // T[r][i], row-major
+constexpr int kChStride = kChT + 2 * kChMax + 4;    // per head: T, a_r, b_r (+4: heads in different banks)
+// the kernel instance and window for which folds take the chunked form
+__host__ __device__ inline bool g_chunked(bool lp, int esz, int L) { return !lp && esz == 2 && L <= kChMax; }
+
 struct GLayout {
-  int no, rmax, hg, nrb, dts;
+  int no, rmax, hg, nrb, dts, kpe;        // kpe: element pitch of the K rows in the group buffer
   int gb_k, gb_q, gb_a, gb_b, gb_bytes;   // group buffer
-  int tb_u0, tb_coef, tb_ab, tb_amax, tab_bytes; // tables (per buffer)
+  int tb_u0, tb_coef, tb_ab, tb_amax, tb_ch, tab_bytes; // tables (per buffer)
   int st_g, st_v, stage_bytes;            // tile stage: [tile 32 KiB][g chunk 16 B][v records]
 };
 
-__host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz) {
+__host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz, bool chunk) {
   GLayout l;
   l.no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
   l.rmax = L + (tmax > 1 ? tmax : 1);
   l.hg = g_heads_per_unit(l.no);
   l.nrb = (R + kFp4Rows - 1) / kFp4Rows;
   l.dts = dt_stride(L);
+  l.kpe = kCols + (chunk ? 16 / esz : 0);
   l.gb_k = kGHdrBytes;
-  l.gb_q = (int)align_up((size_t)l.gb_k + (size_t)l.hg * l.rmax * kCols * esz, 16);
+  l.gb_q = (int)align_up((size_t)l.gb_k + (size_t)l.hg * l.rmax * l.kpe * esz, 16);
   l.gb_a = (int)align_up((size_t)l.gb_q + (size_t)l.hg * l.no * kCols * esz, 16);
   l.gb_b = l.gb_a + l.hg * l.dts * 4;
   l.gb_bytes = (int)align_up((size_t)l.gb_b + (size_t)l.hg * l.dts * 4, 128);
@@ -88,7 +105,8 @@ __host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz) {
   l.tb_coef = l.hg * l.no * kCols * 4;
   l.tb_ab = (int)align_up((size_t)l.tb_coef + (size_t)l.hg * l.no * l.rmax * 4, 16);  // {a, b, 1/a, 0}[hg][rmax]
   l.tb_amax = l.tb_ab + l.hg * l.rmax * 16;
-  l.tab_bytes = (int)align_up((size_t)l.tb_amax + 2 * 8 * 4, 128);   // amax[slot][warp]
+  l.tb_ch = l.tb_amax + 2 * 8 * 4;                                    // amax[slot][warp]
+  l.tab_bytes = (int)align_up((size_t)l.tb_ch + (chunk ? (size_t)l.hg * kChStride * 4 : 0), 128);
   l.st_g = kTileMaxBytes;
   l.st_v = l.st_g + 16;
   l.stage_bytes = (int)align_up((size_t)l.st_v + (size_t)l.rmax * R * esz, 128);
@@ -122,7 +140,9 @@ template <typename TI, int NO, bool LP>
 __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int esz = sizeof(TI);
-  const GLayout lay = g_layout(a.DV, a.L, a.tmax, esz);
+  constexpr bool kChunk = !LP && sizeof(TI) == 2;
+  const bool chunk = kChunk && a.L <= kChMax;  // every fold takes the chunked form (m <= L)
+  const GLayout lay = g_layout(a.DV, a.L, a.tmax, esz, chunk);
   const int NS = a.nstage, R = a.DV, L = a.L, HG = lay.hg, nrb = lay.nrb, dts = lay.dts;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + 8;
@@ -253,7 +273,11 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       }
       __syncwarp();
       if (S.active) {
-        const int per_head = 1 + S.n_new + S.t_out;
+        // a unit that folds in the chunked form takes its K rows at the padded pitch (the ring part row by row)
+        const bool krows = lay.kpe != kCols && S.m > 0;
+        const uint32_t kp = krows ? (uint32_t)lay.kpe * esz : krow;
+        const int nrc = krows ? S.n_ring : 1;  // copies of the ring part of a head's K rows
+        const int per_head = nrc + S.n_new + S.t_out;
         const int ncopy = nh * per_head + 2;
         for (int q = lane; q < ncopy; q += 32) {
           if (q == ncopy - 2) {
@@ -263,18 +287,21 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           } else {
             const int i = q / per_head, w = q % per_head;
             const size_t unit = (size_t)S.b * a.H + S.h0 + i;
-            unsigned char *kd = gb + lay.gb_k + (size_t)i * lay.rmax * krow;
-            if (w == 0) {
-              if (S.n_ring)
+            unsigned char *kd = gb + lay.gb_k + (size_t)i * lay.rmax * kp;
+            if (w < nrc) {
+              if (krows)
+                bulk_g2s(kd + w * kp, reinterpret_cast<const unsigned char *>(a.ring_k) + (unit * 2 * L + S.base_e + w) * krow,
+                         krow, &gfull[gs], pol_keep);
+              else if (S.n_ring)
                 bulk_g2s(kd, reinterpret_cast<const unsigned char *>(a.ring_k) + (unit * 2 * L + S.base_e) * krow,
                          S.n_ring * krow, &gfull[gs], pol_keep);
-            } else if (w <= S.n_new) {
-              const int t = w - 1;
-              bulk_g2s(kd + (S.n_ring + t) * krow,
+            } else if (w < nrc + S.n_new) {
+              const int t = w - nrc;
+              bulk_g2s(kd + (S.n_ring + t) * kp,
                        reinterpret_cast<const unsigned char *>(a.k) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * krow,
                        krow, &gfull[gs], pol_keep);
             } else {
-              const int t = w - 1 - S.n_new;
+              const int t = w - nrc - S.n_new;
               bulk_g2s(gb + lay.gb_q + ((size_t)i * lay.no + t) * krow,
                        reinterpret_cast<const unsigned char *>(a.q) + (((size_t)S.b * a.T + t) * a.H + S.h0 + i) * krow,
                        krow, &gfull[gs], pol_keep);
@@ -414,6 +441,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
       const int active = gh[Q_ACTIVE];
       const int n_rec = gh[Q_NREC], m = gh[Q_M], n_ring = gh[Q_NRING], n_new = gh[Q_NNEW], t_out = gh[Q_TOUT];
       const int slot0 = gh[Q_SLOT0], base_e = gh[Q_BASE];
+      const int kpe = lay.kpe != kCols && m > 0 ? lay.kpe : kCols;  // K row pitch of this unit (elements)
       if (active) {
         // alpha, beta of the new tokens (global loads) -> header; append k, alpha, beta to the ring
         for (int q = pw * 32 + lane; q < n_new * nh; q += 64) {
@@ -430,7 +458,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
         for (int q = pw * 32 + lane; q < n_new * nh * kq; q += 64) {
           const int c16 = q % kq, ti2 = q / kq, t = ti2 / nh, i = ti2 % nh;
           const size_t unit = (size_t)b * a.H + h0 + i;
-          const uint4 v = *reinterpret_cast<const uint4 *>(gb + lay.gb_k + ((size_t)i * lay.rmax + n_ring + t) * kCols * esz + c16 * 16);
+          const uint4 v = *reinterpret_cast<const uint4 *>(gb + lay.gb_k + ((size_t)i * lay.rmax + n_ring + t) * kpe * esz + c16 * 16);
           *reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(a.ring_k) + ((unit * 2 * L + slot0 + t) * kCols) * esz +
                                      c16 * 16) = v;
         }
@@ -472,7 +500,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           };
           float kn[16], aln = 0.f, ben = 0.f;
           if (e_j - 1 >= m) {
-            load_k16(kg + ((size_t)i * lay.rmax + (e_j - 1)) * kCols + sl * 16, kn);
+            load_k16(kg + ((size_t)i * lay.rmax + (e_j - 1)) * kpe + sl * 16, kn);
             gate(e_j - 1, aln, ben);
           }
           for (int r = e_j - 1; r >= m; --r) {
@@ -481,7 +509,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             for (int z = 0; z < 16; ++z) kv[z] = kn[z];
             const float al = aln, be = ben;
             if (r > m) {
-              load_k16(kg + ((size_t)i * lay.rmax + (r - 1)) * kCols + sl * 16, kn);
+              load_k16(kg + ((size_t)i * lay.rmax + (r - 1)) * kpe + sl * 16, kn);
               gate(r - 1, aln, ben);
             }
             float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
@@ -519,6 +547,98 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           abt[i * lay.rmax + r] = make_float4(al, be, __frcp_rn(al), 0.f);
         }
       }
+      if (chunk && active && m > 0) {
+        // chunked fold tables.  (1) The folded K rows (r < m) take the column order of the consumers' fragments:
+        // in each 16-column chunk, columns {0,1,4,5,8,9,12,13} then {2,3,6,7,10,11,14,15} (bf16 pairs stay
+        // together); the ring copies of the new rows were written above in the natural order, and the
+        // walk-back reads only rows >= m.
+        float *cht = reinterpret_cast<float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_ch);
+        const int kpb = kpe * 2;
+        for (int q = pw * 32 + lane; q < nh * m * 8; q += 64) {
+          const int ih = q / (m * 8), rr = (q >> 3) % m, c = q & 7;
+          uint4 *p = reinterpret_cast<uint4 *>(gb + lay.gb_k + ((size_t)ih * lay.rmax + rr) * kpb + c * 32);
+          const uint4 w0 = p[0], w1 = p[1];
+          p[0] = make_uint4(w0.x, w0.z, w1.x, w1.z);
+          p[1] = make_uint4(w0.y, w0.w, w1.y, w1.w);
+        }
+        if (!prep_sync()) {  // K rows reordered
+          if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+          break;
+        }
+        // (2) Per head (warp pw: heads pw, pw + 2), G = K K^T over the first 16 records on the tensor cores
+        // (bf16 products exact, fp32 sums; rows past m repeat row m - 1): the ldmatrix fragments of K serve as
+        // both operands.  The lane's accumulator entries (x, y) with x < y < m give
+        // L_yx = beta_y (prod_{x<j<=y} alpha_j) G_xy, stored at T[y][x].
+        const float *ag = reinterpret_cast<const float *>(gb + lay.gb_a);
+        const float *bg = reinterpret_cast<const float *>(gb + lay.gb_b);
+        auto alpha_of = [&](int ih, int r) { return r < n_ring ? ag[ih * dts + base_e + r] : gf[Q_F + (r - n_ring) * 8 + ih]; };
+        const int gq = lane >> 2, tq = lane & 3;
+        for (int ih = pw; ih < nh; ih += 2) {
+          const unsigned char *kh = gb + lay.gb_k + ((size_t)ih * lay.rmax + min(lane & 15, m - 1)) * kpb + (lane >> 4) * 16;
+          float g0[4] = {0.f, 0.f, 0.f, 0.f}, g1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < kCols / 16; ++ks) {
+            uint32_t r0, r1, r2, r3;
+            ldmatrix_x4(kh + ks * 32, r0, r1, r2, r3);
+            mma_16816(g0, r0, r1, r2, r3, r0, r2);
+            mma_16816(g1, r0, r1, r2, r3, r1, r3);
+          }
+          float al[kChMax];
+#pragma unroll
+          for (int j = 0; j < kChMax; ++j) al[j] = j < m ? alpha_of(ih, j) : 1.f;
+          const float gv[8] = {g0[0], g0[1], g0[2], g0[3], g1[0], g1[1], g1[2], g1[3]};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int x = gq + 8 * ((q >> 1) & 1), y = 2 * tq + (q & 1) + 8 * (q >> 2);
+            if (x < y && y < m) {
+              float pf = y < n_ring ? bg[ih * dts + base_e + y] : gf[Q_FB + (y - n_ring) * 8 + ih];
+#pragma unroll
+              for (int j = 1; j < kChMax; ++j)
+                if (j > x && j <= y) pf *= al[j];
+              cht[ih * kChStride + y * kChMax + x] = pf * gv[q];
+            }
+          }
+        }
+        if (!prep_sync()) {  // L complete
+          if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+          break;
+        }
+        // (3) T = (I + L)^-1 by forward substitution, lanes 0-15 and 16-31 one column each of two heads; the
+        // whole 16 x 16 matrix is written (zero above the diagonal and past m), then a_r and b_r in record order
+        for (int h2 = pw * 2; h2 < nh; h2 += 4) {
+          const int ih = h2 + (lane >> 4), j = lane & 15;  // column j of head ih
+          const bool hv = ih < nh;
+          float *ch = cht + (hv ? ih : 0) * kChStride;
+          float tcol[kChMax];  // T[r][j]
+#pragma unroll
+          for (int r = 0; r < kChMax; ++r) {
+            float v = (r == j && j < m) ? 1.f : 0.f;
+            if (hv && r > j && r < m) {
+              float acc = 0.f;
+#pragma unroll
+              for (int i2 = 0; i2 < r; ++i2)
+                if (i2 >= j) acc = fmaf(ch[r * kChMax + i2], tcol[i2], acc);
+              v = -acc;
+            }
+            tcol[r] = v;
+          }
+          __syncwarp();  // every lane has read L before T overwrites it
+          if (hv) {
+#pragma unroll
+            for (int r = 0; r < kChMax; ++r) ch[r * kChMax + j] = tcol[r];
+            float ar = 0.f, br = 0.f;
+            if (j < m) {
+              ar = 1.f;
+              br = 1.f;
+              for (int jj = 0; jj <= j; ++jj) ar *= alpha_of(ih, jj);
+              for (int jj = j + 1; jj < m; ++jj) br *= alpha_of(ih, jj);
+            }
+            ch[kChT + j] = ar;
+            ch[kChT + kChMax + j] = br;
+          }
+          __syncwarp();
+        }
+      }
       if (!prep_sync()) {  // tables complete
         if (lane == 0) { record_error(a.err, 0, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
         break;
@@ -532,6 +652,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     const uint64_t pol_wr = policy_evict_first();
     const uint64_t pol_ring = policy_evict_last();
     int ti = 0, rdv = 0, fd = 0;  // fd: fold tiles done (the two-axis copy's scratch slot rotates with it)
+    int cft = 0;                  // chunked fold tiles seen (every consumer warp sees every tile)
+
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
       if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag, ws)) {
@@ -569,7 +691,14 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
           // the new tokens' v rows, landed behind the buffered ones in the head's first tile
           // stage, go to the head's ring row with one bulk store (warps take turns); every warp
           // waits for its bulk stores to have read the stage before releasing it
-          if (t == 0 && n_new > 0 && (ti & (kConsumerWarps - 1)) == warp && lane == 0) {
+          // a chunked fold tile is taken by one group of four warps (alternating); the other group only
+          // waits for it to land (so that its release cannot count for the stage's previous use) and releases it
+          const bool gtile = fold && chunk;
+          const int grp = cft & 1;
+          cft += gtile ? 1 : 0;
+          const bool mine = !gtile || (warp >> 2) == grp;
+          const int vw = gtile ? 4 * grp + (ti & 3) : (ti & (kConsumerWarps - 1));
+          if (t == 0 && n_new > 0 && vw == warp && lane == 0) {
             const uint32_t vrow = (uint32_t)R * esz;
             bulk_s2g(reinterpret_cast<unsigned char *>(a.ring_v) + (unit * 2 * a.L + slot0) * vrow,
                      st + lay.st_v + (size_t)n_ring * vrow, (uint32_t)n_new * vrow, pol_ring);
@@ -600,7 +729,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             const float4 e = e2m1x4_to_float4(cw);
             return make_float4(__fmul_rn(e.x, d_b), __fmul_rn(e.y, d_b), __fmul_rn(e.z, d_b), __fmul_rn(e.w, d_b));
           };
-          if (!fold) {
+          if (!mine) {
+          } else if (!fold) {
             // ---------------- non-fold tile: lane owns columns 4l..4l+3 of the warp's 8 rows
             if (row0 < rows) {
               constexpr int V = 8 * NO;
@@ -672,6 +802,178 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                   a.y[(((size_t)b * a.T + j) * a.H + h) * R + kFp4Rows * t + row0 + rr] = part[k2];
               }
             }
+          } else if (chunk) {
+            // ---------------- chunked fold tile: warp (w & 3) of the group owns rows 16(w & 3) .. +15 and computes
+            // their new state alone.  Lane 4g+t holds rows ra = 16(w & 3) + g and rb = ra + 8, and in each
+            // 16-column chunk c the columns 16c + 4t .. +3, which the reordered K rows match as fragments.
+            const float *cht = reinterpret_cast<const float *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_ch) +
+                               i * kChStride;
+            const float4 *abt = reinterpret_cast<const float4 *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_ab) +
+                                (size_t)i * lay.rmax;
+            const int kpb = lay.kpe * 2;  // K row pitch in bytes (bf16)
+            const unsigned char *kb = gb + lay.gb_k + (size_t)i * lay.rmax * kpb;
+            unsigned char *stw = stages + (size_t)s * lay.stage_bytes;
+            const int gq = lane >> 2, qtr = lane & 3, odd = gq & 1;
+            const int wr0 = 16 * (warp & 3), ra = wr0 + gq, rb = ra + 8;
+            const bool va = ra < rows, vb = rb < rows;
+            const bool skp = (skm >> i) & 1u;  // a skipped head folds from zero
+            const bool la = va && !skp, lb = vb && !skp;
+            const int rga = kFp4Rows * t + ra, rgb = rga + 8;  // rows within the head's state
+            auto srow = [&](int r, int c) { return reinterpret_cast<float4 *>(stw + ((size_t)r * kCols + 16 * c + 4 * qtr) * 4); };
+            // chunks cp and cp + 1 of rows ra, rb from the stage; rows of odd g take the pair in the other order,
+            // so that the loads (and the stores back) are free of bank conflicts
+            auto load_pair = [&](int cp, float4 (&xa)[2], float4 (&xb)[2]) {
+              const int c0 = cp + odd, c1 = cp + 1 - odd;
+              const float4 pa = la ? *srow(ra, c0) : f4zero(), pb = lb ? *srow(rb, c0) : f4zero();
+              const float4 qa = la ? *srow(ra, c1) : f4zero(), qb = lb ? *srow(rb, c1) : f4zero();
+              xa[0] = odd ? qa : pa; xa[1] = odd ? pa : qa;
+              xb[0] = odd ? qb : pb; xb[1] = odd ? pb : qb;
+            };
+            // phase 1: Z = S K^T for records 0-7 and 8-15 (rows past m repeat row m - 1; their columns of Z are
+            // not used), S in three exact bf16 pieces, small pieces first
+            float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+            const bool two = m > 8;
+            const unsigned char *kl = kb + (size_t)min((lane & 7) + 8 * (lane >> 4), m - 1) * kpb + ((lane >> 3) & 1) * 16;
+#pragma unroll
+            for (int cp = 0; cp < 8; cp += 2) {
+              float4 xa[2], xb[2];
+              load_pair(cp, xa, xb);
+#pragma unroll
+              for (int o = 0; o < 2; ++o) {
+                uint32_t hp[3][4];
+                split3_bf16x2(xa[o].x, xa[o].y, hp[0][0], hp[1][0], hp[2][0]);
+                split3_bf16x2(xb[o].x, xb[o].y, hp[0][1], hp[1][1], hp[2][1]);
+                split3_bf16x2(xa[o].z, xa[o].w, hp[0][2], hp[1][2], hp[2][2]);
+                split3_bf16x2(xb[o].z, xb[o].w, hp[0][3], hp[1][3], hp[2][3]);
+                uint32_t q0, q1, q2, q3;  // B of records 0-7 (q0, q1) and 8-15 (q2, q3)
+                ldmatrix_x4(kl + (cp + o) * 32, q0, q1, q2, q3);
+#pragma unroll
+                for (int p = 2; p >= 0; --p) mma_16816(z0, hp[p][0], hp[p][1], hp[p][2], hp[p][3], q0, q1);
+                if (two) {
+#pragma unroll
+                  for (int p = 2; p >= 0; --p) mma_16816(z1, hp[p][0], hp[p][1], hp[p][2], hp[p][3], q2, q3);
+                }
+              }
+            }
+            // phase 2: rt_r = beta_r (v_r[row] - a_r z_r) for the lane's records 2t, 2t+1, 2t+8, 2t+9 (zero past
+            // m), then U = RT T^T on the tensor cores (both fp32 operands in three pieces; the six piece
+            // products above 2^-24 kept): U lands on the lane's own records, as the A operand of phase 3 wants
+            float rta[4], rtb[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 2 * qtr + (k & 1) + 8 * (k >> 1);
+              const float za = k < 2 ? z0[k & 1] : z1[k & 1];
+              const float zb = k < 2 ? z0[2 + (k & 1)] : z1[2 + (k & 1)];
+              float xa = 0.f, xb = 0.f;
+              if (r < m) {
+                const float be = abt[r].y, ar = cht[kChT + r];
+                xa = be * ((va ? to_f32(vr[r * R + rga]) : 0.f) - ar * za);
+                xb = be * ((vb ? to_f32(vr[r * R + rgb]) : 0.f) - ar * zb);
+              }
+              rta[k] = xa;
+              rtb[k] = xb;
+            }
+            float wa[4], wb[4];
+            {
+              uint32_t rp[3][4];
+              split3_bf16x2(rta[0], rta[1], rp[0][0], rp[1][0], rp[2][0]);
+              split3_bf16x2(rtb[0], rtb[1], rp[0][1], rp[1][1], rp[2][1]);
+              split3_bf16x2(rta[2], rta[3], rp[0][2], rp[1][2], rp[2][2]);
+              split3_bf16x2(rtb[2], rtb[3], rp[0][3], rp[1][3], rp[2][3]);
+              float u[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                const float *tr = cht + (8 * nt + gq) * kChMax + 2 * qtr;  // B[i][r] = T[r][i], r = 8nt + g
+                const float2 t0 = *reinterpret_cast<const float2 *>(tr), t1 = *reinterpret_cast<const float2 *>(tr + 8);
+                uint32_t tp0[3], tp1[3];
+                split3_bf16x2(t0.x, t0.y, tp0[0], tp0[1], tp0[2]);
+                split3_bf16x2(t1.x, t1.y, tp1[0], tp1[1], tp1[2]);
+                constexpr int kPa[6] = {2, 1, 0, 1, 0, 0}, kPb[6] = {0, 1, 2, 0, 1, 0};
+#pragma unroll
+                for (int q = 0; q < 6; ++q)
+                  mma_16816(u[nt], rp[kPa[q]][0], rp[kPa[q]][1], rp[kPa[q]][2], rp[kPa[q]][3], tp0[kPb[q]], tp1[kPb[q]]);
+              }
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int r = 2 * qtr + (k & 1) + 8 * (k >> 1);
+                const float br = cht[kChT + kChMax + r];  // zero past m
+                wa[k] = br * u[k >> 1][k & 1];
+                wb[k] = br * u[k >> 1][2 + (k & 1)];
+              }
+            }
+            // phase 3: S' = a_{m-1} S + W K over 16 n-tiles: B from the reordered K rows with ldmatrix.trans
+            // (records past m masked to zero), D on the lane's own columns
+            uint32_t wp[3][4];
+            split3_bf16x2(wa[0], wa[1], wp[0][0], wp[1][0], wp[2][0]);
+            split3_bf16x2(wb[0], wb[1], wp[0][1], wp[1][1], wp[2][1]);
+            split3_bf16x2(wa[2], wa[3], wp[0][2], wp[1][2], wp[2][2]);
+            split3_bf16x2(wb[2], wb[3], wp[0][3], wp[1][3], wp[2][3]);
+            const float am = cht[kChT + m - 1];
+            const uint32_t mk0 = (2 * qtr < m ? 0xFFFFu : 0u) | (2 * qtr + 1 < m ? 0xFFFF0000u : 0u);
+            const uint32_t mk1 = (2 * qtr + 8 < m ? 0xFFFFu : 0u) | (2 * qtr + 9 < m ? 0xFFFF0000u : 0u);
+            const unsigned char *kt = kb + (size_t)min((lane & 7) + 8 * ((lane >> 3) & 1), m - 1) * kpb + (lane >> 4) * 16;
+            // S is read again from the stage chunk pair by chunk pair, and S' goes back to the same place
+#pragma unroll
+            for (int cp = 0; cp < 8; cp += 2) {
+              float4 xa[2], xb[2];
+              load_pair(cp, xa, xb);
+#pragma unroll
+              for (int o2 = 0; o2 < 2; ++o2) {
+                const int c = cp + o2;
+                uint32_t q0, q1, q2, q3;  // n-tile (c, 0): q0 (records 0-7), q1 (8-15); n-tile (c, 1): q2, q3
+                ldmatrix_x4_trans(kt + c * 32, q0, q1, q2, q3);
+#pragma unroll
+                for (int o = 0; o < 2; ++o) {
+                  const uint32_t b0 = (o ? q2 : q0) & mk0, b1 = (o ? q3 : q1) & mk1;
+                  float d[4];
+                  if (o == 0) { d[0] = xa[o2].x * am; d[1] = xa[o2].y * am; d[2] = xb[o2].x * am; d[3] = xb[o2].y * am; }
+                  else        { d[0] = xa[o2].z * am; d[1] = xa[o2].w * am; d[2] = xb[o2].z * am; d[3] = xb[o2].w * am; }
+#pragma unroll
+                  for (int p = 2; p >= 0; --p) mma_16816(d, wp[p][0], wp[p][1], wp[p][2], wp[p][3], b0, b1);
+                  if (o == 0) { xa[o2].x = d[0]; xa[o2].y = d[1]; xb[o2].x = d[2]; xb[o2].y = d[3]; }
+                  else        { xa[o2].z = d[0]; xa[o2].w = d[1]; xb[o2].z = d[2]; xb[o2].w = d[3]; }
+                }
+              }
+              const int c0 = cp + odd, c1 = cp + 1 - odd;
+              *srow(ra, c0) = odd ? xa[1] : xa[0];
+              *srow(rb, c0) = odd ? xb[1] : xb[0];
+              *srow(ra, c1) = odd ? xa[0] : xa[1];
+              *srow(rb, c1) = odd ? xb[0] : xb[1];
+            }
+            // the outputs from S' (each lane reads back what it wrote; u_0 carries q_scale), the buffered
+            // records past the fold, then the quad's partial sums
+            for (int j = 0; j < t_out; ++j) {
+              const int e_j = n_rec - t_out + j + 1;
+              float ya = 0.f, yb = 0.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int cc = c ^ odd;  // odd rows in the other chunk order, as written
+                const float4 u = *reinterpret_cast<const float4 *>(u0_h + j * kCols + 16 * cc + 4 * qtr);
+                const float4 sa = *srow(ra, cc), sb = *srow(rb, cc);
+                ya = fmaf(sa.x, u.x, fmaf(sa.y, u.y, fmaf(sa.z, u.z, fmaf(sa.w, u.w, ya))));
+                yb = fmaf(sb.x, u.x, fmaf(sb.y, u.y, fmaf(sb.z, u.z, fmaf(sb.w, u.w, yb))));
+              }
+              for (int r = m + qtr; r < e_j; r += 4) {
+                const float co = co_h[j * lay.rmax + r];
+                if (va) ya = fmaf(co, to_f32(vr[r * R + rga]), ya);
+                if (vb) yb = fmaf(co, to_f32(vr[r * R + rgb]), yb);
+              }
+              ya += __shfl_xor_sync(0xffffffffu, ya, 1);
+              yb += __shfl_xor_sync(0xffffffffu, yb, 1);
+              ya += __shfl_xor_sync(0xffffffffu, ya, 2);
+              yb += __shfl_xor_sync(0xffffffffu, yb, 2);
+              float *yj = a.y + (((size_t)b * a.T + j) * a.H + h) * R;
+              if (qtr == 0 && va) yj[rga] = ya;
+              if (qtr == 0 && vb) yj[rgb] = yb;
+            }
+            fence_async_smem();
+            __syncwarp();
+            const int wrows = min(16, rows - wr0);
+            if (lane == 0 && wrows > 0) {
+              bulk_s2g(static_cast<unsigned char *>(a.hp) + (unit * R + kFp4Rows * t + wr0) * kCols * 4,
+                       stw + (size_t)wr0 * kCols * 4, (uint32_t)(wrows * kCols * 4), pol_wr);
+              bulk_commit();
+            }
           } else {
             // ---------------- fold tile: four lanes per row, 32 columns each, chunks rotated by lane
             const int qtr = lane & 3;
@@ -692,7 +994,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             const float4 *abt = reinterpret_cast<const float4 *>(tabs + (size_t)tsl * lay.tab_bytes + lay.tb_ab) +
                                 (size_t)i * lay.rmax;
             for (int r = 0; r < m; ++r) {
-              const TI *kr = kg + ((size_t)i * lay.rmax + r) * kCols + qtr * 32;
+              const TI *kr = kg + ((size_t)i * lay.rmax + r) * lay.kpe + qtr * 32;
               float4 kv[8];
 #pragma unroll
               for (int c = 0; c < 8; ++c) kv[c] = load4(kr + ((c + lane) & 7) * 4);
@@ -925,18 +1227,25 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
 
 }  // namespace
 
-int g_smem_bytes(int R, int L, int tmax, int esz, int nstage) {
-  const GLayout l = g_layout(R, L, tmax, esz);
+static bool g_lowprec(int hp_mode, int read_mode) { return hp_mode != RSSM_HP_F32 || read_mode != RSSM_READ_SAME; }
+
+int g_smem_bytes(int R, int L, int tmax, int esz, int nstage, int hp_mode, int read_mode) {
+  const GLayout l = g_layout(R, L, tmax, esz, g_chunked(g_lowprec(hp_mode, read_mode), esz, L));
   return kBarBytesG + 2 * l.tab_bytes + kGBG * l.gb_bytes + nstage * l.stage_bytes;
 }
 
-int g_max_stages(int R, int L, int tmax, int esz, int budget) {
+int g_max_stages(int R, int L, int tmax, int esz, int hp_mode, int read_mode, int budget) {
   int n = 8;
-  while (n > 2 && g_smem_bytes(R, L, tmax, esz, n) > budget) --n;
+  while (n > 2 && g_smem_bytes(R, L, tmax, esz, n, hp_mode, read_mode) > budget) --n;
   return n;
 }
 
-int g_extra_smem_bytes(int read_mode) { return read_mode == RSSM_READ_NVFP4D ? kCmBytes : 0; }
+int g_extra_smem_bytes(int L, int esz, int hp_mode, int read_mode) {
+  (void)L;
+  (void)esz;
+  (void)hp_mode;
+  return read_mode == RSSM_READ_NVFP4D ? kCmBytes : 0;
+}
 
 int g_units(int Bt, int H, int tmax) {
   const int no = tmax <= 1 ? 1 : tmax <= 2 ? 2 : tmax <= 4 ? 4 : 8;
@@ -946,9 +1255,10 @@ int g_units(int Bt, int H, int tmax) {
 
 cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream) {
   const int no = a.tmax <= 1 ? 1 : a.tmax <= 2 ? 2 : a.tmax <= 4 ? 4 : 8;
-  const size_t smem = g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage) + g_extra_smem_bytes(a.read_mode);
+  const size_t smem = g_smem_bytes(a.DV, a.L, a.tmax, esz, a.nstage, a.hp_mode, a.read_mode) +
+                      g_extra_smem_bytes(a.L, esz, a.hp_mode, a.read_mode);
   void (*kern)(GArgs) = nullptr;
-  const bool lp = a.hp_mode != RSSM_HP_F32 || a.read_mode != RSSM_READ_SAME;
+  const bool lp = g_lowprec(a.hp_mode, a.read_mode);
 #define RSSM_PICK(TI, NOV) \
   if (no == NOV) kern = lp ? gdn_replay_kernel<TI, NOV, true> : gdn_replay_kernel<TI, NOV, false>;
   if (esz == 2) {

@@ -63,9 +63,10 @@ struct GArgs {
   unsigned int suspend_ns;        // suspend-time hint of each try_wait (0: the hardware's default)
   int withhold;                   // test hook: no block fills its tile with this index (-1: off)
 };
-int g_smem_bytes(int R, int L, int tmax, int esz, int nstage);
-int g_extra_smem_bytes(int read_mode);  // fold scratch of the two-axis read copy
-int g_max_stages(int R, int L, int tmax, int esz, int budget);
+int g_smem_bytes(int R, int L, int tmax, int esz, int nstage, int hp_mode, int read_mode);
+// fold scratch behind the stages: the two-axis read copy's column maxima, or the chunked fold's Z / W
+int g_extra_smem_bytes(int L, int esz, int hp_mode, int read_mode);
+int g_max_stages(int R, int L, int tmax, int esz, int hp_mode, int read_mode, int budget);
 int g_units(int Bt, int H, int tmax);  // work units: (sequence, chunk of heads)
 cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream);
 

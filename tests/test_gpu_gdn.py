@@ -48,6 +48,26 @@ def test_ragged_rows_and_heads(cuda_ok):
     p.check_checkpoint()
 
 
+@pytest.mark.parametrize("dv,nheads,L", [(40, 3, 16), (96, 5, 16), (128, 3, 5), (72, 2, 1)])
+def test_chunked_fold_shapes(cuda_ok, dv, nheads, L):
+    """The fold of an fp32 checkpoint with bf16 inputs runs in the chunked form (Z = S K^T, U = RT T^T,
+    S' = a S + W K on the tensor cores, one group of four warps per tile): partial 16-row blocks (d_v = 40, 72),
+    a 32-row tile (96), windows that fold 16, 5 and 1 records, and verify rounds whose pre-folds take every
+    committed count from 1 to L."""
+    wl = SMALL.replace(batch=3, nheads=nheads, dv=dv, window=L)
+    T = min(4, L)  # drafts per verify are at most the window
+    p = Pair(wl, max_draft=T)
+    run_steps(p, 2 * L + 3, check_every=L)
+    p.check_checkpoint()
+    for rnd in range(8):
+        y, _, y_true = p.verify(T, gdn_draft_inputs(wl, rnd, T))
+        assert head_rel_err(y, y_true).max() <= TOL_F32
+        p.commit(accepted_lengths(wl, rnd, T))
+        p.check_bookkeeping()
+    p.check_checkpoint()
+    assert p.gpu.get_error() == (0, -1)
+
+
 def test_many_units(cuda_ok):
     """More units than SMs, not a multiple of them (151 sequences x 2 units)."""
     wl = SMALL.replace(batch=151, nheads=8)

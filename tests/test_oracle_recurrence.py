@@ -202,3 +202,37 @@ def test_replay_equals_stepwise_gdn_workload_shape():
         y_rep = rc.gdn_replay_output(S0, recs, tok["q"])
         assert np.linalg.norm(y_rep - y) <= 1e-12 * np.linalg.norm(y)
     assert np.linalg.norm(rc.gdn_fold(S0, recs) - S) <= 1e-12 * np.linalg.norm(S)
+
+
+@pytest.mark.parametrize("m,decay", [(1, 0.05), (5, 0.05), (16, 0.05), (16, 3.0)])
+def test_gdn_fold_rank_m_form(m, decay):
+    """The chunked form the GPU fold uses equals folding the records one by one: with a_r = prod_{j<=r} alpha_j,
+    b_r = prod_{r<j<m} alpha_j, L_ri = beta_r (prod_{i<j<=r} alpha_j) k_i.k_r (i < r) and T = (I + L)^-1,
+    each row s becomes a_{m-1} s + sum_r b_r u_r k_r with u = T rt, rt_r = beta_r (v_r[row] - a_r s.k_r).
+    Written out here in float64 with numpy's inverse; decay 3.0 spreads alpha down to ~0.05 (products far
+    below one), and m = 1 leaves L empty."""
+    from synth import GDN_B256, gdn_initial_state, gdn_step_inputs
+    wl = GDN_B256.replace(batch=2, nheads=3, decay_scale=decay)
+    S0 = gdn_initial_state(wl).astype(np.float64)
+    recs = [gdn_step_inputs(wl, t) for t in range(m)]
+    want = rc.gdn_fold(S0, recs)
+    K = np.stack([np.asarray(r["k"], np.float64) for r in recs], axis=-2)        # [B, H, m, dk]
+    V = np.stack([np.asarray(r["v"], np.float64) for r in recs], axis=-1)        # [B, H, dv, m]
+    al = np.stack([np.asarray(r["alpha"], np.float64) for r in recs], axis=-1)   # [B, H, m]
+    be = np.stack([np.asarray(r["beta"], np.float64) for r in recs], axis=-1)
+    got = np.empty_like(want)
+    for b in range(wl.batch):
+        for h in range(wl.nheads):
+            k, v, a_, bt = K[b, h], V[b, h], al[b, h], be[b, h]
+            a = np.cumprod(a_)
+            bsuf = np.array([np.prod(a_[r + 1:]) for r in range(m)])
+            L = np.zeros((m, m))
+            for r in range(m):
+                for i in range(r):
+                    L[r, i] = bt[r] * np.prod(a_[i + 1:r + 1]) * (k[i] @ k[r])
+            T = np.linalg.inv(np.eye(m) + L)
+            Z = S0[b, h] @ k.T                                  # [dv, m]
+            rt = bt[None, :] * (v - a[None, :] * Z)
+            U = rt @ T.T
+            got[b, h] = a[-1] * S0[b, h] + (U * bsuf[None, :]) @ k
+    assert np.linalg.norm(got - want) <= 1e-12 * np.linalg.norm(want)
