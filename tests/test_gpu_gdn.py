@@ -48,14 +48,14 @@ def test_ragged_rows_and_heads(cuda_ok):
     p.check_checkpoint()
 
 
-@pytest.mark.parametrize("dv,nheads,L", [(40, 3, 16), (96, 5, 16), (128, 3, 5), (72, 2, 1)])
-def test_chunked_fold_shapes(cuda_ok, dv, nheads, L):
+@pytest.mark.parametrize("dv,nheads,L,T", [(40, 3, 16, 4), (96, 5, 16, 8), (128, 3, 5, 4), (72, 2, 1, 1),
+                                            (128, 2, 16, 2), (96, 3, 12, 8)])
+def test_chunked_fold_shapes(cuda_ok, dv, nheads, L, T):
     """The fold of an fp32 checkpoint with bf16 inputs runs in the chunked form (Z = S K^T, U = RT T^T,
     S' = a S + W K on the tensor cores, one group of four warps per tile): partial 16-row blocks (d_v = 40, 72),
-    a 32-row tile (96), windows that fold 16, 5 and 1 records, and verify rounds whose pre-folds take every
-    committed count from 1 to L."""
+    a 32-row tile (96), windows that fold 16, 12, 5 and 1 records, and verify rounds of 1 to 8 drafts whose
+    pre-folds take every committed count from 1 to L (their outputs then come from the chunked fold result)."""
     wl = SMALL.replace(batch=3, nheads=nheads, dv=dv, window=L)
-    T = min(4, L)  # drafts per verify are at most the window
     p = Pair(wl, max_draft=T)
     run_steps(p, 2 * L + 3, check_every=L)
     p.check_checkpoint()
