@@ -125,6 +125,17 @@ constexpr int kColScaleOff = kTileMaxBytes / 2 + 1024;
 constexpr int kCmSlotWords = (kFp4Rows / 16) * kCols;
 constexpr int kCmBytes = 3 * kCmSlotWords * 4 + kCmSlotWords * 4;
 
+// d[16x8] += a[16x8] b[8x8], tf32 in (fp32 registers whose low 13 bits are zero), fp32 accumulate.
+// Lane 4g+t holds a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]}, b = {B[t][g], B[t+4][g]},
+// d = {D[g][2t..2t+1], D[g+8][2t..2t+1]}.
+__device__ __forceinline__ void mma_1688_tf32(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 template <typename TI>
 __device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 consecutive elements
 #pragma unroll
@@ -830,28 +841,38 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               xb[0] = odd ? qb : pb; xb[1] = odd ? pb : qb;
             };
             // phase 1: Z = S K^T for records 0-7 and 8-15 (rows past m repeat row m - 1; their columns of Z are
-            // not used), S in three exact bf16 pieces, small pieces first
+            // not used) in tf32: per 16-column chunk two k-steps of 8 (lane t's columns 4t, 4t+1, then 4t+2,
+            // 4t+3), S in two tf32 pieces (hi: the leading 11 bits, lo: the next 11, so |s - hi - lo| < 2^-20 |s|),
+            // K exact (a bf16 widened); the small pieces first
             float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
             const bool two = m > 8;
             const unsigned char *kl = kb + (size_t)min((lane & 7) + 8 * (lane >> 4), m - 1) * kpb + ((lane >> 3) & 1) * 16;
+            auto tf32_split = [](float x, uint32_t &hi, uint32_t &lo) {
+              hi = __float_as_uint(x) & 0xffffe000u;
+              lo = __float_as_uint(x - __uint_as_float(hi)) & 0xffffe000u;
+            };
 #pragma unroll
             for (int cp = 0; cp < 8; cp += 2) {
               float4 xa[2], xb[2];
               load_pair(cp, xa, xb);
 #pragma unroll
               for (int o = 0; o < 2; ++o) {
-                uint32_t hp[3][4];
-                split3_bf16x2(xa[o].x, xa[o].y, hp[0][0], hp[1][0], hp[2][0]);
-                split3_bf16x2(xb[o].x, xb[o].y, hp[0][1], hp[1][1], hp[2][1]);
-                split3_bf16x2(xa[o].z, xa[o].w, hp[0][2], hp[1][2], hp[2][2]);
-                split3_bf16x2(xb[o].z, xb[o].w, hp[0][3], hp[1][3], hp[2][3]);
-                uint32_t q0, q1, q2, q3;  // B of records 0-7 (q0, q1) and 8-15 (q2, q3)
+                uint32_t q0, q1, q2, q3;  // records 0-7: columns (4t, 4t+1) in q0, (4t+2, 4t+3) in q1; 8-15: q2, q3
                 ldmatrix_x4(kl + (cp + o) * 32, q0, q1, q2, q3);
+                uint32_t ah[2][4], al[2][4];  // [k-step][fragment register]
+                tf32_split(xa[o].x, ah[0][0], al[0][0]); tf32_split(xb[o].x, ah[0][1], al[0][1]);
+                tf32_split(xa[o].y, ah[0][2], al[0][2]); tf32_split(xb[o].y, ah[0][3], al[0][3]);
+                tf32_split(xa[o].z, ah[1][0], al[1][0]); tf32_split(xb[o].z, ah[1][1], al[1][1]);
+                tf32_split(xa[o].w, ah[1][2], al[1][2]); tf32_split(xb[o].w, ah[1][3], al[1][3]);
 #pragma unroll
-                for (int p = 2; p >= 0; --p) mma_16816(z0, hp[p][0], hp[p][1], hp[p][2], hp[p][3], q0, q1);
-                if (two) {
-#pragma unroll
-                  for (int p = 2; p >= 0; --p) mma_16816(z1, hp[p][0], hp[p][1], hp[p][2], hp[p][3], q2, q3);
+                for (int kk = 0; kk < 2; ++kk) {
+                  const uint32_t w0 = kk ? q1 : q0, w1 = kk ? q3 : q2;
+                  mma_1688_tf32(z0, al[kk][0], al[kk][1], al[kk][2], al[kk][3], w0 << 16, w0 & 0xffff0000u);
+                  mma_1688_tf32(z0, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], w0 << 16, w0 & 0xffff0000u);
+                  if (two) {
+                    mma_1688_tf32(z1, al[kk][0], al[kk][1], al[kk][2], al[kk][3], w1 << 16, w1 & 0xffff0000u);
+                    mma_1688_tf32(z1, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], w1 << 16, w1 & 0xffff0000u);
+                  }
                 }
               }
             }
