@@ -25,6 +25,9 @@ struct rssm_ctx {
   long long wait_cycles;   // bound of the kernels' waits (RSSM_WAIT_CYCLES, default ~1 s)
   unsigned int suspend_ns; // suspend-time hint of the kernels' barrier polls (RSSM_SUSPEND_NS)
   int withhold;            // test hook RSSM_WITHHOLD_TILE (-1: off)
+  // every sequence's record count in the window when the host knows it (only steps since the checkpoint was
+  // loaded or fully flushed), else -1.  It picks the kernel instance of a step; both fold correctly.
+  int pos;
 };
 
 namespace {
@@ -66,6 +69,16 @@ rssm_status validate(const rssm_config *c) {
   return RSSM_OK;
 }
 
+// a step the host knows to fold nowhere: every sequence's count is known and stays below the window
+bool known_fold_free(const rssm_ctx *x, int op) { return op == OP_STEP && x->pos >= 0 && x->pos + 1 < x->cfg.window; }
+
+// the record count after a successful call (rssm_ctx::pos)
+void advance_pos(rssm_ctx *x, int op, const unsigned char *mask) {
+  if (op == OP_STEP && x->pos >= 0) x->pos = x->pos + 1 == x->cfg.window ? 0 : x->pos + 1;
+  else if (op == OP_FLUSH && mask == nullptr) x->pos = 0;
+  else x->pos = -1;
+}
+
 const int4 *meta_cur(rssm_ctx *x) { return reinterpret_cast<const int4 *>(x->arena + x->lay.meta) + x->parity * x->cfg.batch; }
 int4 *meta_next(rssm_ctx *x) { return reinterpret_cast<int4 *>(x->arena + x->lay.meta) + (1 - x->parity) * x->cfg.batch; }
 int *err_word(rssm_ctx *x) { return reinterpret_cast<int *>(x->arena + x->lay.err); }
@@ -78,6 +91,7 @@ rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, c
   a.Bt = c.batch; a.H = c.nheads; a.P = c.headdim; a.G = c.ngroups; a.L = c.window;
   a.T = T; a.tmax = op == OP_VERIFY ? T : 1; a.op = op;
   a.units = m2_units(c.batch, c.nheads, c.ngroups);
+  a.fold_free = known_fold_free(x, op);
   a.grid = a.units < x->num_sms ? a.units : x->num_sms;
   const int esz = esize(c);
   a.nstage = x->nstage_override > 0 ? x->nstage_override : m2_max_stages(a.P, a.L, a.tmax, esz, x->smem_optin - 1024);
@@ -94,6 +108,7 @@ rssm_status run_m2(rssm_ctx *x, int op, int T, const void *xin, const void *B, c
   cudaError_t e = launch_m2_replay(a, esz, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity ^= 1;
+  advance_pos(x, op, mask);
   return RSSM_OK;
 }
 
@@ -105,6 +120,7 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   a.Bt = c.batch; a.H = c.nheads; a.DV = c.headdim; a.L = c.window;
   a.T = T; a.tmax = op == OP_VERIFY ? T : 1; a.op = op;
   a.units = g_units(c.batch, c.nheads, a.tmax);
+  a.fold_free = known_fold_free(x, op);
   a.grid = a.units < x->num_sms ? a.units : x->num_sms;
   a.hp_mode = c.hp; a.read_mode = c.read; a.seed = c.seed; a.q_scale = c.q_scale;
   const int esz = esize(c);
@@ -130,6 +146,7 @@ rssm_status run_gdn(rssm_ctx *x, int op, int T, const void *q, const void *k, co
   cudaError_t e = launch_gdn_replay(a, esz, stream);
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity ^= 1;
+  advance_pos(x, op, mask);
   return RSSM_OK;
 }
 
@@ -175,6 +192,7 @@ rssm_status rssm_create(const rssm_config *cfg, void *arena, size_t arena_bytes,
   x->cfg = *cfg;
   x->lay = lay;
   x->arena = static_cast<unsigned char *>(arena);
+  x->pos = -1;
   x->parity = 0;
   x->num_sms = sms;
   x->smem_optin = optin;
@@ -222,6 +240,7 @@ rssm_status rssm_load_checkpoint(rssm_ctx *x, const float *S, rssm_stream stream
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity = 0;
   x->loaded = 1;
+  x->pos = 0;
   return RSSM_OK;
 }
 
@@ -263,6 +282,7 @@ rssm_status rssm_commit(rssm_ctx *x, const int *accepted, rssm_stream stream) {
                                 reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   x->parity ^= 1;
+  x->pos = -1;
   return RSSM_OK;
 }
 

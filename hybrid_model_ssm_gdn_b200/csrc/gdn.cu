@@ -146,12 +146,14 @@ __device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 c
 }
 
 // LP: the context stores a low-precision checkpoint or keeps an NVFP4 read copy.  LP = false
-// compiles the fp32-checkpoint path alone, with every format branch folded away.
-template <typename TI, int NO, bool LP>
+// compiles the fp32-checkpoint path alone, with every format branch folded away.  CF: the instance with the
+// chunked fold (fp32 checkpoint, bf16 inputs); steps the host knows to be fold-free take the instance without
+// it, whose streaming path then compiles as it did before the chunked fold.  Both fold correctly.
+template <typename TI, int NO, bool LP, bool CF>
 __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int esz = sizeof(TI);
-  constexpr bool kChunk = !LP && sizeof(TI) == 2;
+  constexpr bool kChunk = CF && !LP && sizeof(TI) == 2;
   const bool chunk = kChunk && a.L <= kChMax;  // every fold takes the chunked form (m <= L)
   const GLayout lay = g_layout(a.DV, a.L, a.tmax, esz, chunk);
   const int NS = a.nstage, R = a.DV, L = a.L, HG = lay.hg, nrb = lay.nrb, dts = lay.dts;
@@ -1280,12 +1282,14 @@ cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream) {
                       g_extra_smem_bytes(a.L, esz, a.hp_mode, a.read_mode);
   void (*kern)(GArgs) = nullptr;
   const bool lp = g_lowprec(a.hp_mode, a.read_mode);
-#define RSSM_PICK(TI, NOV) \
-  if (no == NOV) kern = lp ? gdn_replay_kernel<TI, NOV, true> : gdn_replay_kernel<TI, NOV, false>;
+#define RSSM_PICK(TI, NOV, CFV) \
+  if (no == NOV) kern = lp ? gdn_replay_kernel<TI, NOV, true, false> : gdn_replay_kernel<TI, NOV, false, CFV>;
   if (esz == 2) {
-    RSSM_PICK(__nv_bfloat16, 1) RSSM_PICK(__nv_bfloat16, 2) RSSM_PICK(__nv_bfloat16, 4) RSSM_PICK(__nv_bfloat16, 8)
+    RSSM_PICK(__nv_bfloat16, 1, true) RSSM_PICK(__nv_bfloat16, 2, true) RSSM_PICK(__nv_bfloat16, 4, true)
+    RSSM_PICK(__nv_bfloat16, 8, true)
+    if (no == 1 && !lp && a.fold_free) kern = gdn_replay_kernel<__nv_bfloat16, 1, false, false>;
   } else {
-    RSSM_PICK(float, 1) RSSM_PICK(float, 2) RSSM_PICK(float, 4) RSSM_PICK(float, 8)
+    RSSM_PICK(float, 1, false) RSSM_PICK(float, 2, false) RSSM_PICK(float, 4, false) RSSM_PICK(float, 8, false)
   }
 #undef RSSM_PICK
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

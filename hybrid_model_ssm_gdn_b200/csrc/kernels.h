@@ -14,6 +14,7 @@ struct M2Args {
   int tmax;       // sizes the per-stage record area: L + max(tmax, 1) records
   int op;
   int units;      // Bt * H
+  int fold_free;  // the host knows that no unit of this launch folds (the instance without the chunked fold)
   int grid, nstage, stage_base;
   const int4 *meta_in;
   int4 *meta_out;
@@ -40,6 +41,7 @@ cudaError_t launch_m2_replay(M2Args a, int esz, cudaStream_t stream);
 struct GArgs {
   int Bt, H, DV, L;
   int T, tmax, op, units, grid, nstage, stage_base;
+  int fold_free;  // the host knows that no unit of this launch folds (the instance without the chunked fold)
   int hp_mode, read_mode;         // rssm_hp, rssm_read
   unsigned long long seed;
   float q_scale;

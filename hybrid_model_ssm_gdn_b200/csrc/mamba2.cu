@@ -31,9 +31,12 @@
 //    products, transpose reduction, buffered part of y), appends the head's new x rows
 //    with one bulk store when it is its turn, and releases the stage on its own.  With
 //    bf16 inputs and 5..8 outputs, S'.C and the buffered term run on tensor cores
-//    (mma.sync, register operands).  No block-wide barrier sits on the streaming path,
-//    so one block per SM keeps the checkpoint stream in flight while the next unit is
-//    being prepared.
+//    (mma.sync, register operands).  With bf16 inputs, one output and windows up to 16, a
+//    fold tile is taken by one group of four consumer warps (the groups alternate), each
+//    warp owning 16 rows: S' = af S + X' B on tensor cores, X' = wf_r x_r cut into three
+//    bf16 pieces whose sum is exact, B the group's records reordered by the prep warp for
+//    ldmatrix.trans.  No block-wide barrier sits on the streaming path, so one block per SM
+//    keeps the checkpoint stream in flight while the next unit is being prepared.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -53,6 +56,8 @@ enum {
   G_DT = G_D + kHG           // dt of new tokens [8][16]
 };
 
+constexpr int kBkPitch = 272;  // bytes per reordered B record (128 bf16 + 16)
+
 struct M2Layout {
   int rmax, no;
   bool mma;                  // output contraction on tensor cores (bf16 inputs, 8 outputs per row)
@@ -62,6 +67,7 @@ struct M2Layout {
   int stage_bytes;
   int gb_B, gb_C, gb_dt, gb_bytes;  // group buffer
   int tab_bytes;
+  int tb_bk;                 // chunked fold: the folded B records, reordered, in each table buffer (0: none)
   int cx_bytes;              // fold scratch: per consumer warp, wf_r x_r[row] for its 8 rows
 };
 
@@ -82,7 +88,12 @@ __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
   // [kHG][nq][32 lanes][4 words]), ao[kHG][no], wf[kHG][rmax], af[kHG], flags[8]
   const int coef_floats = l.mma ? kHG * l.nq * 32 * 4 : kHG * l.no * l.rmax;
   const int floats = l.no * l.rmax + coef_floats + kHG * l.no + kHG * l.rmax + kHG + 8;
-  l.tab_bytes = (int)align_up((size_t)floats * 4, 128);
+  // chunked fold (bf16 inputs, CUDA-core output path, windows up to 16): the folded B records, reordered for
+  // ldmatrix.trans at a pitch of 272 bytes (no bank conflicts), in each table buffer
+  const bool tcf = esz == 2 && l.no == 1 && L <= 16;
+  const size_t tb = align_up((size_t)floats * 4, 16);
+  l.tb_bk = tcf ? (int)tb : 0;
+  l.tab_bytes = (int)align_up(tb + (tcf ? (size_t)16 * kBkPitch : 0), 128);
   l.cx_bytes = (int)align_up((size_t)kConsumerWarps * l.rmax * 8 * 4, 128);
   return l;
 }
@@ -93,7 +104,11 @@ constexpr int kGB = 3;  // group buffers: the producer loads a unit's group data
 constexpr int kM2Threads = kConsumers + 64;  // + producer warp + prep warp
 constexpr int kProducerWarp = kConsumerWarps, kPrepWarp = kConsumerWarps + 1;
 
-template <typename TI, int NO>
+// TCF: the instance with the chunked fold on tensor cores (bf16 inputs, one output, windows up to 16).  Launches
+// the host knows to be fold-free take the instance without it: its streaming path compiles as it did before the
+// chunked fold (plain launches measured 5% slower with the fold code present, whether inline or out of line, and
+// with the register allocation capped).  Both instances fold correctly; the choice only affects speed.
+template <typename TI, int NO, bool TCF>
 __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
   // S'.C_j on tensor cores for 5..8 drafts (measured: at 4 the CUDA-core reduction is as fast): C_j is
@@ -507,6 +522,20 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
           T.af[i] = __expf(A * sfx);
         }
       }
+      if (TCF && lay.tb_bk > 0 && gh[G_ACTIVE] && gh[G_M] > 0) {
+        // the folded B records (r < m) as the chunked fold's B operand: in each 16-column chunk, columns
+        // {0,1,4,5,8,9,12,13} then {2,3,6,7,10,11,14,15} (bf16 pairs stay together), at a pitch of 272 bytes
+        const int mf = gh[G_M];
+        unsigned char *bk = tabs + (size_t)tsl * lay.tab_bytes + lay.tb_bk;
+        for (int q = lane; q < mf * 8; q += 32) {
+          const int r = q >> 3, c = q & 7;
+          const uint4 *src = reinterpret_cast<const uint4 *>(gb + lay.gb_B + (size_t)r * kCols * 2 + c * 32);
+          const uint4 w0 = src[0], w1 = src[1];
+          uint4 *dst = reinterpret_cast<uint4 *>(bk + (size_t)r * kBkPitch + c * 32);
+          dst[0] = make_uint4(w0.x, w0.z, w1.x, w1.z);
+          dst[1] = make_uint4(w0.y, w0.w, w1.y, w1.w);
+        }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&tfull[tsl]);
     }
@@ -515,6 +544,7 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
     const int row0 = warp * 8;
     const uint64_t pol_ring = policy_evict_last();
     int ti = 0;
+    int cft = 0;  // chunked fold tiles seen (every consumer warp sees every tile)
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGB, tsl = gi & 1;
       if (!mbar_wait_or_abort(&tfull[tsl], (uint32_t)((gi >> 1) & 1), abort_flag, ws)) {
@@ -565,17 +595,129 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
           const TI *xr = reinterpret_cast<const TI *>(st + lay.xr);
           const int h = h0 + i;
           const size_t unit = (size_t)b * a.H + h;
+          // a fold tile of the chunked form is taken by one group of four warps (alternating); the other group
+          // only waits for it to land (so that its release cannot count for the stage's previous use)
+          const bool gtile = TCF && lay.tb_bk > 0 && m > 0;
+          const int grp = cft & 1;
+          cft += gtile ? 1 : 0;
+          const bool mine = !gtile || (warp >> 2) == grp;
           // the new tokens' x rows, landed in the stage behind the buffered ones, go to the head's
           // ring row with one bulk store (warps take turns); the stage is released after it has
           // been read
-          const bool appender = (ti & (kConsumerWarps - 1)) == warp && n_new > 0;
+          const bool appender = (gtile ? 4 * grp + (ti & 3) : (ti & (kConsumerWarps - 1))) == warp && n_new > 0;
           if (appender && lane == 0) {
             const uint32_t xrow = (uint32_t)a.P * esz;
             bulk_s2g(reinterpret_cast<unsigned char *>(a.ring_x) + (unit * 2 * a.L + slot0) * xrow,
                      st + lay.xr + (size_t)n_ring * xrow, (uint32_t)n_new * xrow, pol_ring);
             bulk_commit();
           }
-          if (row0 < a.P) {
+          if (!mine) {
+          } else if (gtile) {
+            // ---- chunked fold: S' = af S + X' B with X'[row][r] = wf_r x_r[row] (r < m <= 16) on the tensor
+            // cores.  Warp (w & 3) of the group owns rows 16(w & 3) .. +15; lane 4g+t holds rows ra = .. + g and
+            // rb = ra + 8 and, in each 16-column chunk c, the columns 16c + 4t .. +3, which the reordered B
+            // records match as fragments.  X' is cut into three bf16 pieces whose sum is exact; B is exact.
+            const int gq = lane >> 2, qtr = lane & 3, odd = gq & 1;
+            const int ra = 16 * (warp & 3) + gq, rb = ra + 8;
+            const bool va = ra < a.P, vb = rb < a.P;
+            const bool skp = (skm >> i) & 1u;  // a skipped head folds from zero
+            const bool la = va && !skp, lb = vb && !skp;
+            float *tw = const_cast<float *>(tile);
+            auto srow = [&](int r, int c) { return reinterpret_cast<float4 *>(tw + (size_t)r * kCols + 16 * c + 4 * qtr); };
+            float xa4[4], xb4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 2 * qtr + (k & 1) + 8 * (k >> 1);
+              float u = 0.f, v = 0.f;
+              if (r < m) {
+                const float wr = t_wf[i * rmax + r];
+                if (va) u = wr * to_f32(xr[r * a.P + ra]);
+                if (vb) v = wr * to_f32(xr[r * a.P + rb]);
+              }
+              xa4[k] = u;
+              xb4[k] = v;
+            }
+            uint32_t wp[3][4];
+            split3_bf16x2(xa4[0], xa4[1], wp[0][0], wp[1][0], wp[2][0]);
+            split3_bf16x2(xb4[0], xb4[1], wp[0][1], wp[1][1], wp[2][1]);
+            split3_bf16x2(xa4[2], xa4[3], wp[0][2], wp[1][2], wp[2][2]);
+            split3_bf16x2(xb4[2], xb4[3], wp[0][3], wp[1][3], wp[2][3]);
+            const float af = t_af[i];
+            const unsigned char *kt = tabs + (size_t)tsl * lay.tab_bytes + lay.tb_bk +
+                                      (size_t)min((lane & 7) + 8 * ((lane >> 3) & 1), m - 1) * kBkPitch + (lane >> 4) * 16;
+            float *dst = a.hp + unit * a.P * kCols;
+#pragma unroll
+            for (int cp = 0; cp < 8; cp += 2) {
+              // rows of odd g take the chunk pair in the other order: no bank conflicts
+              const int c0 = cp + odd, c1 = cp + 1 - odd;
+              float4 xa[2], xb[2];
+              {
+                const float4 pa = la ? *srow(ra, c0) : f4zero(), pb = lb ? *srow(rb, c0) : f4zero();
+                const float4 qa = la ? *srow(ra, c1) : f4zero(), qb = lb ? *srow(rb, c1) : f4zero();
+                xa[0] = odd ? qa : pa; xa[1] = odd ? pa : qa;
+                xb[0] = odd ? qb : pb; xb[1] = odd ? pb : qb;
+              }
+#pragma unroll
+              for (int o2 = 0; o2 < 2; ++o2) {
+                uint32_t q0, q1, q2, q3;  // n-tile (chunk, 0): q0 (records 0-7), q1 (8-15); (chunk, 1): q2, q3
+                ldmatrix_x4_trans(kt + (cp + o2) * 32, q0, q1, q2, q3);
+#pragma unroll
+                for (int o = 0; o < 2; ++o) {
+                  float d[4];
+                  if (o == 0) { d[0] = xa[o2].x * af; d[1] = xa[o2].y * af; d[2] = xb[o2].x * af; d[3] = xb[o2].y * af; }
+                  else        { d[0] = xa[o2].z * af; d[1] = xa[o2].w * af; d[2] = xb[o2].z * af; d[3] = xb[o2].w * af; }
+#pragma unroll
+                  for (int pz = 2; pz >= 0; --pz) mma_16816(d, wp[pz][0], wp[pz][1], wp[pz][2], wp[pz][3], o ? q2 : q0, o ? q3 : q1);
+                  if (o == 0) { xa[o2].x = d[0]; xa[o2].y = d[1]; xb[o2].x = d[2]; xb[o2].y = d[3]; }
+                  else        { xa[o2].z = d[0]; xa[o2].w = d[1]; xb[o2].z = d[2]; xb[o2].w = d[3]; }
+                }
+              }
+              if (va) {
+                *srow(ra, c0) = odd ? xa[1] : xa[0];
+                *srow(ra, c1) = odd ? xa[0] : xa[1];
+                __stcs(reinterpret_cast<float4 *>(dst + (size_t)ra * kCols + 16 * cp + 4 * qtr), xa[0]);
+                __stcs(reinterpret_cast<float4 *>(dst + (size_t)ra * kCols + 16 * (cp + 1) + 4 * qtr), xa[1]);
+              }
+              if (vb) {
+                *srow(rb, c0) = odd ? xb[1] : xb[0];
+                *srow(rb, c1) = odd ? xb[0] : xb[1];
+                __stcs(reinterpret_cast<float4 *>(dst + (size_t)rb * kCols + 16 * cp + 4 * qtr), xb[0]);
+                __stcs(reinterpret_cast<float4 *>(dst + (size_t)rb * kCols + 16 * (cp + 1) + 4 * qtr), xb[1]);
+              }
+            }
+            // outputs from S' (each lane reads back what it wrote): ao_j (S' . C_j) + sum_r coef_jr x_r[row]
+            for (int j = 0; j < t_out; ++j) {
+              float ya = 0.f, yb = 0.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int cc = c ^ odd;  // odd rows in the other chunk order, as written
+                const float4 cj = load4(Cg + j * kCols + 16 * cc + 4 * qtr);
+                if (va) {
+                  const float4 sa = *srow(ra, cc);
+                  ya = fmaf(sa.x, cj.x, fmaf(sa.y, cj.y, fmaf(sa.z, cj.z, fmaf(sa.w, cj.w, ya))));
+                }
+                if (vb) {
+                  const float4 sb = *srow(rb, cc);
+                  yb = fmaf(sb.x, cj.x, fmaf(sb.y, cj.y, fmaf(sb.z, cj.z, fmaf(sb.w, cj.w, yb))));
+                }
+              }
+              const float ao = t_ao[i * NO + j];
+              ya *= ao;
+              yb *= ao;
+              for (int r = qtr; r < n_rec; r += 4) {
+                const float co = t_coef[(i * NO + j) * rmax + r];
+                if (va) ya = fmaf(co, to_f32(xr[r * a.P + ra]), ya);
+                if (vb) yb = fmaf(co, to_f32(xr[r * a.P + rb]), yb);
+              }
+              ya += __shfl_xor_sync(0xffffffffu, ya, 1);
+              yb += __shfl_xor_sync(0xffffffffu, yb, 1);
+              ya += __shfl_xor_sync(0xffffffffu, ya, 2);
+              yb += __shfl_xor_sync(0xffffffffu, yb, 2);
+              float *yj = a.y + (((size_t)b * a.T + j) * a.H + h) * a.P;
+              if (qtr == 0 && va) yj[ra] = ya;
+              if (qtr == 0 && vb) yj[rb] = yb;
+            }
+          } else if (row0 < a.P) {
             // a head flagged for decay-aware skipping has no tile in the stage: its checkpoint term is zero
             const bool skp = (skm >> i) & 1u;
             float4 sv[8];
@@ -747,9 +889,10 @@ cudaError_t launch_m2_replay(M2Args a, int esz, cudaStream_t stream) {
   const size_t smem = m2_smem_bytes(a.P, a.L, a.tmax, esz, a.nstage);
   void (*kern)(M2Args) = nullptr;
 #define RSSM_PICK(TI, NOV) \
-  if (no == NOV) kern = m2_replay_kernel<TI, NOV>;
+  if (no == NOV) kern = m2_replay_kernel<TI, NOV, false>;
   if (esz == 2) {
     RSSM_PICK(__nv_bfloat16, 1) RSSM_PICK(__nv_bfloat16, 2) RSSM_PICK(__nv_bfloat16, 4) RSSM_PICK(__nv_bfloat16, 8)
+    if (no == 1 && !a.fold_free) kern = m2_replay_kernel<__nv_bfloat16, 1, true>;
   } else {
     RSSM_PICK(float, 1) RSSM_PICK(float, 2) RSSM_PICK(float, 4) RSSM_PICK(float, 8)
   }
