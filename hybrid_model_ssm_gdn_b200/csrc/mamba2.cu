@@ -90,7 +90,7 @@ __host__ __device__ inline M2Layout m2_layout(int P, int L, int tmax, int esz) {
   const int floats = l.no * l.rmax + coef_floats + kHG * l.no + kHG * l.rmax + kHG + 8;
   // chunked fold (bf16 inputs, CUDA-core output path, windows up to 16): the folded B records, reordered for
   // ldmatrix.trans at a pitch of 272 bytes (no bank conflicts), in each table buffer
-  const bool tcf = esz == 2 && l.no == 1 && L <= 16;
+  const bool tcf = esz == 2 && (l.no == 1 || l.mma) && L <= 16;
   const size_t tb = align_up((size_t)floats * 4, 16);
   l.tb_bk = tcf ? (int)tb : 0;
   l.tab_bytes = (int)align_up(tb + (tcf ? (size_t)16 * kBkPitch : 0), 128);
@@ -685,37 +685,82 @@ __global__ void __launch_bounds__(kM2Threads, 1) m2_replay_kernel(M2Args a) {
                 __stcs(reinterpret_cast<float4 *>(dst + (size_t)rb * kCols + 16 * (cp + 1) + 4 * qtr), xb[1]);
               }
             }
-            // outputs from S' (each lane reads back what it wrote): ao_j (S' . C_j) + sum_r coef_jr x_r[row]
-            for (int j = 0; j < t_out; ++j) {
-              float ya = 0.f, yb = 0.f;
+            if constexpr (kMma) {
+              // 8 outputs on the tensor cores, as on the streaming path but for the group's 16 rows: S' (read back,
+              // each lane its own values) in bf16 hi and lo pieces times [C_1 .. C_8], then the buffered term
+              // [x_r] times the coefficient fragments of the prep warp
+              float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
-                const int cc = c ^ odd;  // odd rows in the other chunk order, as written
-                const float4 cj = load4(Cg + j * kCols + 16 * cc + 4 * qtr);
-                if (va) {
-                  const float4 sa = *srow(ra, cc);
-                  ya = fmaf(sa.x, cj.x, fmaf(sa.y, cj.y, fmaf(sa.z, cj.z, fmaf(sa.w, cj.w, ya))));
-                }
-                if (vb) {
-                  const float4 sb = *srow(rb, cc);
-                  yb = fmaf(sb.x, cj.x, fmaf(sb.y, cj.y, fmaf(sb.z, cj.z, fmaf(sb.w, cj.w, yb))));
-                }
+                const float4 sa = va ? *srow(ra, c) : f4zero(), sb = vb ? *srow(rb, c) : f4zero();
+                uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
+                split_bf16x2(sa.x, sa.y, h0, l0);
+                split_bf16x2(sb.x, sb.y, h1, l1);
+                split_bf16x2(sa.z, sa.w, h2, l2);
+                split_bf16x2(sb.z, sb.w, h3, l3);
+                mma_16816(d1, l0, l1, l2, l3, ac[c][0], ac[c][1]);
+                mma_16816(d0, h0, h1, h2, h3, ac[c][0], ac[c][1]);
               }
-              const float ao = t_ao[i * NO + j];
-              ya *= ao;
-              yb *= ao;
-              for (int r = qtr; r < n_rec; r += 4) {
-                const float co = t_coef[(i * NO + j) * rmax + r];
-                if (va) ya = fmaf(co, to_f32(xr[r * a.P + ra]), ya);
-                if (vb) yb = fmaf(co, to_f32(xr[r * a.P + rb]), yb);
+              float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+              const uint4 *cf = reinterpret_cast<const uint4 *>(t_coef) + (size_t)i * lay.nq * 32;
+              const unsigned short *xs = reinterpret_cast<const unsigned short *>(xr);
+              for (int q = 0; q * 16 < n_rec; ++q) {
+                const uint4 w = cf[q * 32 + lane];
+                const int r0 = 16 * q + 2 * qtr;
+                auto xw = [&](int r, int row, bool v) -> uint32_t { return (v && r < n_rec) ? xs[r * a.P + row] : 0u; };
+                const uint32_t xa0 = xw(r0, ra, va) | (xw(r0 + 1, ra, va) << 16);
+                const uint32_t xb0 = xw(r0, rb, vb) | (xw(r0 + 1, rb, vb) << 16);
+                const uint32_t xa8 = xw(r0 + 8, ra, va) | (xw(r0 + 9, ra, va) << 16);
+                const uint32_t xb8 = xw(r0 + 8, rb, vb) | (xw(r0 + 9, rb, vb) << 16);
+                mma_16816(e0, xa0, xb0, xa8, xb8, w.x, w.y);
+                mma_16816(e1, xa0, xb0, xa8, xb8, w.z, w.w);
               }
-              ya += __shfl_xor_sync(0xffffffffu, ya, 1);
-              yb += __shfl_xor_sync(0xffffffffu, yb, 1);
-              ya += __shfl_xor_sync(0xffffffffu, ya, 2);
-              yb += __shfl_xor_sync(0xffffffffu, yb, 2);
-              float *yj = a.y + (((size_t)b * a.T + j) * a.H + h) * a.P;
-              if (qtr == 0 && va) yj[ra] = ya;
-              if (qtr == 0 && vb) yj[rb] = yb;
+              const int j0 = 2 * qtr;
+              const size_t jstride = (size_t)a.H * a.P;
+              float *yo = a.y + (((size_t)b * a.T + j0) * a.H + h) * a.P;
+              if (j0 < t_out) {
+                const float ao = t_ao[i * NO + j0];
+                if (va) yo[ra] = ao * (d0[0] + d1[0]) + (e0[0] + e1[0]);
+                if (vb) yo[rb] = ao * (d0[2] + d1[2]) + (e0[2] + e1[2]);
+              }
+              if (j0 + 1 < t_out) {
+                const float ao = t_ao[i * NO + j0 + 1];
+                if (va) yo[jstride + ra] = ao * (d0[1] + d1[1]) + (e0[1] + e1[1]);
+                if (vb) yo[jstride + rb] = ao * (d0[3] + d1[3]) + (e0[3] + e1[3]);
+              }
+            } else {
+              // outputs from S' (each lane reads back what it wrote): ao_j (S' . C_j) + sum_r coef_jr x_r[row]
+              for (int j = 0; j < t_out; ++j) {
+                float ya = 0.f, yb = 0.f;
+  #pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const int cc = c ^ odd;  // odd rows in the other chunk order, as written
+                  const float4 cj = load4(Cg + j * kCols + 16 * cc + 4 * qtr);
+                  if (va) {
+                    const float4 sa = *srow(ra, cc);
+                    ya = fmaf(sa.x, cj.x, fmaf(sa.y, cj.y, fmaf(sa.z, cj.z, fmaf(sa.w, cj.w, ya))));
+                  }
+                  if (vb) {
+                    const float4 sb = *srow(rb, cc);
+                    yb = fmaf(sb.x, cj.x, fmaf(sb.y, cj.y, fmaf(sb.z, cj.z, fmaf(sb.w, cj.w, yb))));
+                  }
+                }
+                const float ao = t_ao[i * NO + j];
+                ya *= ao;
+                yb *= ao;
+                for (int r = qtr; r < n_rec; r += 4) {
+                  const float co = t_coef[(i * NO + j) * rmax + r];
+                  if (va) ya = fmaf(co, to_f32(xr[r * a.P + ra]), ya);
+                  if (vb) yb = fmaf(co, to_f32(xr[r * a.P + rb]), yb);
+                }
+                ya += __shfl_xor_sync(0xffffffffu, ya, 1);
+                yb += __shfl_xor_sync(0xffffffffu, yb, 1);
+                ya += __shfl_xor_sync(0xffffffffu, ya, 2);
+                yb += __shfl_xor_sync(0xffffffffu, yb, 2);
+                float *yj = a.y + (((size_t)b * a.T + j) * a.H + h) * a.P;
+                if (qtr == 0 && va) yj[ra] = ya;
+                if (qtr == 0 && vb) yj[rb] = yb;
+              }
             }
           } else if (row0 < a.P) {
             // a head flagged for decay-aware skipping has no tile in the stage: its checkpoint term is zero
@@ -893,6 +938,7 @@ cudaError_t launch_m2_replay(M2Args a, int esz, cudaStream_t stream) {
   if (esz == 2) {
     RSSM_PICK(__nv_bfloat16, 1) RSSM_PICK(__nv_bfloat16, 2) RSSM_PICK(__nv_bfloat16, 4) RSSM_PICK(__nv_bfloat16, 8)
     if (no == 1 && !a.fold_free) kern = m2_replay_kernel<__nv_bfloat16, 1, true>;
+    if (no == 8) kern = m2_replay_kernel<__nv_bfloat16, 8, true>;
   } else {
     RSSM_PICK(float, 1) RSSM_PICK(float, 2) RSSM_PICK(float, 4) RSSM_PICK(float, 8)
   }
