@@ -78,8 +78,12 @@ __host__ __device__ inline int g_heads_per_unit(int no) { return no == 1 ? 4 : n
 constexpr int kChMax = 16;
 constexpr int kChT = kChMax * kChMax;               // T[r][i], row-major
 constexpr int kChStride = kChT + 2 * kChMax + 4;    // per head: T, a_r, b_r (+4: heads in different banks)
-// the kernel instance and window for which folds take the chunked form
-__host__ __device__ inline bool g_chunked(bool lp, int esz, int L) { return !lp && esz == 2 && L <= kChMax; }
+// the checkpoint formats and window for which folds take the chunked form: an fp32 checkpoint, read as it is
+// or through the NVFP4 copy (re-quantised from the chunked result), with bf16 inputs
+__host__ __device__ inline bool g_chunked(int hp_mode, int read_mode, int esz, int L) {
+  return hp_mode == RSSM_HP_F32 && (read_mode == RSSM_READ_SAME || read_mode == RSSM_READ_NVFP4) && esz == 2 &&
+         L <= kChMax;
+}
 
 struct GLayout {
   int no, rmax, hg, nrb, dts, kpe;        // kpe: element pitch of the K rows in the group buffer
@@ -113,7 +117,7 @@ __host__ __device__ inline GLayout g_layout(int R, int L, int tmax, int esz, boo
   return l;
 }
 
-constexpr int kBarBytesG = 512;  // mbarriers (29 x 8 B) + armed phases + abort flag
+constexpr int kBarBytesG = 512;  // mbarriers (31 x 8 B) + armed phases + abort flag
 constexpr int kGBG = 3;  // group buffers: the producer loads a unit's group data one unit ahead
 
 // tile source formats
@@ -147,14 +151,15 @@ __device__ __forceinline__ void load_k16(const TI *p, float (&o)[16]) {  // 16 c
 
 // LP: the context stores a low-precision checkpoint or keeps an NVFP4 read copy.  LP = false
 // compiles the fp32-checkpoint path alone, with every format branch folded away.  CF: the instance with the
-// chunked fold (fp32 checkpoint, bf16 inputs); steps the host knows to be fold-free take the instance without
-// it, whose streaming path then compiles as it did before the chunked fold.  Both fold correctly.
+// chunked fold (fp32 checkpoint, bf16 inputs, read as it is or through the NVFP4 copy); steps the host knows to be
+// fold-free take the instance without it, whose streaming path then compiles as it did before the chunked fold.
+// Both fold correctly.
 template <typename TI, int NO, bool LP, bool CF>
 __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int esz = sizeof(TI);
-  constexpr bool kChunk = CF && !LP && sizeof(TI) == 2;
-  const bool chunk = kChunk && a.L <= kChMax;  // every fold takes the chunked form (m <= L)
+  constexpr bool kChunk = CF && sizeof(TI) == 2;
+  const bool chunk = kChunk && g_chunked(a.hp_mode, a.read_mode, esz, a.L);  // every fold takes it (m <= L)
   const GLayout lay = g_layout(a.DV, a.L, a.tmax, esz, chunk);
   const int NS = a.nstage, R = a.DV, L = a.L, HG = lay.hg, nrb = lay.nrb, dts = lay.dts;
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
@@ -165,7 +170,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
   uint64_t *tempty = tfull + 2;      // [2] consumers done with the tables
   uint64_t *psync = tempty + 2;      // rendezvous of the two prep warps (count 2)
   uint64_t *fsync = psync + 1;       // rendezvous of the eight consumer warps (NVFP4 tile maximum)
-  volatile int *armed = reinterpret_cast<volatile int *>(fsync + 1);  // [8 + kGBG]
+  uint64_t *csync = fsync + 1;       // [2] rendezvous of a group of four (chunked fold, NVFP4 tile maximum)
+  volatile int *armed = reinterpret_cast<volatile int *>(csync + 2);  // [8 + kGBG]
   volatile int *abort_flag = armed + 8 + kGBG;
   unsigned char *tabs = smem + kBarBytesG;
   unsigned char *gbuf = tabs + 2 * lay.tab_bytes;
@@ -200,6 +206,8 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     }
     mbar_init(psync, 2);
     mbar_init(fsync, kConsumerWarps);
+    mbar_init(&csync[0], 4);
+    mbar_init(&csync[1], 4);
     for (int s = 0; s < 8 + kGBG; ++s) armed[s] = -1;
     *abort_flag = 0;
     fence_barrier_init();
@@ -666,6 +674,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
     const uint64_t pol_ring = policy_evict_last();
     int ti = 0, rdv = 0, fd = 0;  // fd: fold tiles done (the two-axis copy's scratch slot rotates with it)
     int cft = 0;                  // chunked fold tiles seen (every consumer warp sees every tile)
+    int crdv = 0;                 // rendezvous of this warp's group of four (chunked fold, NVFP4 copy)
 
     for (int gi = 0;; ++gi) {
       const int gs = gi % kGBG, tsl = gi & 1;
@@ -845,13 +854,18 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             // phase 1: Z = S K^T for records 0-7 and 8-15 (rows past m repeat row m - 1; their columns of Z are
             // not used) in tf32: per 16-column chunk two k-steps of 8 (lane t's columns 4t, 4t+1, then 4t+2,
             // 4t+3), S in two tf32 pieces (hi: the leading 11 bits, lo: the next 11, so |s - hi - lo| < 2^-20 |s|),
-            // K exact (a bf16 widened); the small pieces first
+            // K exact (a bf16 widened); the small pieces first.  Where the fold result is re-quantised (the
+            // NVFP4 copy), S takes three pieces (the third holds the last 2 bits, so the sum is exact): Z then
+            // carries no representation error, and the copy's decisions follow the fp32 result more closely.
+            constexpr bool kZ3 = LP;
             float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
             const bool two = m > 8;
             const unsigned char *kl = kb + (size_t)min((lane & 7) + 8 * (lane >> 4), m - 1) * kpb + ((lane >> 3) & 1) * 16;
-            auto tf32_split = [](float x, uint32_t &hi, uint32_t &lo) {
+            auto tf32_split = [](float x, uint32_t &hi, uint32_t &lo, uint32_t &lo2) {
               hi = __float_as_uint(x) & 0xffffe000u;
-              lo = __float_as_uint(x - __uint_as_float(hi)) & 0xffffe000u;
+              const float r = x - __uint_as_float(hi);
+              lo = __float_as_uint(r) & 0xffffe000u;
+              lo2 = kZ3 ? __float_as_uint(r - __uint_as_float(lo)) : 0u;
             };
 #pragma unroll
             for (int cp = 0; cp < 8; cp += 2) {
@@ -861,17 +875,19 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               for (int o = 0; o < 2; ++o) {
                 uint32_t q0, q1, q2, q3;  // records 0-7: columns (4t, 4t+1) in q0, (4t+2, 4t+3) in q1; 8-15: q2, q3
                 ldmatrix_x4(kl + (cp + o) * 32, q0, q1, q2, q3);
-                uint32_t ah[2][4], al[2][4];  // [k-step][fragment register]
-                tf32_split(xa[o].x, ah[0][0], al[0][0]); tf32_split(xb[o].x, ah[0][1], al[0][1]);
-                tf32_split(xa[o].y, ah[0][2], al[0][2]); tf32_split(xb[o].y, ah[0][3], al[0][3]);
-                tf32_split(xa[o].z, ah[1][0], al[1][0]); tf32_split(xb[o].z, ah[1][1], al[1][1]);
-                tf32_split(xa[o].w, ah[1][2], al[1][2]); tf32_split(xb[o].w, ah[1][3], al[1][3]);
+                uint32_t ah[2][4], al[2][4], a3[2][4];  // [k-step][fragment register]
+                tf32_split(xa[o].x, ah[0][0], al[0][0], a3[0][0]); tf32_split(xb[o].x, ah[0][1], al[0][1], a3[0][1]);
+                tf32_split(xa[o].y, ah[0][2], al[0][2], a3[0][2]); tf32_split(xb[o].y, ah[0][3], al[0][3], a3[0][3]);
+                tf32_split(xa[o].z, ah[1][0], al[1][0], a3[1][0]); tf32_split(xb[o].z, ah[1][1], al[1][1], a3[1][1]);
+                tf32_split(xa[o].w, ah[1][2], al[1][2], a3[1][2]); tf32_split(xb[o].w, ah[1][3], al[1][3], a3[1][3]);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                   const uint32_t w0 = kk ? q1 : q0, w1 = kk ? q3 : q2;
+                  if (kZ3) mma_1688_tf32(z0, a3[kk][0], a3[kk][1], a3[kk][2], a3[kk][3], w0 << 16, w0 & 0xffff0000u);
                   mma_1688_tf32(z0, al[kk][0], al[kk][1], al[kk][2], al[kk][3], w0 << 16, w0 & 0xffff0000u);
                   mma_1688_tf32(z0, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], w0 << 16, w0 & 0xffff0000u);
                   if (two) {
+                    if (kZ3) mma_1688_tf32(z1, a3[kk][0], a3[kk][1], a3[kk][2], a3[kk][3], w1 << 16, w1 & 0xffff0000u);
                     mma_1688_tf32(z1, al[kk][0], al[kk][1], al[kk][2], al[kk][3], w1 << 16, w1 & 0xffff0000u);
                     mma_1688_tf32(z1, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], w1 << 16, w1 & 0xffff0000u);
                   }
@@ -996,6 +1012,52 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               bulk_s2g(static_cast<unsigned char *>(a.hp) + (unit * R + kFp4Rows * t + wr0) * kCols * 4,
                        stw + (size_t)wr0 * kCols * 4, (uint32_t)(wrows * kCols * 4), pol_wr);
               bulk_commit();
+            }
+            if (fp4_read) {
+              // the NVFP4 read copy of S': the tile scale from the maximum over the group's four warps (their
+              // rendezvous through an mbarrier with bounded waits), then per row the block scales and codes,
+              // chunk c of a row being its block c (the quad's four lanes share a block)
+              float am = 0.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const float4 pa = va ? *srow(ra, c ^ odd) : f4zero(), pb = vb ? *srow(rb, c ^ odd) : f4zero();
+                am = fmaxf(am, fmaxf(fmaxf(fmaxf(fabsf(pa.x), fabsf(pa.y)), fmaxf(fabsf(pa.z), fabsf(pa.w))),
+                                     fmaxf(fmaxf(fabsf(pb.x), fabsf(pb.y)), fmaxf(fabsf(pb.z), fabsf(pb.w)))));
+              }
+#pragma unroll
+              for (int off = 16; off >= 1; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+              float *gmx = amx + grp * 8 + (crdv & 1) * 4;  // [group][slot][warp of the group]
+              if (lane == 0) gmx[warp & 3] = am;
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&csync[grp]);
+              if (!mbar_wait_or_abort(&csync[grp], (uint32_t)(crdv & 1), abort_flag, ws)) {
+                if (lane == 0) { record_error(a.err, b, RSSM_DEV_TIMEOUT); *abort_flag = 1; }
+                break;
+              }
+              ++crdv;
+              const float g = nvfp4_tile_scale(fmaxf(fmaxf(gmx[0], gmx[1]), fmaxf(gmx[2], gmx[3])));
+              if ((warp & 3) == 0 && lane == 0) a.rg[unit * nrb + t] = g;
+#pragma unroll
+              for (int hr = 0; hr < 2; ++hr) {
+                const bool vrow = hr ? vb : va;
+                const int rr = hr ? rb : ra;
+                const size_t rowq = unit * R + (hr ? rgb : rga);
+                uint2 scw = make_uint2(0u, 0u);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const int cc = c ^ odd;
+                  const float4 v = vrow ? *srow(rr, cc) : f4zero();
+                  float bm = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+                  bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+                  bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+                  float d_b;
+                  const uint32_t sc = nvfp4_block_scale(bm, g, &d_b);
+                  if (cc < 4) scw.x |= sc << (8 * cc); else scw.y |= sc << (8 * (cc - 4));
+                  const uint32_t cw = nvfp4_code4(v, d_b, __frcp_rn(d_b));
+                  if (vrow) *reinterpret_cast<uint16_t *>(a.rq + rowq * (kCols / 2) + cc * 8 + qtr * 2) = (uint16_t)cw;
+                }
+                if (vrow && qtr == 0) *reinterpret_cast<uint2 *>(a.rs + rowq * (kCols / 16)) = scw;
+              }
             }
           } else {
             // ---------------- fold tile: four lanes per row, 32 columns each, chunks rotated by lane
@@ -1213,12 +1275,11 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                 *reinterpret_cast<uint16_t *>(a.rs + (unit * R + rowg) * (kCols / 16) + qtr * 2) =
                     (uint16_t)(sc0 | (sc1 << 8));
                 unsigned char *cd = a.rq + (unit * R + rowg) * (kCols / 2) + qtr * 16;
+                const float rb0 = __frcp_rn(db0), rb1 = __frcp_rn(db1);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                   const int ch = (c + lane) & 7;
-                  const float d_b = ch < 4 ? db0 : db1;
-                  const uint32_t cw = nvfp4_code(sv[c].x, d_b) | (nvfp4_code(sv[c].y, d_b) << 4) |
-                                      (nvfp4_code(sv[c].z, d_b) << 8) | (nvfp4_code(sv[c].w, d_b) << 12);
+                  const uint32_t cw = nvfp4_code4(sv[c], ch < 4 ? db0 : db1, ch < 4 ? rb0 : rb1);
                   *reinterpret_cast<uint16_t *>(cd + ch * 2) = (uint16_t)cw;
                 }
               }
@@ -1253,7 +1314,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
 static bool g_lowprec(int hp_mode, int read_mode) { return hp_mode != RSSM_HP_F32 || read_mode != RSSM_READ_SAME; }
 
 int g_smem_bytes(int R, int L, int tmax, int esz, int nstage, int hp_mode, int read_mode) {
-  const GLayout l = g_layout(R, L, tmax, esz, g_chunked(g_lowprec(hp_mode, read_mode), esz, L));
+  const GLayout l = g_layout(R, L, tmax, esz, g_chunked(hp_mode, read_mode, esz, L));
   return kBarBytesG + 2 * l.tab_bytes + kGBG * l.gb_bytes + nstage * l.stage_bytes;
 }
 
@@ -1282,8 +1343,13 @@ cudaError_t launch_gdn_replay(GArgs a, int esz, cudaStream_t stream) {
                       g_extra_smem_bytes(a.L, esz, a.hp_mode, a.read_mode);
   void (*kern)(GArgs) = nullptr;
   const bool lp = g_lowprec(a.hp_mode, a.read_mode);
-#define RSSM_PICK(TI, NOV, CFV) \
-  if (no == NOV) kern = lp ? gdn_replay_kernel<TI, NOV, true, false> : gdn_replay_kernel<TI, NOV, false, CFV>;
+  // the low-precision instance with the chunked fold serves the fp32 checkpoint with an NVFP4 read copy, at
+  // steps that may fold
+  const bool lpc = lp && g_chunked(a.hp_mode, a.read_mode, esz, a.L) && !a.fold_free;
+#define RSSM_PICK(TI, NOV, CFV)                                                                    \
+  if (no == NOV)                                                                                   \
+    kern = lp ? (CFV && lpc ? gdn_replay_kernel<TI, NOV, true, CFV> : gdn_replay_kernel<TI, NOV, true, false>) \
+              : gdn_replay_kernel<TI, NOV, false, CFV>;
   if (esz == 2) {
     RSSM_PICK(__nv_bfloat16, 1, true) RSSM_PICK(__nv_bfloat16, 2, true) RSSM_PICK(__nv_bfloat16, 4, true)
     RSSM_PICK(__nv_bfloat16, 8, true)

@@ -132,23 +132,6 @@ __device__ __forceinline__ float e4m3_signed_value(uint32_t code) {
 // FP8 checkpoint tile scale from the tile's largest magnitude.
 __device__ __forceinline__ float fp8_tile_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f; }
 
-// E4M3FN round-to-nearest-even of v >= 0, saturating at 448 (value, not code).
-__device__ __forceinline__ float e4m3_round(float v) {
-  if (v >= 448.f) return 448.f;
-  if (v < 0.015625f) return rintf(v * 512.f) * (1.f / 512.f);  // subnormal spacing 2^-9
-  int e;
-  frexpf(v, &e);                                                 // v = m 2^e, m in [0.5, 1)
-  return ldexpf(rintf(ldexpf(v, 4 - e)), e - 4);                 // spacing 2^(floor(log2 v) - 3)
-}
-
-__device__ __forceinline__ uint32_t e4m3_code(float q) {  // q >= 0 on the E4M3 grid
-  if (q < 0.015625f) return (uint32_t)(q * 512.f);
-  int e;
-  frexpf(q, &e);
-  const int E = e - 1 + 7;
-  const uint32_t m = (uint32_t)ldexpf(q, 4 - e) - 8u;
-  return ((uint32_t)E << 3) | m;
-}
 
 // Decoders for the kernels' tile reads, through the hardware pair conversions to f16x2 (every
 // E4M3 and E2M1 value is exactly an f16 value).  The first element sits in the low byte / low
@@ -195,12 +178,18 @@ __device__ __forceinline__ float e2m1_value(uint32_t idx) {
 // NVFP4 tile scale from the tile's largest magnitude.
 __device__ __forceinline__ float nvfp4_tile_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 2688.f) : 1.f; }
 
+// E4M3FN code of v >= 0, rounded to nearest even and saturating at 448 (the hardware conversion; subnormal
+// spacing 2^-9).
+__device__ __forceinline__ uint32_t e4m3_rn_code(float v) {
+  return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
 // Block scale code and the block's dequantisation step d_b = s_b * g.
 __device__ __forceinline__ uint32_t nvfp4_block_scale(float amax_b, float g, float *d_b) {
   const float t = __fmul_rn(6.f, g);
-  const float sb = e4m3_round(__fdiv_rn(amax_b, t));
-  *d_b = __fmul_rn(sb, g);
-  return e4m3_code(sb);
+  const uint32_t code = e4m3_rn_code(__fdiv_rn(amax_b, t));
+  *d_b = __fmul_rn(e4m3_to_float(code), g);
+  return code;
 }
 
 // 4-bit code of x in a block with step d_b (d_b == 0 when the block scale is zero).
@@ -210,18 +199,42 @@ __device__ __forceinline__ uint32_t nvfp4_code(float x, float d_b) {
   return idx | (x < 0.f ? 8u : 0u);
 }
 
+// Four codes of one block (nibble i = element i), the same as nvfp4_code elementwise, without a division per
+// element.  With r = 1/d_b correctly rounded, q' = |x| r lies within 2^-22 (relative) of the correctly rounded
+// quotient q that nvfp4_code rounds, so q'(1 - 2^-19) < q < q'(1 + 2^-19) after rounding; the E2M1 conversion
+// (round to nearest even, saturating at 6: the index rule of e2m1_index) is monotone, so where both ends of the
+// bracket give the same code, q gives it too.  Elements whose bracket straddles a decision threshold, and blocks
+// whose step is too small for a finite reciprocal, take the division.
+__device__ __forceinline__ uint32_t nvfp4_code4(float4 x, float d_b, float r) {
+  if (d_b == 0.f) return 0u;
+  const uint32_t sgn = (x.x < 0.f ? 0x8u : 0u) | (x.y < 0.f ? 0x80u : 0u) | (x.z < 0.f ? 0x800u : 0u) |
+                       (x.w < 0.f ? 0x8000u : 0u);
+  if (d_b >= 0x1p-120f) {
+    const float qx = __fmul_rn(fabsf(x.x), r), qy = __fmul_rn(fabsf(x.y), r);
+    const float qz = __fmul_rn(fabsf(x.z), r), qw = __fmul_rn(fabsf(x.w), r);
+    constexpr float kLo = 1.f - 0x1p-19f, kHi = 1.f + 0x1p-19f;
+    const uint32_t lo = (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(qx * kLo, qy * kLo), __NV_E2M1, cudaRoundNearest) |
+                        ((uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(qz * kLo, qw * kLo), __NV_E2M1, cudaRoundNearest) << 8);
+    const uint32_t hi = (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(qx * kHi, qy * kHi), __NV_E2M1, cudaRoundNearest) |
+                        ((uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(qz * kHi, qw * kHi), __NV_E2M1, cudaRoundNearest) << 8);
+    if (lo == hi) return lo | sgn;
+  }
+  return nvfp4_code(x.x, d_b) | (nvfp4_code(x.y, d_b) << 4) | (nvfp4_code(x.z, d_b) << 8) |
+         (nvfp4_code(x.w, d_b) << 12);
+}
+
 // Two-axis copy: column-group scale code and step k = c * g from the group's largest magnitude.
 __device__ __forceinline__ uint32_t nvfp4d_col_scale(float amax_grp, float g, float *k) {
-  const float c = e4m3_round(__fdiv_rn(amax_grp, __fmul_rn(6.f, g)));
-  *k = __fmul_rn(c, g);
-  return e4m3_code(c);
+  const uint32_t code = e4m3_rn_code(__fdiv_rn(amax_grp, __fmul_rn(6.f, g)));
+  *k = __fmul_rn(e4m3_to_float(code), g);
+  return code;
 }
 
 // Two-axis copy: row-block scale code and block step d_b = s_b * 2^-8 (exact) of the divided values.
 __device__ __forceinline__ uint32_t nvfp4d_block_scale(float amax_b, float *d_b) {
-  const float sb = e4m3_round(__fdiv_rn(amax_b, 0.0234375f));   // 6 * 2^-8
-  *d_b = sb * 0.00390625f;
-  return e4m3_code(sb);
+  const uint32_t code = e4m3_rn_code(__fdiv_rn(amax_b, 0.0234375f));   // 6 * 2^-8
+  *d_b = e4m3_to_float(code) * 0.00390625f;
+  return code;
 }
 
 __device__ __forceinline__ float nvfp4_value(uint32_t code, float d_b) {

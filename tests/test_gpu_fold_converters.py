@@ -9,7 +9,10 @@ tests pin the ones inside the fold kernel, which quantise in registers with a ti
   scales, tile scales) must equal the oracle's NVFP4 quantisation of the exported fp32 checkpoint, bit for bit.
 * fp16-SR and E4M3-SR checkpoints: a companion context with an fp32 checkpoint runs the same fold from the same
   stored values (the low-precision checkpoint, exported and loaded into it at each window boundary), so its
-  exported checkpoint is the fp32 fold result the low-precision context rounded.  The low-precision checkpoint
+  exported checkpoint is the fp32 fold result the low-precision context rounded.  The companion keeps the
+  two-axis read copy: that instance folds with the same sequential row update as the low-precision checkpoints
+  (an fp32 checkpoint read as it is or through the one-axis copy folds in the chunked form, whose rounding
+  differs).  The low-precision checkpoint
   must equal the oracle's stochastic rounding of that result with the Philox words of (sequence x head, epoch
   written, element / 4), bit for bit, and its read copy the oracle's NVFP4 quantisation of it.
 * shared NVFP4: the same, with the shared copy as the state.
@@ -89,7 +92,7 @@ def test_fold_rounding_is_the_oracle_rounding_of_the_fp32_fold(cuda_ok, hp, read
     bf = torch.bfloat16
     S0 = torch.from_numpy(gdn_initial_state(wl)).cuda()
     low = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, 128, 1, wl.window, 0, bf, hp, read, SEED)
-    ref = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, 128, 1, wl.window, 0, bf, "f32", "nvfp4", SEED)
+    ref = ReplaySSM("gdn", wl.batch, wl.nheads, wl.dv, 128, 1, wl.window, 0, bf, "f32", "nvfp4d", SEED)
     low.load_checkpoint(S0)
     units = np.arange(wl.batch)[:, None] * wl.nheads + np.arange(wl.nheads)[None, :]
     n = wl.dv * 128
