@@ -952,6 +952,7 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
             const uint32_t mk1 = (2 * qtr + 8 < m ? 0xFFFFu : 0u) | (2 * qtr + 9 < m ? 0xFFFF0000u : 0u);
             const unsigned char *kt = kb + (size_t)min((lane & 7) + 8 * ((lane >> 3) & 1), m - 1) * kpb + (lane >> 4) * 16;
             // S is read again from the stage chunk pair by chunk pair, and S' goes back to the same place
+            float smax = 0.f;  // the largest magnitude of the lane's rows of S' (NVFP4 copy: the tile scale)
 #pragma unroll
             for (int cp = 0; cp < 8; cp += 2) {
               float4 xa[2], xb[2];
@@ -971,6 +972,10 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
                   for (int p = 2; p >= 0; --p) mma_16816(d, wp[p][0], wp[p][1], wp[p][2], wp[p][3], b0, b1);
                   if (o == 0) { xa[o2].x = d[0]; xa[o2].y = d[1]; xb[o2].x = d[2]; xb[o2].y = d[3]; }
                   else        { xa[o2].z = d[0]; xa[o2].w = d[1]; xb[o2].z = d[2]; xb[o2].w = d[3]; }
+                }
+                if (fp4_read) {
+                  if (va) smax = fmaxf(smax, fmaxf(fmaxf(fabsf(xa[o2].x), fabsf(xa[o2].y)), fmaxf(fabsf(xa[o2].z), fabsf(xa[o2].w))));
+                  if (vb) smax = fmaxf(smax, fmaxf(fmaxf(fabsf(xb[o2].x), fabsf(xb[o2].y)), fmaxf(fabsf(xb[o2].z), fabsf(xb[o2].w))));
                 }
               }
               const int c0 = cp + odd, c1 = cp + 1 - odd;
@@ -1017,17 +1022,11 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               // the NVFP4 read copy of S': the tile scale from the maximum over the group's four warps (their
               // rendezvous through an mbarrier with bounded waits), then per row the block scales and codes,
               // chunk c of a row being its block c (the quad's four lanes share a block)
-              float am = 0.f;
+              float wmx = smax;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const float4 pa = va ? *srow(ra, c ^ odd) : f4zero(), pb = vb ? *srow(rb, c ^ odd) : f4zero();
-                am = fmaxf(am, fmaxf(fmaxf(fmaxf(fabsf(pa.x), fabsf(pa.y)), fmaxf(fabsf(pa.z), fabsf(pa.w))),
-                                     fmaxf(fmaxf(fabsf(pb.x), fabsf(pb.y)), fmaxf(fabsf(pb.z), fabsf(pb.w)))));
-              }
-#pragma unroll
-              for (int off = 16; off >= 1; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+              for (int off = 16; off >= 1; off >>= 1) wmx = fmaxf(wmx, __shfl_xor_sync(0xffffffffu, wmx, off));
               float *gmx = amx + grp * 8 + (crdv & 1) * 4;  // [group][slot][warp of the group]
-              if (lane == 0) gmx[warp & 3] = am;
+              if (lane == 0) gmx[warp & 3] = wmx;
               __syncwarp();
               if (lane == 0) mbar_arrive(&csync[grp]);
               if (!mbar_wait_or_abort(&csync[grp], (uint32_t)(crdv & 1), abort_flag, ws)) {
@@ -1037,26 +1036,58 @@ __global__ void __launch_bounds__(kGdnThreads, 1) gdn_replay_kernel(GArgs a) {
               ++crdv;
               const float g = nvfp4_tile_scale(fmaxf(fmaxf(gmx[0], gmx[1]), fmaxf(gmx[2], gmx[3])));
               if ((warp & 3) == 0 && lane == 0) a.rg[unit * nrb + t] = g;
+              // the quad's 16 (row, block) pairs p = 8 hr + c (row ra or rb, chunk slot c, block c ^ odd): their
+              // maxima by a transposing reduction over the quad, after which lane qtr holds the pairs
+              // 8 b0 + 4 b1 + k (b0 = qtr & 1, b1 = qtr >> 1) and computes their scales once; the steps and
+              // their reciprocals then travel back to every lane of the quad
+              const bool b0 = qtr & 1, b1 = (qtr >> 1) & 1;
+              float bmx[16];
 #pragma unroll
-              for (int hr = 0; hr < 2; ++hr) {
-                const bool vrow = hr ? vb : va;
-                const int rr = hr ? rb : ra;
-                const size_t rowq = unit * R + (hr ? rgb : rga);
-                uint2 scw = make_uint2(0u, 0u);
+              for (int c = 0; c < 8; ++c) {
+                const float4 pa = va ? *srow(ra, c ^ odd) : f4zero(), pb = vb ? *srow(rb, c ^ odd) : f4zero();
+                bmx[c] = fmaxf(fmaxf(fabsf(pa.x), fabsf(pa.y)), fmaxf(fabsf(pa.z), fabsf(pa.w)));
+                bmx[8 + c] = fmaxf(fmaxf(fabsf(pb.x), fabsf(pb.y)), fmaxf(fabsf(pb.z), fabsf(pb.w)));
+              }
+              float w8[8], w4[4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                  const int cc = c ^ odd;
-                  const float4 v = vrow ? *srow(rr, cc) : f4zero();
-                  float bm = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-                  bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-                  bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-                  float d_b;
-                  const uint32_t sc = nvfp4_block_scale(bm, g, &d_b);
-                  if (cc < 4) scw.x |= sc << (8 * cc); else scw.y |= sc << (8 * (cc - 4));
-                  const uint32_t cw = nvfp4_code4(v, d_b, __frcp_rn(d_b));
-                  if (vrow) *reinterpret_cast<uint16_t *>(a.rq + rowq * (kCols / 2) + cc * 8 + qtr * 2) = (uint16_t)cw;
+              for (int k = 0; k < 8; ++k)
+                w8[k] = fmaxf(b0 ? bmx[k + 8] : bmx[k], __shfl_xor_sync(0xffffffffu, b0 ? bmx[k] : bmx[k + 8], 1));
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                w4[k] = fmaxf(b1 ? w8[k + 4] : w8[k], __shfl_xor_sync(0xffffffffu, b1 ? w8[k] : w8[k + 4], 2));
+              float dq[4], rq[4];
+              uint32_t scw = 0u;
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                scw |= nvfp4_block_scale(w4[k], g, &dq[k]) << (8 * (k ^ odd));
+                rq[k] = __frcp_rn(dq[k]);
+              }
+              if (b0 ? vb : va)  // row rb (b0) or ra, blocks 4 b1 .. 4 b1 + 3
+                *reinterpret_cast<uint32_t *>(a.rs + (unit * R + (b0 ? rgb : rga)) * (kCols / 16) + 4 * b1) = scw;
+              float d8[8], r8[8], d16[16], r16[16];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float od = __shfl_xor_sync(0xffffffffu, dq[k], 2), orr = __shfl_xor_sync(0xffffffffu, rq[k], 2);
+                d8[k] = b1 ? od : dq[k]; d8[k + 4] = b1 ? dq[k] : od;
+                r8[k] = b1 ? orr : rq[k]; r8[k + 4] = b1 ? rq[k] : orr;
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float od = __shfl_xor_sync(0xffffffffu, d8[k], 1), orr = __shfl_xor_sync(0xffffffffu, r8[k], 1);
+                d16[k] = b0 ? od : d8[k]; d16[k + 8] = b0 ? d8[k] : od;
+                r16[k] = b0 ? orr : r8[k]; r16[k + 8] = b0 ? r8[k] : orr;
+              }
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int cc = c ^ odd;
+                if (va) {
+                  const uint32_t cw = nvfp4_code4(*srow(ra, cc), d16[c], r16[c]);
+                  *reinterpret_cast<uint16_t *>(a.rq + (unit * R + rga) * (kCols / 2) + cc * 8 + qtr * 2) = (uint16_t)cw;
                 }
-                if (vrow && qtr == 0) *reinterpret_cast<uint2 *>(a.rs + rowq * (kCols / 16)) = scw;
+                if (vb) {
+                  const uint32_t cw = nvfp4_code4(*srow(rb, cc), d16[8 + c], r16[8 + c]);
+                  *reinterpret_cast<uint16_t *>(a.rq + (unit * R + rgb) * (kCols / 2) + cc * 8 + qtr * 2) = (uint16_t)cw;
+                }
               }
             }
           } else {

@@ -199,6 +199,12 @@ __device__ __forceinline__ uint32_t nvfp4_code(float x, float d_b) {
   return idx | (x < 0.f ? 8u : 0u);
 }
 
+// The division for the four codes, out of line: kernels call it only for the rare element near a decision
+// threshold, and keep their unrolled code loops compact.
+static __device__ __noinline__ uint32_t nvfp4_code4_div(float4 x, float d_b) {
+  return nvfp4_code(x.x, d_b) | (nvfp4_code(x.y, d_b) << 4) | (nvfp4_code(x.z, d_b) << 8) | (nvfp4_code(x.w, d_b) << 12);
+}
+
 // Four codes of one block (nibble i = element i), the same as nvfp4_code elementwise, without a division per
 // element.  With r = 1/d_b correctly rounded, q' = |x| r lies within 2^-22 (relative) of the correctly rounded
 // quotient q that nvfp4_code rounds, so q'(1 - 2^-19) < q < q'(1 + 2^-19) after rounding; the E2M1 conversion
@@ -219,8 +225,7 @@ __device__ __forceinline__ uint32_t nvfp4_code4(float4 x, float d_b, float r) {
                         ((uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(qz * kHi, qw * kHi), __NV_E2M1, cudaRoundNearest) << 8);
     if (lo == hi) return lo | sgn;
   }
-  return nvfp4_code(x.x, d_b) | (nvfp4_code(x.y, d_b) << 4) | (nvfp4_code(x.z, d_b) << 8) |
-         (nvfp4_code(x.w, d_b) << 12);
+  return nvfp4_code4_div(x, d_b);
 }
 
 // Two-axis copy: column-group scale code and step k = c * g from the group's largest magnitude.

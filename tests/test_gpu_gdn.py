@@ -180,7 +180,7 @@ def test_load_converters_bit_exact(cuda_ok, hp, read):
 #   outputs above 1e-4 apply.
 TOL_FLIP = 1e-2
 FLIP_FRACTION = 0.02
-FLIP_CODE_RATE = 1e-4
+FLIP_CODE_RATE = 2e-5   # measured: at most 3 of 1.6 M codes (1.8e-6), small, full-batch and verify cases
 TOL_CKPT_G = 1e-5   # tile scales, relative: the bound of the checkpoint after folds
 # With stochastic rounding the oracle's trajectory is one sample among many: one rounding decision taken
 # differently changes the checkpoint by one fp16 (or E4M3) step, and the trajectories then differ within the
